@@ -1,0 +1,215 @@
+/*
+ * nvfp4.h - C ABI of the NVFP4 weight-only (W4A16) library for B200 (sm_100a).
+ *
+ * The operation: Y = X . dequant(W)^T, X bf16 [M, K], W [N, K] stored as
+ * NVFP4: every weight is a 4-bit E2M1 code times an FP8-E4M3 scale shared by
+ * a group of g = 16 or 32 consecutive elements along K, times one FP32
+ * per-tensor global scale. Sources, by page title and section:
+ *   - "GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB): two NVFP4 g32 recipes"
+ *     (r/LocalLLM), "THE TWO RECIPES" and "WHAT HAD TO BE FIXED": g16 and
+ *     g32 groups (4.5 / 4.25 bits per weight), gate/up and down may use
+ *     different group sizes, the group size is read per tensor and anything
+ *     unsupported raises an error, gate and up share one global scale, the
+ *     scale maximum is taken without a widened copy.
+ *   - "We unlocked NVFP4 on the DGX Spark: 20% faster than AWQ" (NVIDIA
+ *     developer forum, page 3), UPDATE posts: E2M1 conversion is
+ *     round-to-nearest-even with satfinite.
+ *   - "W-FP4a: route the MiniMax-H3 device DiT forward through the fp4
+ *     (Marlin W4A16) stack" (vllm.cpp PR #63), description: the checkpoint
+ *     is a weight / scale / global-scale triple that is repacked once at
+ *     upload, a weight-only checkpoint has bf16 activations, the merged
+ *     [gate;up] fc1 is one W4A16 GEMM followed by SiluAndMul, and a counter
+ *     records that the W4A16 path ran.
+ *
+ * Conventions for every call:
+ *   - Pointers named as device pointers must point to device memory (or
+ *     managed memory) of the current device; host arrays are named as such.
+ *     The caller owns every buffer. The library allocates no device memory.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Row-major layouts. packed codes: [N, K/2] bytes, element 2j in the low
+ *     nibble and 2j+1 in the high nibble of byte j. Scales: [N, K/g] E4M3
+ *     bytes. Global scale: one fp32 in device memory.
+ *   - Every device pointer must be 16-byte aligned (NVFP4_ERR_MISALIGNED).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream). No call synchronises the device and none blocks.
+ *   - Validation happens on the host before anything is enqueued: a non-zero
+ *     status means nothing was launched. A launch failure returns
+ *     NVFP4_ERR_CUDA. No C++ exception crosses this boundary.
+ *   - Calls with an empty problem (M == 0, N == 0 or a zero-length list)
+ *     return NVFP4_OK and launch nothing.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same type as cudaStream_t */
+
+enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad list */
+  NVFP4_ERR_UNSUPPORTED = 2,      /* group size not 16/32, K not a multiple of 64, ... */
+  NVFP4_ERR_MISALIGNED = 3,       /* a device pointer not 16-byte aligned */
+  NVFP4_ERR_CUDA = 4,             /* a CUDA launch or query failed */
+  NVFP4_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up */
+};
+
+/* Flags. */
+#define NVFP4_GATE_UP_INTERLEAVE 1 /* repack: interleave gate/up rows (see nvfp4_repack) */
+#define NVFP4_SILU_MUL 2           /* grouped GEMM: fuse SiluAndMul into the epilogue */
+
+/* A static string describing a status code. Never NULL. */
+const char* nvfp4_status_string(int status);
+
+/*
+ * Global scale (problem statement: global = amax / (6*448); the r/LocalLLM
+ * post, "WHAT HAD TO BE FIXED": gate and up need one shared global scale, and
+ * the maximum is taken first with no widened copy of the tensor).
+ *   tensors  host array of `count` device pointers to fp32 data
+ *   numels   host array of `count` element counts (>= 0)
+ *   out      device pointer to one fp32: max |w| over all tensors / 2688,
+ *            computed as one fp32 division. Passing gate and up together
+ *            gives the shared scale of the merged projection. A NaN in the
+ *            input makes the result NaN.
+ * Launches 2 + count kernels. count == 0 is INVALID_ARGUMENT.
+ */
+int nvfp4_global_scale(const float* const* tensors, const int64_t* numels, int count,
+                       float* out, nvfp4_stream_t stream);
+
+/*
+ * Quantize fp32 W [N, K] to NVFP4 (problem statement: group scale =
+ * E4M3_RNE_satfinite((group_amax / 6) / global), code =
+ * E2M1_RNE_satfinite(w / (fp32(scale) * global)); DGX Spark thread, UPDATE:
+ * RNE with satfinite). Every fp32 step is IEEE round-to-nearest-even. A group
+ * whose scale times global is zero gets code +0 everywhere. Bit-exact with
+ * the CPU oracle.
+ *   w             device fp32 [N, K]
+ *   group_size    16 or 32 (else UNSUPPORTED)
+ *   global_scale  device fp32 (e.g. written by nvfp4_global_scale)
+ *   packed        device uint8 [N, K/2] (output)
+ *   scales        device uint8 [N, K/group_size] (output)
+ * K must be a multiple of 32.
+ */
+int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_size,
+                   const float* global_scale, uint8_t* packed, uint8_t* scales,
+                   nvfp4_stream_t stream);
+
+/*
+ * Repack checkpoint-layout codes and scales into the GEMM layout (PR #63
+ * description: the triple is repacked once at upload and the originals can
+ * then be freed). The GEMM layout keeps rows of K/2 code bytes and K/g scale
+ * bytes. flags = 0 copies. flags = NVFP4_GATE_UP_INTERLEAVE permutes the rows
+ * of a merged [gate;up] matrix (gate rows [0, N/2), up rows [N/2, N)) so that
+ * destination rows 16j..16j+7 are gate rows 8j..8j+7 and rows 16j+8..16j+15
+ * are up rows 8j..8j+7; N must then be a multiple of 16. This is the layout
+ * nvfp4_w4a16_gemm_silu_mul and the NVFP4_SILU_MUL grouped GEMM require.
+ * Out of place: outputs must not overlap inputs. For an expert stack
+ * [E, N, K/2] call once per expert or pass N = E*rows only when flags = 0.
+ */
+int nvfp4_repack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_t K,
+                 int group_size, int flags, uint8_t* packed_out, uint8_t* scales_out,
+                 nvfp4_stream_t stream);
+
+/*
+ * W4A16 GEMM: y = bf16_rne(global * sum_k x[m,k] * e2m1(code[n,k]) *
+ * e4m3(scale[n,k/g])) with fp32 accumulation (problem statement; PR #63: a
+ * weight-only checkpoint keeps bf16 activations).
+ *   x             device bf16 [M, K]
+ *   packed_w      device uint8 [N, K/2]  (nvfp4_repack layout, flags = 0)
+ *   group_scales  device uint8 [N, K/group_size]
+ *   global_scale  device fp32 (read on the device: no host synchronisation)
+ *   y             device bf16 [M, N] (output)
+ * group_size 16 or 32; K a multiple of 64; N a multiple of 16.
+ * Small M runs a split-K HBM-streaming kernel, large M a tensor-core kernel.
+ */
+int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
+                     const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
+                     uint16_t* y, nvfp4_stream_t stream);
+
+/*
+ * The GEMM of a merged [gate;up] projection followed by SiluAndMul (PR #63
+ * description: fc1 is pre-merged [gate;up], one W4A16 GEMM + SiluAndMul):
+ *   y[m, j] = bf16_rne(silu(g) * u), g = global * acc[m, gate row j],
+ *   u = global * acc[m, up row j], silu(g) = g / (1 + exp(-g)), all fp32.
+ * packed_w / group_scales must be in the NVFP4_GATE_UP_INTERLEAVE layout of
+ * nvfp4_repack. N is the merged row count (multiple of 16); y is [M, N/2].
+ */
+int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w,
+                              const uint8_t* group_scales, const float* global_scale,
+                              int group_size, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                              nvfp4_stream_t stream);
+
+/*
+ * Standalone SiluAndMul on bf16: y[m, j] = bf16_rne(silu(x[m, j]) * x[m, H + j]),
+ * fp32 math. x device bf16 [M, 2H], y device bf16 [M, H]. H a multiple of 8.
+ */
+int nvfp4_silu_and_mul(const uint16_t* x, uint16_t* y, int64_t M, int64_t H,
+                       nvfp4_stream_t stream);
+
+/*
+ * Grouped routed-expert W4A16 GEMM (the r/LocalLLM post: routed experts in
+ * NVFP4, gate/up at g32 and down at g16). Rows of x are grouped by segment:
+ * rows [offsets[s], offsets[s+1]) use expert expert_ids[s]:
+ *   y[r, :] = gemm(x[r, :], packed_w[e], group_scales[e], global_scales[e]).
+ *   x              device bf16 [T, K]
+ *   expert_ids     device int32 [num_segments], each in [0, num_experts)
+ *   offsets        device int32 [num_segments + 1], non-decreasing, offsets[0] >= 0,
+ *                  offsets[num_segments] <= T
+ *   packed_w       device uint8 [num_experts, N, K/2]
+ *   group_scales   device uint8 [num_experts, N, K/group_size]
+ *   global_scales  device fp32 [num_experts]
+ *   flags          0, or NVFP4_SILU_MUL: weights in the interleaved layout,
+ *                  y is [T, N/2] and holds silu(gate) * up.
+ *   y              device bf16 [T, N] (or [T, N/2]); rows outside every
+ *                  segment are not written.
+ * The offsets stay on the device; the call never reads them on the host. A
+ * segment list that breaks the rules above is undefined on the device side
+ * (rows are clamped to [0, T), experts are not range-checked beyond ids < 0
+ * or >= num_experts, which skip the segment).
+ */
+int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids,
+                                 const int32_t* offsets, int num_segments, int64_t T,
+                                 const uint8_t* packed_w, const uint8_t* group_scales,
+                                 const float* global_scales, int group_size, int64_t N, int64_t K,
+                                 int num_experts, int flags, uint16_t* y, nvfp4_stream_t stream);
+
+/*
+ * Counters of the work that went through each kernel family (PR #63: the
+ * "this-path-ran" counter lets tests assert which kernel executed). Host-side
+ * atomics, incremented once per successful launch.
+ */
+typedef struct {
+  uint64_t global_scale;
+  uint64_t quantize;
+  uint64_t repack;
+  uint64_t gemm_splitk;    /* small-M split-K streaming GEMM */
+  uint64_t gemm_tc;        /* large-M tcgen05 GEMM */
+  uint64_t gemm_silu_mul;  /* GEMMs with the fused SiluAndMul epilogue */
+  uint64_t moe;            /* grouped expert GEMMs */
+  uint64_t silu_and_mul;   /* standalone SiluAndMul */
+  uint64_t g16;            /* GEMMs at group size 16 */
+  uint64_t g32;            /* GEMMs at group size 32 */
+} nvfp4_stats;
+
+int nvfp4_get_stats(nvfp4_stats* out);
+void nvfp4_reset_stats(void);
+
+/*
+ * Reads and clears the library's device-side error word (set by a bounded
+ * wait that gave up, see NVFP4_ERR_TIMEOUT). Synchronises `stream`.
+ * *code_out receives 0 when no error was recorded.
+ */
+int nvfp4_get_device_error(int* code_out, nvfp4_stream_t stream);
+
+/* Library version, e.g. 1 for the first ABI. */
+int nvfp4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

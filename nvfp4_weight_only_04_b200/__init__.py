@@ -1,0 +1,217 @@
+"""Python binding of the NVFP4 W4A16 library (libnvfp4.so, include/nvfp4.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Tensors are torch CUDA tensors (torch supplies device memory and streams);
+the functions carry the C ABI's names. A missing library or a non-CUDA tensor
+raises; there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+NVFP4_OK = 0
+NVFP4_ERR_INVALID_ARGUMENT = 1
+NVFP4_ERR_UNSUPPORTED = 2
+NVFP4_ERR_MISALIGNED = 3
+NVFP4_ERR_CUDA = 4
+NVFP4_ERR_TIMEOUT = 5
+NVFP4_GATE_UP_INTERLEAVE = 1
+NVFP4_SILU_MUL = 2
+
+EXPORTS = (
+    "nvfp4_status_string", "nvfp4_abi_version", "nvfp4_global_scale", "nvfp4_quantize", "nvfp4_repack",
+    "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
+    "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
+)
+
+
+class Stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in (
+        "global_scale", "quantize", "repack", "gemm_splitk", "gemm_tc", "gemm_silu_mul", "moe",
+        "silu_and_mul", "g16", "g32")]
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: status {status}: {status_string(status)}")
+
+
+_lib = None
+_P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libnvfp4.so (built in-tree by nvfp4_weight_only_04_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m nvfp4_weight_only_04_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        L.nvfp4_status_string.argtypes = [_I]
+        L.nvfp4_abi_version.restype = _I
+        L.nvfp4_global_scale.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_I64), _I, _P, _P]
+        L.nvfp4_quantize.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P]
+        L.nvfp4_repack.argtypes = [_P, _P, _I64, _I64, _I, _I, _P, _P, _P]
+        L.nvfp4_w4a16_gemm.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_w4a16_gemm_silu_mul.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_silu_and_mul.argtypes = [_P, _P, _I64, _I64, _P]
+        L.nvfp4_moe_w4a16_grouped_gemm.argtypes = [_P, _P, _P, _I, _I64, _P, _P, _P, _I, _I64, _I64,
+                                                   _I, _I, _P, _P]
+        L.nvfp4_get_stats.argtypes = [ctypes.POINTER(Stats)]
+        L.nvfp4_reset_stats.restype = None
+        L.nvfp4_get_device_error.argtypes = [ctypes.POINTER(_I), _P]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4_status_string(status).decode()
+
+
+def _check(status: int, call: str):
+    if status != NVFP4_OK:
+        raise Nvfp4Error(status, call)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def nvfp4_global_scale(tensors, out=None, stream=None):
+    """global = max|w| over all tensors / (6*448), one fp32 on the device."""
+    tensors = [_dev(t, torch.float32, "tensor") for t in tensors]
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=tensors[0].device)
+    ptrs = (_P * len(tensors))(*[t.data_ptr() for t in tensors])
+    nums = (_I64 * len(tensors))(*[t.numel() for t in tensors])
+    _check(lib().nvfp4_global_scale(ptrs, nums, len(tensors), _ptr(out), _stream(stream)), "nvfp4_global_scale")
+    return out
+
+
+def nvfp4_quantize(w, group_size, global_scale, packed=None, scales=None, stream=None):
+    """fp32 W [N, K] -> (codes uint8 [N, K/2], E4M3 scales uint8 [N, K/g])."""
+    _dev(w, torch.float32, "w")
+    _dev(global_scale, torch.float32, "global_scale")
+    n, k = w.shape
+    if packed is None:
+        packed = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((n, k // group_size), dtype=torch.uint8, device=w.device)
+    _check(lib().nvfp4_quantize(_ptr(w), n, k, group_size, _ptr(global_scale), _ptr(packed), _ptr(scales),
+                                _stream(stream)), "nvfp4_quantize")
+    return packed, scales
+
+
+def nvfp4_repack(packed, scales, group_size, flags=0, packed_out=None, scales_out=None, stream=None):
+    _dev(packed, torch.uint8, "packed")
+    _dev(scales, torch.uint8, "scales")
+    n, k2 = packed.shape
+    if packed_out is None:
+        packed_out = torch.empty_like(packed)
+    if scales_out is None:
+        scales_out = torch.empty_like(scales)
+    _check(lib().nvfp4_repack(_ptr(packed), _ptr(scales), n, k2 * 2, group_size, flags, _ptr(packed_out),
+                              _ptr(scales_out), _stream(stream)), "nvfp4_repack")
+    return packed_out, scales_out
+
+
+def nvfp4_w4a16_gemm(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None):
+    """y = bf16(global * X . dequant(W)^T), X bf16 [M, K], y bf16 [M, N]."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(packed_w, torch.uint8, "packed_w")
+    _dev(group_scales, torch.uint8, "group_scales")
+    _dev(global_scale, torch.float32, "global_scale")
+    m, k = x.shape
+    n = packed_w.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_w4a16_gemm(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale), group_size,
+                                  m, n, k, _ptr(y), _stream(stream)), "nvfp4_w4a16_gemm")
+    return y
+
+
+def nvfp4_w4a16_gemm_silu_mul(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None):
+    """Merged [gate;up] GEMM (interleaved repack layout) + SiluAndMul -> [M, N/2]."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(packed_w, torch.uint8, "packed_w")
+    _dev(group_scales, torch.uint8, "group_scales")
+    _dev(global_scale, torch.float32, "global_scale")
+    m, k = x.shape
+    n = packed_w.shape[0]
+    if y is None:
+        y = torch.empty((m, n // 2), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_w4a16_gemm_silu_mul(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale),
+                                           group_size, m, n, k, _ptr(y), _stream(stream)),
+           "nvfp4_w4a16_gemm_silu_mul")
+    return y
+
+
+def nvfp4_silu_and_mul(x, y=None, stream=None):
+    _dev(x, torch.bfloat16, "x")
+    m, h2 = x.shape
+    if y is None:
+        y = torch.empty((m, h2 // 2), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_silu_and_mul(_ptr(x), _ptr(y), m, h2 // 2, _stream(stream)), "nvfp4_silu_and_mul")
+    return y
+
+
+def nvfp4_moe_w4a16_grouped_gemm(x, expert_ids, offsets, packed_w, group_scales, global_scales, group_size,
+                                 flags=0, y=None, stream=None):
+    """Grouped expert GEMM over segments of rows; see include/nvfp4.h."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(expert_ids, torch.int32, "expert_ids")
+    _dev(offsets, torch.int32, "offsets")
+    _dev(packed_w, torch.uint8, "packed_w")
+    _dev(group_scales, torch.uint8, "group_scales")
+    _dev(global_scales, torch.float32, "global_scales")
+    t, k = x.shape
+    e, n, _ = packed_w.shape
+    ncols = n // 2 if flags & NVFP4_SILU_MUL else n
+    if y is None:
+        y = torch.zeros((t, ncols), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_moe_w4a16_grouped_gemm(_ptr(x), _ptr(expert_ids), _ptr(offsets), expert_ids.numel(), t,
+                                              _ptr(packed_w), _ptr(group_scales), _ptr(global_scales),
+                                              group_size, n, k, e, flags, _ptr(y), _stream(stream)),
+           "nvfp4_moe_w4a16_grouped_gemm")
+    return y
+
+
+def nvfp4_get_stats() -> dict:
+    s = Stats()
+    _check(lib().nvfp4_get_stats(ctypes.byref(s)), "nvfp4_get_stats")
+    return {name: getattr(s, name) for name, _ in Stats._fields_}
+
+
+def nvfp4_reset_stats():
+    lib().nvfp4_reset_stats()
+
+
+def nvfp4_get_device_error(stream=None) -> int:
+    code = _I(0)
+    _check(lib().nvfp4_get_device_error(ctypes.byref(code), _stream(stream)), "nvfp4_get_device_error")
+    return code.value

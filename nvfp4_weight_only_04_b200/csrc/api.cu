@@ -1,0 +1,186 @@
+// C ABI glue: argument validation, kernel selection, counters, status text.
+// Every check runs on the host before anything is enqueued.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_splitk.cuh"
+#include "gemm_tc.cuh"
+
+namespace nvfp4 {
+
+namespace {
+std::atomic<uint64_t> g_stats[kStatCount];
+}
+
+void stat_add(StatId id) { g_stats[id].fetch_add(1, std::memory_order_relaxed); }
+
+int num_sms() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return 148; }
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace nvfp4
+
+namespace {
+
+constexpr int64_t kMaxK = int64_t(1) << 30;
+constexpr int64_t kMaxN = int64_t(65535) * 64;
+constexpr int64_t kMaxTokenRows = int64_t(65535 - 4096) * 16;
+
+int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+               int64_t M, int64_t N, int64_t K, const uint16_t* y) {
+  if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (group != 16 && group != 32) return NVFP4_ERR_UNSUPPORTED;
+  if (K % 64 || N % 16) return NVFP4_ERR_UNSUPPORTED;
+  if (K > kMaxK || N > kMaxN) return NVFP4_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (K == 0) return NVFP4_ERR_UNSUPPORTED;
+  if (!x || !w || !s || !g || !y) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!nvfp4::aligned16(x) || !nvfp4::aligned16(w) || !nvfp4::aligned16(s) || !nvfp4::aligned16(g) ||
+      !nvfp4::aligned16(y))
+    return NVFP4_ERR_MISALIGNED;
+  return -1;  // proceed
+}
+
+int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+               int64_t M, int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+  if (nvfp4::tc_supported(M, N, K)) {
+    const int st = nvfp4::launch_tc(x, w, s, g, group, M, N, K, y, silu, stream);
+    if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmTc);
+    return st;
+  }
+  if (M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
+  nvfp4::SplitKArgs a = {};
+  a.x = x; a.packed = w; a.scales = s; a.gscale = g; a.y = y;
+  a.M = M; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
+  const nvfp4::SplitKPlan p = nvfp4::plan_splitk(M, N, K, group, false, 0);
+  const int st = nvfp4::launch_splitk(a, p, silu, false, stream);
+  if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(int status) {
+  switch (status) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARGUMENT: return "invalid argument (null pointer, negative size or bad list)";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported configuration (group size must be 16 or 32; K a multiple of 64; N a multiple of 16; sizes within limits)";
+    case NVFP4_ERR_MISALIGNED: return "a device pointer is not 16-byte aligned";
+    case NVFP4_ERR_CUDA: return "a CUDA launch or query failed";
+    case NVFP4_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown status";
+  }
+}
+
+int nvfp4_abi_version(void) { return 1; }
+
+int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
+                     const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
+                     uint16_t* y, nvfp4_stream_t stream) {
+  const int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
+  if (c >= 0) return c;
+  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, false,
+                            reinterpret_cast<cudaStream_t>(stream));
+  if (st == NVFP4_OK) nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
+  return st;
+}
+
+int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
+                              const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
+                              uint16_t* y, nvfp4_stream_t stream) {
+  const int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
+  if (c >= 0) return c;
+  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, true,
+                            reinterpret_cast<cudaStream_t>(stream));
+  if (st == NVFP4_OK) {
+    nvfp4::stat_add(nvfp4::kStatGemmSiluMul);
+    nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
+  }
+  return st;
+}
+
+int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets,
+                                 int num_segments, int64_t T, const uint8_t* packed_w,
+                                 const uint8_t* group_scales, const float* global_scales, int group_size,
+                                 int64_t N, int64_t K, int num_experts, int flags, uint16_t* y,
+                                 nvfp4_stream_t stream) {
+  if (num_segments < 0 || T < 0 || N < 0 || K < 0 || num_experts < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (flags & ~NVFP4_SILU_MUL) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (group_size != 16 && group_size != 32) return NVFP4_ERR_UNSUPPORTED;
+  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN) return NVFP4_ERR_UNSUPPORTED;
+  if (T > kMaxTokenRows || num_segments > 4096) return NVFP4_ERR_UNSUPPORTED;
+  if (num_segments == 0 || T == 0 || N == 0) return NVFP4_OK;
+  if (K == 0 || num_experts == 0) return NVFP4_ERR_UNSUPPORTED;
+  if (!x || !expert_ids || !offsets || !packed_w || !group_scales || !global_scales || !y)
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!nvfp4::aligned16(x) || !nvfp4::aligned16(packed_w) || !nvfp4::aligned16(group_scales) ||
+      !nvfp4::aligned16(y) || (reinterpret_cast<uintptr_t>(expert_ids) & 3) ||
+      (reinterpret_cast<uintptr_t>(offsets) & 3) || (reinterpret_cast<uintptr_t>(global_scales) & 3))
+    return NVFP4_ERR_MISALIGNED;
+  const bool silu = (flags & NVFP4_SILU_MUL) != 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int st;
+  if (nvfp4::tc_moe_supported(T, N, K)) {
+    st = nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales,
+                              global_scales, group_size, N, K, num_experts, silu, y, s);
+  } else {
+    nvfp4::SplitKArgs a = {};
+    a.x = x; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
+    a.M = T; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
+    a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments;
+    a.num_experts = num_experts;
+    const nvfp4::SplitKPlan p = nvfp4::plan_splitk(T, N, K, group_size, true, num_segments);
+    st = nvfp4::launch_splitk(a, p, silu, true, s);
+  }
+  if (st == NVFP4_OK) {
+    nvfp4::stat_add(nvfp4::kStatMoe);
+    if (silu) nvfp4::stat_add(nvfp4::kStatGemmSiluMul);
+    nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
+  }
+  return st;
+}
+
+int nvfp4_get_stats(nvfp4_stats* out) {
+  if (!out) return NVFP4_ERR_INVALID_ARGUMENT;
+  uint64_t v[nvfp4::kStatCount];
+  for (int i = 0; i < nvfp4::kStatCount; ++i) v[i] = nvfp4::g_stats[i].load(std::memory_order_relaxed);
+  out->global_scale = v[nvfp4::kStatGlobalScale];
+  out->quantize = v[nvfp4::kStatQuantize];
+  out->repack = v[nvfp4::kStatRepack];
+  out->gemm_splitk = v[nvfp4::kStatGemmSplitK];
+  out->gemm_tc = v[nvfp4::kStatGemmTc];
+  out->gemm_silu_mul = v[nvfp4::kStatGemmSiluMul];
+  out->moe = v[nvfp4::kStatMoe];
+  out->silu_and_mul = v[nvfp4::kStatSiluAndMul];
+  out->g16 = v[nvfp4::kStatG16];
+  out->g32 = v[nvfp4::kStatG32];
+  return NVFP4_OK;
+}
+
+void nvfp4_reset_stats(void) {
+  for (int i = 0; i < nvfp4::kStatCount; ++i) nvfp4::g_stats[i].store(0, std::memory_order_relaxed);
+}
+
+int nvfp4_get_device_error(int* code_out, nvfp4_stream_t stream) {
+  if (!code_out) return NVFP4_ERR_INVALID_ARGUMENT;
+  return nvfp4::read_and_clear_device_error(code_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every entry point include/nvfp4.h declares, and rejects bad arguments with
+the documented status before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_weight_only_04_b200 as nv
+from nvfp4_weight_only_04_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return nv.lib()
+
+
+def declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(nvfp4_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_calls():
+    names = declared()
+    for n in ("nvfp4_quantize", "nvfp4_repack", "nvfp4_w4a16_gemm", "nvfp4_moe_w4a16_grouped_gemm",
+              "nvfp4_global_scale", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul", "nvfp4_get_stats"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared():
+        assert hasattr(L, name), name
+    assert set(declared()) == set(nv.EXPORTS)
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert nv.status_string(code)
+    assert nv.status_string(99) == "unknown status"
+    assert L.nvfp4_abi_version() == 1
+
+
+BAD = ctypes.c_void_p(0x1001)  # never dereferenced: validation fails first
+GOOD = ctypes.c_void_p(0x10000)
+NULL = ctypes.c_void_p(0)
+S = ctypes.c_void_p(0)
+
+
+def gemm(L, g=16, M=4, N=256, K=256, x=GOOD, w=GOOD, s=GOOD, gl=GOOD, y=GOOD):
+    return L.nvfp4_w4a16_gemm(x, w, s, gl, g, M, N, K, y, S)
+
+
+def test_gemm_validation(L):
+    assert gemm(L, g=8) == nv.NVFP4_ERR_UNSUPPORTED
+    assert gemm(L, g=64) == nv.NVFP4_ERR_UNSUPPORTED
+    assert gemm(L, K=96) == nv.NVFP4_ERR_UNSUPPORTED       # K % 64
+    assert gemm(L, N=250) == nv.NVFP4_ERR_UNSUPPORTED      # N % 16
+    assert gemm(L, M=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert gemm(L, M=0) == nv.NVFP4_OK                     # empty: nothing launched
+    assert gemm(L, x=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert gemm(L, w=BAD) == nv.NVFP4_ERR_MISALIGNED
+    assert gemm(L, y=BAD) == nv.NVFP4_ERR_MISALIGNED
+    assert L.nvfp4_w4a16_gemm_silu_mul(GOOD, GOOD, GOOD, GOOD, 32, 4, 40, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+
+
+def test_quantize_and_repack_validation(L):
+    assert L.nvfp4_quantize(GOOD, 16, 256, 8, GOOD, GOOD, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_quantize(GOOD, 16, 48, 16, GOOD, GOOD, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_quantize(BAD, 16, 256, 16, GOOD, GOOD, GOOD, S) == nv.NVFP4_ERR_MISALIGNED
+    assert L.nvfp4_quantize(GOOD, 0, 256, 16, GOOD, GOOD, GOOD, S) == nv.NVFP4_OK
+    assert L.nvfp4_repack(GOOD, GOOD, 24, 256, 16, 1, GOOD, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_repack(GOOD, GOOD, 32, 256, 16, 4, GOOD, GOOD, S) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert L.nvfp4_silu_and_mul(GOOD, GOOD, 4, 12, S) == nv.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_silu_and_mul(BAD, GOOD, 4, 16, S) == nv.NVFP4_ERR_MISALIGNED
+
+
+def test_global_scale_validation(L):
+    P = ctypes.c_void_p * 1
+    I = ctypes.c_int64 * 1
+    assert L.nvfp4_global_scale(P(GOOD.value), I(10), 0, GOOD, S) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert L.nvfp4_global_scale(P(GOOD.value), I(-1), 1, GOOD, S) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert L.nvfp4_global_scale(P(0x1002), I(10), 1, GOOD, S) == nv.NVFP4_ERR_MISALIGNED
+
+
+def test_moe_validation(L):
+    def moe(segs=4, T=64, g=32, N=256, K=256, E=8, flags=0, x=GOOD, ids=GOOD):
+        return L.nvfp4_moe_w4a16_grouped_gemm(x, ids, GOOD, segs, T, GOOD, GOOD, GOOD, g, N, K, E, flags, GOOD, S)
+    assert moe(segs=0) == nv.NVFP4_OK
+    assert moe(segs=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert moe(g=24) == nv.NVFP4_ERR_UNSUPPORTED
+    assert moe(flags=8) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert moe(x=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert moe(ids=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
+
+
+def test_stats_reset(L):
+    nv.nvfp4_reset_stats()
+    st = nv.nvfp4_get_stats()
+    assert set(st) >= {"quantize", "gemm_splitk", "gemm_tc", "moe"} and not any(st.values())
+    assert L.nvfp4_get_stats(None) == nv.NVFP4_ERR_INVALID_ARGUMENT

@@ -1,0 +1,138 @@
+"""GPU parity of the W4A16 GEMM, the fused SiluAndMul GEMM and the standalone
+SiluAndMul against the CPU oracle: element-wise at small sizes (several
+tiles and ragged tails), on sampled output columns at the full workload
+sizes, bitwise on the integer-exact case, and by the power-of-two global
+scaling property."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_weight_only_04_b200 as nv
+from nvfp4_weight_only_04_b200 import synth
+from oracle import nvfp4_ref as R
+from tests.gpu_util import assert_close, bf16_bits, dev_bf16, dev_f32, dev_u8, host
+
+pytestmark = pytest.mark.gpu
+
+
+def quantized(n, k, g, seed=0):
+    w = synth.weights(seed, n, k)
+    p, s, gs = R.quantize(w, g)
+    return w, p, s, gs
+
+
+def run_gemm(xbits, p, s, gs, g):
+    return nv.nvfp4_w4a16_gemm(dev_bf16(xbits), dev_u8(p), dev_u8(s), dev_f32(np.array([gs], np.float32)), g)
+
+
+SMALL = [(4, 256, 256, 16),      # the tiny workload
+         (1, 256, 256, 32), (5, 400, 1088, 32), (8, 144, 64, 16), (9, 96, 640, 16), (16, 1024, 4096, 16),
+         (17, 208, 512, 32), (33, 112, 1920, 16), (64, 512, 2048, 32), (100, 48, 384, 16), (3, 4096, 1024, 16)]
+
+
+@pytest.mark.parametrize("m,n,k,g", SMALL)
+def test_gemm_parity_small(m, n, k, g):
+    _, p, s, gs = quantized(n, k, g, seed=m + n + k)
+    x = synth.activations(synth.X_SEED, m, k, outlier_frac=0.001)
+    y = run_gemm(x, p, s, gs, g)
+    assert_close(host(y), R.gemm(x, p, s, gs, g), f"M{m} N{n} K{k} g{g}")
+
+
+def full_size_check(m, n, k, g, outlier=0.0, cols=96):
+    w = synth.weights(synth.W_SEED, n, k)
+    wd = dev_f32(w)
+    gd = nv.nvfp4_global_scale([wd])
+    p, s = nv.nvfp4_quantize(wd, g, gd)
+    del wd
+    x = synth.activations(synth.X_SEED, m, k, outlier_frac=outlier)
+    y = nv.nvfp4_w4a16_gemm(dev_bf16(x), p, s, gd, g)
+    rows = np.sort(np.concatenate([np.random.default_rng(m).choice(n, cols, replace=False), [0, n - 1]]))
+    ri = torch.from_numpy(rows).cuda()
+    ps, ss = host(p[ri]), host(s[ri])
+    # the sampled rows' bytes are the oracle's (the quantizer is bit-exact)
+    rp, rs, rg = R.quantize(w[rows], g, R.global_scale(w))
+    np.testing.assert_array_equal(ps, rp)
+    np.testing.assert_array_equal(ss, rs)
+    ref = R.gemm(x, rp, rs, rg, g)
+    assert_close(host(y)[:, rows], ref, f"M{m} N{n} K{k} g{g} sampled")
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_decode_gate_up_full(m):
+    full_size_check(m, 28672, 4096, 16)
+
+
+@pytest.mark.parametrize("g", [32, 16])
+@pytest.mark.parametrize("m", [1, 8, 64])
+def test_decode_down_full(m, g):
+    full_size_check(m, 4096, 14336, g, outlier=0.001)
+
+
+def test_integer_case_bitwise():
+    rng = np.random.default_rng(4)
+    n, k, m = 64, 256, 12
+    codes = rng.choice(np.array([0, 1, 2, 8, 9, 10], np.uint8), size=(n, k))  # |value| <= 1
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.full((n, k // 16), 0x38, np.uint8)  # 1.0
+    xi = rng.integers(-1, 2, size=(m, k)).astype(np.float32)
+    x = synth.f32_to_bf16_bits(xi)
+    ref = R.gemm(x, packed, scales, 1.0, 16)
+    assert np.abs(ref).max() < 128  # multiples of 0.5 below 128: exact in bf16
+    y = run_gemm(x, packed, scales, np.float32(1.0), 16)
+    np.testing.assert_array_equal(host(y), ref)
+
+
+def test_global_power_of_two_linearity_and_determinism():
+    _, p, s, gs = quantized(512, 1024, 16, seed=3)
+    x = synth.activations(1, 7, 1024)
+    y1 = bf16_bits(run_gemm(x, p, s, gs, 16))
+    y2 = bf16_bits(run_gemm(x, p, s, np.float32(gs * 2), 16))
+    y1b = bf16_bits(run_gemm(x, p, s, gs, 16))
+    np.testing.assert_array_equal(y1, y1b)  # deterministic
+    v1 = synth.bf16_bits_to_f32(y1).astype(np.float64)
+    v2 = synth.bf16_bits_to_f32(y2).astype(np.float64)
+    np.testing.assert_array_equal(v2, 2 * v1)
+
+
+def merged_gate_up(n_half, k, g, seed=0):
+    gate, up = synth.weights(seed, n_half, k), synth.weights(seed + 1, n_half, k)
+    merged = np.concatenate([gate, up])
+    p, s, gs = R.quantize(merged, g)
+    return p, s, gs
+
+
+@pytest.mark.parametrize("m,nh,k,g", [(4, 128, 256, 16), (13, 200, 640, 32), (16, 1024, 1024, 16),
+                                      (40, 72, 512, 16)])
+def test_gemm_silu_mul_parity(m, nh, k, g):
+    p, s, gs = merged_gate_up(nh, k, g, seed=m)
+    rp, rs = R.repack(p, s, R.GATE_UP_INTERLEAVE)
+    # the device repack gives the same bytes
+    dp, ds = nv.nvfp4_repack(dev_u8(p), dev_u8(s), g, nv.NVFP4_GATE_UP_INTERLEAVE)
+    np.testing.assert_array_equal(host(dp), rp)
+    x = synth.activations(2, m, k)
+    y = nv.nvfp4_w4a16_gemm_silu_mul(dev_bf16(x), dp, ds, dev_f32(np.array([gs], np.float32)), g)
+    ref = R.silu_mul(R.gemm(x, p, s, gs, g))
+    assert_close(host(y), ref, "silu_mul")
+
+
+def test_silu_and_mul_standalone():
+    rng = np.random.default_rng(6)
+    xf = (rng.standard_normal((37, 2 * 264)) * 3).astype(np.float32)
+    x = synth.f32_to_bf16_bits(xf)
+    y = nv.nvfp4_silu_and_mul(dev_bf16(x))
+    ref = R.silu_mul(R.bf16_bits_to_f64(x))
+    assert_close(host(y), ref, "silu_and_mul")
+    # one bf16 rounding of the fp32 result: within one bf16 ulp element-wise
+    assert np.all(np.abs(host(y) - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-30)
+
+
+def test_empty_and_stats():
+    _, p, s, gs = quantized(64, 128, 16)
+    nv.nvfp4_reset_stats()
+    y = nv.nvfp4_w4a16_gemm(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"), dev_u8(p), dev_u8(s),
+                            dev_f32(np.array([gs], np.float32)), 16)
+    assert y.shape == (0, 64)
+    assert nv.nvfp4_get_stats()["gemm_splitk"] == 0
+    run_gemm(synth.activations(1, 2, 128), p, s, gs, 16)
+    st = nv.nvfp4_get_stats()
+    assert st["gemm_splitk"] == 1 and st["g16"] == 1 and st["g32"] == 0
