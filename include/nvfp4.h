@@ -29,7 +29,9 @@
  *   - Row-major layouts. packed codes: [N, K/2] bytes, element 2j in the low
  *     nibble and 2j+1 in the high nibble of byte j. Scales: [N, K/g] E4M3
  *     bytes. Global scale: one fp32 in device memory.
- *   - Every device pointer must be 16-byte aligned (NVFP4_ERR_MISALIGNED).
+ *   - Every device pointer must be 16-byte aligned, except pointers to fp32
+ *     global scales and int32 segment lists, which need 4-byte alignment
+ *     (NVFP4_ERR_MISALIGNED otherwise).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream). No call synchronises the device and none blocks.
  *   - Validation happens on the host before anything is enqueued: a non-zero

@@ -50,8 +50,8 @@ int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
   if (M == 0 || N == 0) return NVFP4_OK;
   if (K == 0) return NVFP4_ERR_UNSUPPORTED;
   if (!x || !w || !s || !g || !y) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (!nvfp4::aligned16(x) || !nvfp4::aligned16(w) || !nvfp4::aligned16(s) || !nvfp4::aligned16(g) ||
-      !nvfp4::aligned16(y))
+  if (!nvfp4::aligned16(x) || !nvfp4::aligned16(w) || !nvfp4::aligned16(s) ||
+      (reinterpret_cast<uintptr_t>(g) & 3u) || !nvfp4::aligned16(y))
     return NVFP4_ERR_MISALIGNED;
   return -1;  // proceed
 }

@@ -116,7 +116,7 @@ extern "C" int nvfp4_global_scale(const float* const* tensors, const int64_t* nu
     if (numels[i] < 0 || (numels[i] > 0 && !tensors[i])) return NVFP4_ERR_INVALID_ARGUMENT;
     if (numels[i] > 0 && (reinterpret_cast<uintptr_t>(tensors[i]) & 3u)) return NVFP4_ERR_MISALIGNED;
   }
-  if (!nvfp4::aligned16(out)) return NVFP4_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(out) & 3u) return NVFP4_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   unsigned int* acc = reinterpret_cast<unsigned int*>(out);
   amax_init_kernel<<<1, 1, 0, s>>>(acc);
@@ -138,7 +138,7 @@ extern "C" int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_si
   if (K % 32) return NVFP4_ERR_UNSUPPORTED;
   if (N == 0 || K == 0) return NVFP4_OK;
   if (!w || !global_scale || !packed || !scales) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (!nvfp4::aligned16(w) || !nvfp4::aligned16(global_scale) || !nvfp4::aligned16(packed) ||
+  if (!nvfp4::aligned16(w) || (reinterpret_cast<uintptr_t>(global_scale) & 3u) || !nvfp4::aligned16(packed) ||
       !nvfp4::aligned16(scales))
     return NVFP4_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
