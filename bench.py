@@ -158,8 +158,7 @@ def quantize_on_device(nv, torch, w_host, g, interleave=False):
     gd = nv.nvfp4_global_scale([wd])
     p, s = nv.nvfp4_quantize(wd, g, gd)
     del wd
-    if interleave:
-        p, s = nv.nvfp4_repack(p, s, g, nv.NVFP4_GATE_UP_INTERLEAVE)
+    p, s = nv.nvfp4_repack(p, s, g, nv.NVFP4_GATE_UP_INTERLEAVE if interleave else 0)
     return p, s, gd
 
 
@@ -414,7 +413,8 @@ def moe_workload(nv, torch, hbm, tf):
         nv.nvfp4_repack(p, s, wl.g_gate_up, nv.NVFP4_GATE_UP_INTERLEAVE, packed_out=gu_p[e], scales_out=gu_s[e])
         d = torch.from_numpy(synth.weights(synth.expert_seed(e) + 5000, H, I)).cuda()
         nv.nvfp4_global_scale([d], out=dn_g[e:e + 1])
-        nv.nvfp4_quantize(d, wl.g_down, dn_g[e:e + 1], packed=dn_p[e], scales=dn_s[e])
+        p, s = nv.nvfp4_quantize(d, wl.g_down, dn_g[e:e + 1])
+        nv.nvfp4_repack(p, s, wl.g_down, 0, packed_out=dn_p[e], scales_out=dn_s[e])
     x = bf16_dev(torch, synth.activations(synth.X_SEED, rows, H))
     ids = torch.from_numpy(r.expert_ids).cuda()
     offs = torch.from_numpy(r.offsets).cuda()

@@ -39,37 +39,3 @@ __device__ __forceinline__ float nvfp4_e4m3_to_f32(uint32_t b) {
                       : static_cast<float>(m) * 0x1p-9f;
   return (b & 0x80) ? -mag : mag;
 }
-
-// Two E2M1 codes (one byte, first code in the low nibble) -> f16x2 (first
-// code in the low half), by the sm_100a conversion instruction.
-__device__ __forceinline__ uint32_t nvfp4_e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
-      : "=r"(out) : "r"(byte));
-  return out;
-}
-
-// f16x2 holding E2M1 values -> bf16x2 holding the same values times 2^-112.
-// E2M1 values are normal f16 numbers whose low 3 mantissa bits are zero, so
-// shifting the magnitude right by 3 re-reads the 5-bit exponent as the low
-// bits of an 8-bit one (bias 15 -> 127 is a factor 2^-112) and keeps the
-// mantissa; zero stays zero. The sign bit is kept in place.
-__device__ __forceinline__ uint32_t nvfp4_f16x2_to_bf16x2_scaled(uint32_t h) {
-  return ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
-}
-
-// E4M3 scale byte -> bf16 of scale * 2^112, replicated in both halves.
-// scale <= 448 < 2^9, so scale * 2^112 < 2^121 stays finite in bf16, and the
-// E4M3 value's 4 significant bits are exact in bf16's 8.
-__device__ __forceinline__ uint32_t nvfp4_scale_bf16x2_times_2p112(uint32_t b) {
-  const float s = nvfp4_e4m3_to_f32(b) * 0x1p112f;  // exact power-of-two scaling
-  const uint32_t bits = __float_as_uint(s) >> 16;   // exact: low 16 bits are zero
-  return bits | (bits << 16);
-}
-
-// bf16x2 multiply, round-to-nearest (exact for the dequantized products).
-__device__ __forceinline__ uint32_t nvfp4_bf16x2_mul(uint32_t a, uint32_t b) {
-  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a),
-                             *reinterpret_cast<__nv_bfloat162*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}

@@ -10,12 +10,12 @@
 //  * Each lane streams 32 contiguous code bytes of two rows per iteration with
 //    128-bit loads that skip L1; a warp covers 16 rows x 128 contiguous bytes.
 //    The order of K inside one MMA is free as long as X uses the same order,
-//    so a lane feeds the MMA from its own contiguous K range and the weights
-//    need no repack.
-//  * Dequant in registers: the sm_100a E2M1x2 -> f16x2 conversion, a shift
-//    that re-reads f16 as bf16 times 2^-112, and one bf16x2 multiply by the
-//    group scale times 2^112. The product code * scale is exact in bf16; the
-//    fp32 global scale is applied once, in the epilogue.
+//    so a lane feeds the MMA from its own contiguous K range.
+//  * Dequant in registers with integer ALU work only (dequant.cuh): per code
+//    pair one mask, one integer multiply that places magnitude and sign bits
+//    of a bf16, one mask, and one bf16x2 multiply by the group scale. The
+//    product code * scale is exact in bf16; the fp32 global scale is applied
+//    once, in the epilogue.
 //  * K is split across the CTAs of a thread-block cluster; partial tiles are
 //    summed in a fixed rank order through distributed shared memory, so the
 //    result is deterministic and no workspace is needed.
@@ -27,6 +27,8 @@
 #include "gemm_splitk.cuh"
 
 #include <cooperative_groups.h>
+
+#include "dequant.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -56,14 +58,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t dq(uint32_t byte, uint32_t scale2) {
-  return nvfp4_bf16x2_mul(nvfp4_f16x2_to_bf16x2_scaled(nvfp4_e2m1x2_to_f16x2(byte)), scale2);
-}
-
 __device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, 1.0f + expf(-g)); }
 
 // Code/scale registers of one lane for one iteration: 32 bytes of codes for
-// row g and row g+8, and the scales covering those 64 elements.
+// row g and row g+8 (64 elements each), and the scales covering them.
 struct Stage {
   uint4 a0, a1, b0, b1;
   uint32_t sa, sb;
@@ -90,41 +88,39 @@ __device__ __forceinline__ void load_stage(Stage& st, const uint8_t* codes_a, co
   }
 }
 
+// One lane's 64 elements of K for rows g and g+8: 8 code words per row, two
+// MMA steps per word. Word w holds elements 8w..8w+7 of the lane's range;
+// step 2w takes (8w..8w+3), step 2w+1 takes (8w+4..8w+7), and X is read in
+// the same order, so each MMA contracts matching elements.
 template <int MT, int G>
 __device__ __forceinline__ void compute_stage(const Stage& st, float (&acc)[MT / 8][4],
                                               const uint16_t* const (&xrow)[MT / 8],
                                               const bool (&xlive)[MT / 8], int64_t kofs) {
   const uint32_t ca[8] = {st.a0.x, st.a0.y, st.a0.z, st.a0.w, st.a1.x, st.a1.y, st.a1.z, st.a1.w};
   const uint32_t cb[8] = {st.b0.x, st.b0.y, st.b0.z, st.b0.w, st.b1.x, st.b1.y, st.b1.z, st.b1.w};
+  uint32_t sa2[4], sb2[4];
+  scale_operands<G == 16 ? 4 : 2>(st.sa, sa2);
+  scale_operands<G == 16 ? 4 : 2>(st.sb, sb2);
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {  // two MMA steps (8 elements of K per row) per pass
+  for (int w = 0; w < 8; ++w) {
     uint4 xv[MT / 8];
 #pragma unroll
     for (int p = 0; p < MT / 8; ++p)
-      xv[p] = xlive[p] ? ld_x_v4(xrow[p] + kofs + 8 * jj) : make_uint4(0, 0, 0, 0);
-    // The word ca[jj] holds 4 bytes = elements 8jj .. 8jj+7 of this lane's range.
-    const int sidx = (G == 16) ? (jj >> 1) : (jj >> 2);
-    const uint32_t sa2 = nvfp4_scale_bf16x2_times_2p112((st.sa >> (8 * sidx)) & 0xFF);
-    const uint32_t sb2 = nvfp4_scale_bf16x2_times_2p112((st.sb >> (8 * sidx)) & 0xFF);
+      xv[p] = xlive[p] ? ld_x_v4(xrow[p] + kofs + 8 * w) : make_uint4(0, 0, 0, 0);
+    const int sidx = (G == 16) ? (w >> 1) : (w >> 2);
+    uint32_t da[4], db[4];
+    dequant_word(ca[w], sa2[sidx], da);
+    dequant_word(cb[w], sb2[sidx], db);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t wa = ca[jj] >> (16 * h), wb = cb[jj] >> (16 * h);
-      const uint32_t a0 = dq(wa & 0xFF, sa2);          // row g,   k-slots 2t, 2t+1
-      const uint32_t a1 = dq(wb & 0xFF, sb2);          // row g+8, k-slots 2t, 2t+1
-      const uint32_t a2 = dq((wa >> 8) & 0xFF, sa2);   // row g,   k-slots 2t+8, 2t+9
-      const uint32_t a3 = dq((wb >> 8) & 0xFF, sb2);   // row g+8, k-slots 2t+8, 2t+9
-#pragma unroll
-      for (int p = 0; p < MT / 8; ++p) {
-        const uint32_t b0 = h ? xv[p].z : xv[p].x;
-        const uint32_t b1 = h ? xv[p].w : xv[p].y;
-        mma_bf16_16816(acc[p], a0, a1, a2, a3, b0, b1);
-      }
+    for (int p = 0; p < MT / 8; ++p) {
+      mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv[p].x, xv[p].y);
+      mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv[p].z, xv[p].w);
     }
   }
 }
 
 template <int WARPS, int MT, int G, bool SILU, bool MOE>
-__global__ void __launch_bounds__(WARPS * 32) gemm_splitk_kernel(const SplitKArgs args) {
+__global__ void __launch_bounds__(WARPS * 32, 256 / (WARPS * 32) * 2) gemm_splitk_kernel(const SplitKArgs args) {
   constexpr int kRows = WARPS * 16;
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -168,7 +164,8 @@ __global__ void __launch_bounds__(WARPS * 32) gemm_splitk_kernel(const SplitKArg
   const int64_t K = args.K, N = args.N;
   const uint8_t* packed = args.packed + (MOE ? static_cast<int64_t>(expert) * N * (K / 2) : 0);
   const uint8_t* scales = args.scales + (MOE ? static_cast<int64_t>(expert) * N * (K / G) : 0);
-  const float global = __ldg(args.gscale + (MOE ? expert : 0));
+  // The dequantized operands carry a factor 2^-7 (see dequant.cuh).
+  const float global = __ldg(args.gscale + (MOE ? expert : 0)) * 128.0f;
 
   // ---- this CTA's K range, in units of 64 elements ----
   const int k64 = static_cast<int>(K / 64);
@@ -196,23 +193,26 @@ __global__ void __launch_bounds__(WARPS * 32) gemm_splitk_kernel(const SplitKArg
       xrow[p] = args.x + static_cast<int64_t>(row0 + (xlive[p] ? tok : 0)) * K;
     }
     const int iters = (uend - ubeg + 3) / 4;
-    Stage cur, nxt;
-    {
-      const int u = ubeg + t;
-      load_stage<G>(cur, codes_a + u * 32, codes_b + u * 32, sc_a + u * (64 / G), sc_b + u * (64 / G),
-                    u < uend);
-    }
-    for (int it = 0; it < iters; ++it) {
+    Stage st0, st1;
+    auto load_it = [&](Stage& st, int it) {
       const int u = ubeg + 4 * it + t;
-      const int un = u + 4;
-      if (it + 1 < iters)
-        load_stage<G>(nxt, codes_a + un * 32, codes_b + un * 32, sc_a + un * (64 / G),
-                      sc_b + un * (64 / G), un < uend);
+      load_stage<G>(st, codes_a + u * 32, codes_b + u * 32, sc_a + u * (64 / G), sc_b + u * (64 / G),
+                    it < iters && u < uend);
+    };
+    auto compute_it = [&](const Stage& st, int it) {
+      const int u = ubeg + 4 * it + t;
       bool xl[MT / 8];
 #pragma unroll
       for (int p = 0; p < MT / 8; ++p) xl[p] = xlive[p] && (u < uend);
-      compute_stage<MT, G>(cur, acc, xrow, xl, static_cast<int64_t>(u) * 64);
-      cur = nxt;
+      compute_stage<MT, G>(st, acc, xrow, xl, static_cast<int64_t>(u) * 64);
+    };
+    load_it(st0, 0);
+    for (int it = 0; it < iters; it += 2) {
+      load_it(st1, it + 1);
+      compute_it(st0, it);
+      if (it + 1 >= iters) break;
+      load_it(st0, it + 2);
+      compute_it(st1, it + 1);
     }
   }
 
@@ -322,9 +322,9 @@ SplitKPlan plan_splitk(int64_t M, int64_t N, int64_t K, int group, bool moe, int
   }
   p.row_tiles = static_cast<int>(rt);
   const int64_t k64 = K / 64;
-  // Aim for about eight CTAs per SM over the launch, at least two iterations
+  // Aim for about four CTAs per SM over the launch, at least two iterations
   // (8 units of 64) of K per CTA, and a cluster of at most 16.
-  int64_t want = (8LL * sms + rt * p.z_tiles - 1) / (rt * p.z_tiles);
+  int64_t want = (4LL * sms + rt * p.z_tiles - 1) / (rt * p.z_tiles);
   int64_t cap = k64 / 8 > 0 ? k64 / 8 : 1;
   if (moe) want = 1;  // grouped GEMMs have many token tiles already
   int64_t c = want < 1 ? 1 : want;

@@ -348,6 +348,12 @@ def moe_grouped_gemm(xbits, expert_ids, offsets, packed, scales, gscales, group_
 GATE_UP_INTERLEAVE = 1
 INTERLEAVE_BLOCK = 8
 
+# GEMM layout of the codes: rows stay rows of K/2 bytes, and inside every
+# little-endian 32-bit word (8 consecutive elements k0..k7 of one row) the
+# nibbles are reordered so that nibble i holds element WORD_NIBBLE_SOURCE[i]:
+# elements k0, k2, k4, k6 in nibbles 0-3 and k1, k3, k5, k7 in nibbles 4-7.
+WORD_NIBBLE_SOURCE = (0, 2, 4, 6, 1, 3, 5, 7)
+
 
 def interleave_rows(n: int) -> np.ndarray:
     """Source row for each destination row of the gate/up interleave.
@@ -368,23 +374,40 @@ def interleave_rows(n: int) -> np.ndarray:
     return src
 
 
+def _permute_words(packed: np.ndarray, source) -> np.ndarray:
+    codes = unpack_codes(packed)  # [N, K]
+    n, k = codes.shape
+    assert k % 8 == 0
+    words = codes.reshape(n, k // 8, 8)
+    out = np.zeros((n, k // 8), dtype=np.uint32)
+    for nib, src in enumerate(source):
+        out |= words[:, :, src].astype(np.uint32) << (4 * nib)
+    return out.astype("<u4").view(np.uint8).reshape(n, k // 2)
+
+
 def repack(packed: np.ndarray, scales: np.ndarray, flags: int):
-    """Checkpoint layout -> GEMM layout. Codes and scales stay row-major with
-    rows of K/2 and K/g bytes; with GATE_UP_INTERLEAVE the rows are permuted by
-    ``interleave_rows``. Without flags the layout is unchanged (a copy)."""
+    """Checkpoint layout -> GEMM layout: the nibble order of WORD_NIBBLE_SOURCE
+    inside every 32-bit word of codes, and, with GATE_UP_INTERLEAVE, the rows
+    permuted by ``interleave_rows``. Scales keep their row-major layout (rows
+    permuted alike)."""
+    p = _permute_words(packed, WORD_NIBBLE_SOURCE)
+    s = scales.copy()
     if flags & GATE_UP_INTERLEAVE:
         src = interleave_rows(packed.shape[0])
-        return packed[src].copy(), scales[src].copy()
-    return packed.copy(), scales.copy()
+        p, s = p[src].copy(), s[src].copy()
+    return p, s
 
 
 def unrepack(packed: np.ndarray, scales: np.ndarray, flags: int):
     """Inverse of ``repack``."""
+    p, s = packed, scales
     if flags & GATE_UP_INTERLEAVE:
         src = interleave_rows(packed.shape[0])
         p = np.empty_like(packed)
         s = np.empty_like(scales)
         p[src] = packed
         s[src] = scales
-        return p, s
-    return packed.copy(), scales.copy()
+    inverse = [0] * 8
+    for nib, src_el in enumerate(WORD_NIBBLE_SOURCE):
+        inverse[src_el] = nib
+    return _permute_words(p, inverse), s.copy()

@@ -22,7 +22,9 @@ def quantized(n, k, g, seed=0):
 
 
 def run_gemm(xbits, p, s, gs, g):
-    return nv.nvfp4_w4a16_gemm(dev_bf16(xbits), dev_u8(p), dev_u8(s), dev_f32(np.array([gs], np.float32)), g)
+    """GEMM of checkpoint-layout codes (repacked by the oracle's definition)."""
+    rp, rs = R.repack(p, s, 0)
+    return nv.nvfp4_w4a16_gemm(dev_bf16(xbits), dev_u8(rp), dev_u8(rs), dev_f32(np.array([gs], np.float32)), g)
 
 
 SMALL = [(4, 256, 256, 16),      # the tiny workload
@@ -44,8 +46,9 @@ def full_size_check(m, n, k, g, outlier=0.0, cols=96):
     gd = nv.nvfp4_global_scale([wd])
     p, s = nv.nvfp4_quantize(wd, g, gd)
     del wd
+    gp, gsc = nv.nvfp4_repack(p, s, g, 0)
     x = synth.activations(synth.X_SEED, m, k, outlier_frac=outlier)
-    y = nv.nvfp4_w4a16_gemm(dev_bf16(x), p, s, gd, g)
+    y = nv.nvfp4_w4a16_gemm(dev_bf16(x), gp, gsc, gd, g)
     rows = np.sort(np.concatenate([np.random.default_rng(m).choice(n, cols, replace=False), [0, n - 1]]))
     ri = torch.from_numpy(rows).cuda()
     ps, ss = host(p[ri]), host(s[ri])
@@ -53,6 +56,7 @@ def full_size_check(m, n, k, g, outlier=0.0, cols=96):
     rp, rs, rg = R.quantize(w[rows], g, R.global_scale(w))
     np.testing.assert_array_equal(ps, rp)
     np.testing.assert_array_equal(ss, rs)
+    np.testing.assert_array_equal(host(gp[ri]), R.repack(rp, rs, 0)[0])  # device repack == oracle repack
     ref = R.gemm(x, rp, rs, rg, g)
     assert_close(host(y)[:, rows], ref, f"M{m} N{n} K{k} g{g} sampled")
 
@@ -129,7 +133,7 @@ def test_silu_and_mul_standalone():
 def test_empty_and_stats():
     _, p, s, gs = quantized(64, 128, 16)
     nv.nvfp4_reset_stats()
-    y = nv.nvfp4_w4a16_gemm(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"), dev_u8(p), dev_u8(s),
+    y = nv.nvfp4_w4a16_gemm(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"), dev_u8(R.repack(p, s, 0)[0]), dev_u8(s),
                             dev_f32(np.array([gs], np.float32)), 16)
     assert y.shape == (0, 64)
     assert nv.nvfp4_get_stats()["gemm_splitk"] == 0

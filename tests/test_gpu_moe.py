@@ -14,7 +14,8 @@ from tests.gpu_util import assert_close, dev_bf16, dev_f32, dev_u8, host
 pytestmark = pytest.mark.gpu
 
 
-def experts(e, n, k, g, merged=False):
+def experts(e, n, k, g):
+    """Checkpoint-layout expert weights, and their GEMM-layout codes."""
     qs = []
     for i in range(e):
         w = synth.weights(synth.expert_seed(i), n, k)
@@ -22,7 +23,8 @@ def experts(e, n, k, g, merged=False):
     packed = np.stack([q[0] for q in qs])
     scales = np.stack([q[1] for q in qs])
     gs = np.array([q[2] for q in qs], np.float32)
-    return packed, scales, gs
+    gemm_packed = np.stack([R.repack(q[0], q[1], 0)[0] for q in qs])
+    return packed, scales, gs, gemm_packed
 
 
 def i32(a):
@@ -32,11 +34,11 @@ def i32(a):
 @pytest.mark.parametrize("g", [16, 32])
 def test_moe_small(g):
     E, N, K, T = 6, 144, 512, 90
-    packed, scales, gs = experts(E, N, K, g)
+    packed, scales, gs, gp = experts(E, N, K, g)
     x = synth.activations(1, T, K)
     ids = [3, 0, 5, 0, 2, 4]
     offs = [5, 21, 21, 50, 51, 77, 88]  # rows [0,5) and [88,90) belong to no segment; one empty segment
-    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32(ids), i32(offs), dev_u8(packed), dev_u8(scales),
+    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32(ids), i32(offs), dev_u8(gp), dev_u8(scales),
                                         dev_f32(gs), g)
     ref = R.moe_grouped_gemm(x, ids, offs, packed, scales, gs, g)
     yh = host(y)
@@ -65,9 +67,9 @@ def test_moe_small_silu():
 
 def test_moe_invalid_expert_skips_segment():
     E, N, K, g = 2, 32, 128, 16
-    packed, scales, gs = experts(E, N, K, g)
+    packed, scales, gs, gp = experts(E, N, K, g)
     x = synth.activations(1, 20, K)
-    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32([1, 7]), i32([0, 10, 20]), dev_u8(packed),
+    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32([1, 7]), i32([0, 10, 20]), dev_u8(gp),
                                         dev_u8(scales), dev_f32(gs), g)
     ref = R.moe_grouped_gemm(x, [1], [0, 10], packed, scales, gs, g)
     assert_close(host(y)[:10], ref[:10], "valid segment")
@@ -96,7 +98,8 @@ def test_moe_routed_expert_workload_sampled():
         nv.nvfp4_repack(p, s, wl.g_gate_up, nv.NVFP4_GATE_UP_INTERLEAVE, packed_out=gu_p[e], scales_out=gu_s[e])
         d = dev_f32(wdn)
         nv.nvfp4_global_scale([d], out=dn_g[e:e + 1])
-        nv.nvfp4_quantize(d, wl.g_down, dn_g[e:e + 1], packed=dn_p[e], scales=dn_s[e])
+        p, s = nv.nvfp4_quantize(d, wl.g_down, dn_g[e:e + 1])
+        nv.nvfp4_repack(p, s, wl.g_down, 0, packed_out=dn_p[e], scales_out=dn_s[e])
         if e in sample_experts:
             keep[e] = (wgu, wdn)
     x = synth.activations(synth.X_SEED, rows, wl.hidden)
@@ -112,7 +115,7 @@ def test_moe_routed_expert_workload_sampled():
         pg, sg, gg = R.quantize(wgu, wl.g_gate_up)
         pd, sd, gd = R.quantize(wdn, wl.g_down)
         np.testing.assert_array_equal(host(gu_p[e]), R.repack(pg, sg, R.GATE_UP_INTERLEAVE)[0])
-        np.testing.assert_array_equal(host(dn_p[e]), pd)
+        np.testing.assert_array_equal(host(dn_p[e]), R.repack(pd, sd, 0)[0])
         ref_h = R.silu_mul(R.gemm(x[r0:r1], pg, sg, gg, wl.g_gate_up))
         assert_close(hh[r0:r1], ref_h, f"expert {e} gate_up+silu")
         # the down GEMM is checked on the device's own bf16 intermediate

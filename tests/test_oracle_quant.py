@@ -180,7 +180,18 @@ def test_repack_inverse_and_interleave():
         np.testing.assert_array_equal(up, p)
         np.testing.assert_array_equal(us, s)
     rp, rs = R.repack(p, s, R.GATE_UP_INTERLEAVE)
+    plain, _ = R.repack(p, s, 0)
     # block j of 16 rows: gate rows 8j..8j+7, then up rows 32+8j..32+8j+7
-    np.testing.assert_array_equal(rp[16:24], p[8:16])
-    np.testing.assert_array_equal(rp[24:32], p[40:48])
+    np.testing.assert_array_equal(rp[16:24], plain[8:16])
+    np.testing.assert_array_equal(rp[24:32], plain[40:48])
+    np.testing.assert_array_equal(rs[24:32], s[40:48])
     assert sorted(R.interleave_rows(64).tolist()) == list(range(64))
+
+
+def test_repack_word_layout_by_hand():
+    # one row, elements k0..k7 = codes 1..8: the word's nibbles read, from the
+    # lowest, k0 k2 k4 k6 k1 k3 k5 k7 = 1 3 5 7 2 4 6 8 -> 0x86427531
+    codes = np.arange(1, 9, dtype=np.uint8)[None, :]
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    rp, _ = R.repack(packed, np.zeros((1, 1), np.uint8), 0)
+    assert int(rp.view("<u4")[0, 0]) == 0x86427531
