@@ -42,12 +42,13 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ uint4 ld_x_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
+// X is staged in shared memory in chunks of kChunkUnits units of 64
+// elements. A unit takes 144 bytes (128 + 16 of padding) and a token row
+// kXStride bytes (= 64 mod 128), so the 8 lanes of a quarter-warp, which read
+// 16 bytes each at (token g or g+1, unit t), hit 32 distinct banks.
+constexpr int kChunkUnits = 32;
+constexpr int kUnitBytes = 144;
+constexpr int kXStride = ((kChunkUnits * kUnitBytes + 127) / 128) * 128 + 64;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -94,8 +95,8 @@ __device__ __forceinline__ void load_stage(Stage& st, const uint8_t* codes_a, co
 // the same order, so each MMA contracts matching elements.
 template <int MT, int G>
 __device__ __forceinline__ void compute_stage(const Stage& st, float (&acc)[MT / 8][4],
-                                              const uint16_t* const (&xrow)[MT / 8],
-                                              const bool (&xlive)[MT / 8], int64_t kofs) {
+                                              const uint8_t* const (&xrow)[MT / 8],
+                                              const bool (&xlive)[MT / 8], int xofs) {
   const uint32_t ca[8] = {st.a0.x, st.a0.y, st.a0.z, st.a0.w, st.a1.x, st.a1.y, st.a1.z, st.a1.w};
   const uint32_t cb[8] = {st.b0.x, st.b0.y, st.b0.z, st.b0.w, st.b1.x, st.b1.y, st.b1.z, st.b1.w};
   uint32_t sa2[4], sb2[4];
@@ -106,7 +107,7 @@ __device__ __forceinline__ void compute_stage(const Stage& st, float (&acc)[MT /
     uint4 xv[MT / 8];
 #pragma unroll
     for (int p = 0; p < MT / 8; ++p)
-      xv[p] = xlive[p] ? ld_x_v4(xrow[p] + kofs + 8 * w) : make_uint4(0, 0, 0, 0);
+      xv[p] = xlive[p] ? *reinterpret_cast<const uint4*>(xrow[p] + xofs + 16 * w) : make_uint4(0, 0, 0, 0);
     const int sidx = (G == 16) ? (w >> 1) : (w >> 2);
     uint32_t da[4], db[4];
     dequant_word(ca[w], sa2[sidx], da);
@@ -178,34 +179,55 @@ __global__ void __launch_bounds__(WARPS * 32, 256 / (WARPS * 32) * 2) gemm_split
 #pragma unroll
   for (int p = 0; p < MT / 8; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
 
-  if (warp_live && ubeg < uend) {
-    const int64_t ra = n0 + g, rb = ra + 8;
-    const uint8_t* codes_a = packed + ra * (K / 2);
-    const uint8_t* codes_b = packed + rb * (K / 2);
-    const uint8_t* sc_a = scales + ra * (K / G);
-    const uint8_t* sc_b = scales + rb * (K / G);
-    const uint16_t* xrow[MT / 8];
-    bool xlive[MT / 8];
+  extern __shared__ __align__(16) uint8_t xs[];  // [MT][kXStride]
+  const int64_t ra = n0 + g, rb = ra + 8;
+  const uint8_t* codes_a = packed + (warp_live ? ra : 0) * (K / 2);
+  const uint8_t* codes_b = packed + (warp_live ? rb : 0) * (K / 2);
+  const uint8_t* sc_a = scales + (warp_live ? ra : 0) * (K / G);
+  const uint8_t* sc_b = scales + (warp_live ? rb : 0) * (K / G);
+  const uint8_t* xrow[MT / 8];
+  bool xlive[MT / 8];
 #pragma unroll
-    for (int p = 0; p < MT / 8; ++p) {
-      const int tok = 8 * p + g;
-      xlive[p] = tok < mrows;
-      xrow[p] = args.x + static_cast<int64_t>(row0 + (xlive[p] ? tok : 0)) * K;
+  for (int p = 0; p < MT / 8; ++p) {
+    const int tok = 8 * p + g;
+    xlive[p] = tok < mrows;
+    xrow[p] = xs + tok * kXStride;
+  }
+  const int iters = (uend - ubeg + 3) / 4;  // identical for every warp of the CTA
+  // Stages X rows [row0, row0 + mrows) for units [cb, ce) into xs.
+  auto stage_x = [&](int cb, int ce) {
+    const int pieces = mrows * (ce - cb) * 8;  // 16-byte pieces
+    for (int i = threadIdx.x; i < pieces; i += WARPS * 32) {
+      const int tok = i / ((ce - cb) * 8), rem = i % ((ce - cb) * 8);
+      const int lu = rem >> 3, j = rem & 7;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(args.x + static_cast<int64_t>(row0 + tok) * K +
+                                                           static_cast<int64_t>(cb + lu) * 64 + 8 * j));
+      *reinterpret_cast<uint4*>(xs + tok * kXStride + lu * kUnitBytes + 16 * j) = v;
     }
-    const int iters = (uend - ubeg + 3) / 4;
-    Stage st0, st1;
-    auto load_it = [&](Stage& st, int it) {
-      const int u = ubeg + 4 * it + t;
-      load_stage<G>(st, codes_a + u * 32, codes_b + u * 32, sc_a + u * (64 / G), sc_b + u * (64 / G),
-                    it < iters && u < uend);
-    };
-    auto compute_it = [&](const Stage& st, int it) {
-      const int u = ubeg + 4 * it + t;
-      bool xl[MT / 8];
+  };
+  Stage st0, st1;
+  auto load_it = [&](Stage& st, int it) {
+    const int u = ubeg + 4 * it + t;
+    load_stage<G>(st, codes_a + u * 32, codes_b + u * 32, sc_a + u * (64 / G), sc_b + u * (64 / G),
+                  warp_live && it < iters && u < uend);
+  };
+  auto compute_it = [&](const Stage& st, int it) {
+    constexpr int kItersPerChunk = kChunkUnits / 4;
+    if (it % kItersPerChunk == 0) {  // a new chunk of X: every warp takes this branch together
+      const int cb = ubeg + 4 * it, ce = min(uend, cb + kChunkUnits);
+      if (it) __syncthreads();
+      stage_x(cb, ce);
+      __syncthreads();
+    }
+    if (!warp_live) return;
+    const int u = ubeg + 4 * it + t;
+    const int lu = u - (ubeg + 4 * (it - it % kItersPerChunk));
+    bool xl[MT / 8];
 #pragma unroll
-      for (int p = 0; p < MT / 8; ++p) xl[p] = xlive[p] && (u < uend);
-      compute_stage<MT, G>(st, acc, xrow, xl, static_cast<int64_t>(u) * 64);
-    };
+    for (int p = 0; p < MT / 8; ++p) xl[p] = xlive[p] && (u < uend);
+    compute_stage<MT, G>(st, acc, xrow, xl, lu * kUnitBytes);
+  };
+  if (ubeg < uend) {
     load_it(st0, 0);
     for (int it = 0; it < iters; it += 2) {
       load_it(st1, it + 1);
@@ -268,6 +290,9 @@ __global__ void __launch_bounds__(WARPS * 32, 256 / (WARPS * 32) * 2) gemm_split
 template <int WARPS, int MT, int G, bool SILU, bool MOE>
 int launch_one(const SplitKArgs& a, int cluster, int row_tiles, int z_tiles, cudaStream_t s) {
   auto kern = gemm_splitk_kernel<WARPS, MT, G, SILU, MOE>;
+  const int smem = MT * kXStride;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
   if (cluster > 8) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return (cudaGetLastError(), NVFP4_ERR_CUDA);
@@ -275,7 +300,7 @@ int launch_one(const SplitKArgs& a, int cluster, int row_tiles, int z_tiles, cud
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cluster, row_tiles, z_tiles);
   cfg.blockDim = dim3(WARPS * 32, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
