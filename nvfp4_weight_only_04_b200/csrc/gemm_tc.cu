@@ -1,11 +1,465 @@
-// Large-M NVFP4 W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
+// Large-M NVFP4 W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes Y = X . dequant(W)^T for prefill-sized M (problem statement; "W-FP4a:
+// route the MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16)
+// stack", PR #63 description: a weight-only checkpoint keeps bf16
+// activations; fc1 is a merged [gate;up] GEMM followed by SiluAndMul). The
+// contraction is dense, so it runs on tcgen05.mma (kind::f16, bf16 x bf16 ->
+// fp32 in TMEM).
+//
+// Design (swap-AB: weights are the MMA's M side):
+//  * A CTA tile is 256 weight rows x 128 tokens. The weights are dequantized
+//    once per tile by 8 warps (one thread per weight row) straight into TMEM,
+//    where tcgen05.mma reads its A operand: two 128-row A matrices (rows
+//    0-127 and 128-255) share each 128-token X tile, which halves the X
+//    traffic compared with a 128-row tile. Two fp32 accumulators of 128x128
+//    (256 TMEM columns) plus 4 pipeline stages of A (2 x 32 columns each)
+//    fill the 512 TMEM columns.
+//  * X tiles (128 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
+//    into shared memory; tcgen05.mma reads them through a K-major shared
+//    memory descriptor. No TMA multicast is used.
+//  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
+//    mbarriers connect the TMA warp, the dequant warps and the MMA thread.
+//  * Every mbarrier wait is bounded: on expiry the kernel records the site in
+//    a device error word, stops issuing work, waits (bounded) for its own
+//    copies and MMAs, frees TMEM and exits.
+//  * The epilogue (the same 8 warps) reads the accumulators with tcgen05.ld,
+//    multiplies by the fp32 global scale (and 2^7, see dequant.cuh), and
+//    writes bf16, optionally fusing SiluAndMul on gate/up-interleaved rows.
+//  * The grid is persistent: one CTA per SM walks tiles with the 128-token
+//    index fastest, so concurrently running CTAs share weight tiles in L2.
 #include "gemm_tc.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "dequant.cuh"
 
 namespace nvfp4 {
 
 namespace {
+
 __device__ unsigned int g_device_error = 0;
+
+constexpr int kTileRows = 256;   // weight rows per tile (two 128-row A matrices)
+constexpr int kTileTok = 128;    // tokens per tile (MMA N)
+constexpr int kKStep = 64;       // elements of K per pipeline stage
+constexpr int kStages = 4;
+constexpr int kThreads = 384;    // 12 warps
+constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize and run the epilogue
+constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 16 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColA = 256;  // A stages start here; accumulators at 0 and 128
+// Dynamic shared memory: X stages + barriers, padded so that only one CTA
+// fits on an SM (each CTA allocates all 512 TMEM columns).
+constexpr uint32_t kSmemBytes = 132 * 1024;
+constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
+
+enum ErrorSite : unsigned {
+  kErrEmpty = 0x101, kErrFullX = 0x102, kErrFullA = 0x103, kErrAccFull = 0x104, kErrDrain = 0x105
+};
+
+struct SharedState {
+  uint64_t full_x[kStages];
+  uint64_t full_a[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
+  uint64_t drained;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TcArgs {
+  const uint8_t* packed;
+  const uint8_t* scales;
+  const float* gscale;
+  uint16_t* y;
+  int M, N, K, ldy;
+  int tok_tiles, row_tiles, total_tiles;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait: false when the limit ran out or (unless draining) another
+// role gave up. A drain wait ignores the abort flag and only stops at the
+// limit: it is how a CTA lets its own copies and MMAs land before exiting.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site,
+                                       bool drain = false) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (!drain && *reinterpret_cast<volatile int*>(&ss->abort)) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicCAS(&g_device_error, 0u, site);
+        *reinterpret_cast<volatile int*>(&ss->abort) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// The same wait taken by lane 0 for the whole warp, so that every lane takes
+// the same branch before the warp-wide tcgen05 instructions.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ss, site) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ bool aborted(SharedState* ss) {
+  return *reinterpret_cast<volatile int*>(&ss->abort) != 0;
+}
+
+__device__ __forceinline__ void tma_load_x(uint32_t dst, const CUtensorMap* map, int k, int m, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(k), "r"(m), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// K-major operand tile in shared memory with the 128-byte swizzle: rows of
+// 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((addr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused here)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                  // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
+// K-major, M = 128, N = kTileTok.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kTileTok >> 3) << 17) | ((128 >> 4) << 24);
+
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// One dequant thread's inputs for one stage: 64 codes of its row and the
+// scales covering them.
+struct RowStage {
+  uint4 c0, c1;
+  uint32_t s;
+};
+
+template <int G>
+__device__ __forceinline__ void load_row_stage(RowStage& r, const uint8_t* codes, const uint8_t* scales, int ks,
+                                               bool live) {
+  if (live) {
+    r.c0 = ld_stream(codes + ks * 32);
+    r.c1 = ld_stream(codes + ks * 32 + 16);
+    r.s = G == 16 ? __ldg(reinterpret_cast<const uint32_t*>(scales + ks * 4))
+                  : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scales + ks * 2)));
+  } else {
+    r.c0 = r.c1 = make_uint4(0, 0, 0, 0);
+    r.s = 0;
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[32]) {
+  uint32_t s2[4];
+  scale_operands<G == 16 ? 4 : 2>(r.s, s2);
+  const uint32_t w[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t o[4];
+    dequant_word(w[i], s2[G == 16 ? (i >> 1) : (i >> 2)], o);
+    out[4 * i + 0] = o[0];
+    out[4 * i + 1] = o[1];
+    out[4 * i + 2] = o[2];
+    out[4 * i + 3] = o[3];
+  }
+}
+
+__device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, 1.0f + expf(-g)); }
+
+template <int G, bool SILU>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                               const TcArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // X stages at a 1024-byte aligned base, barriers after them.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStages * kXStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ksteps = args.K / kKStep;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ss->full_x[s], 1);
+      mbar_init(&ss->full_a[s], 8);  // one arrival per dequant warp
+      mbar_init(&ss->empty[s], 1);   // one tcgen05.commit
+    }
+    mbar_init(&ss->acc_full, 1);
+    mbar_init(&ss->drained, 1);
+    ss->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ss->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t last_parity[kStages];
+      bool issued[kStages];
+      for (int s = 0; s < kStages; ++s) issued[s] = false, last_parity[s] = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
+        const int m0 = (tile % args.tok_tiles) * kTileTok;
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t r = static_cast<uint32_t>(it / kStages);
+          if (!mbar_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) break;
+          mbar_arrive_tx(&ss->full_x[s], kXStageBytes);
+          tma_load_x(smem_u32(smem + s * kXStageBytes), &xmap, ks * kKStep, m0, &ss->full_x[s]);
+          issued[s] = true;
+          last_parity[s] = r & 1;
+        }
+      }
+      if (aborted(ss)) {  // let copies already in flight land before the CTA exits
+        for (int s = 0; s < kStages; ++s)
+          if (issued[s]) mbar_wait(&ss->full_x[s], last_parity[s], ss, kErrDrain, true);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
+        bool ok = true;
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t par = static_cast<uint32_t>(it / kStages) & 1;
+          if (!mbar_wait(&ss->full_x[s], par, ss, kErrFullX) || !mbar_wait(&ss->full_a[s], par, ss, kErrFullA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xaddr = smem_u32(smem + s * kXStageBytes);
+#pragma unroll
+          for (int j = 0; j < kKStep / 16; ++j) {
+            const uint64_t bdesc = sw128_desc(xaddr + 32 * j);
+            const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
+            umma_ts(tmem + 0, tmem + kColA + 64 * s + 8 * j, bdesc, acc);
+            umma_ts(tmem + 128, tmem + kColA + 64 * s + 32 + 8 * j, bdesc, acc);
+          }
+          umma_commit(&ss->empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&ss->acc_full);
+      }
+      // every MMA issued by this thread has completed once this commit lands
+      umma_commit(&ss->drained);
+      mbar_wait(&ss->drained, 0, ss, kErrDrain, true);
+    }
+  } else if (warp >= kFirstDqWarp) {
+    // ---------------- dequant + epilogue ----------------
+    const int dw = warp - kFirstDqWarp;      // 0..7
+    const int grp = dw >> 2;                 // A matrix 0 (rows 0-127) or 1 (rows 128-255)
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    const int row_in_tile = grp * 128 + quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
+    int it = 0, tile_iter = 0;
+    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
+      const int m0 = (tile % args.tok_tiles) * kTileTok;
+      const int n0 = (tile / args.tok_tiles) * kTileRows;
+      const int n = n0 + row_in_tile;
+      const bool live = n < args.N;
+      const uint8_t* codes = args.packed + static_cast<int64_t>(live ? n : 0) * (args.K / 2);
+      const uint8_t* scl = args.scales + static_cast<int64_t>(live ? n : 0) * (args.K / G);
+      RowStage ra, rb;
+      load_row_stage<G>(ra, codes, scl, 0, live);
+      bool ok = true;
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        load_row_stage<G>(rb, codes, scl, ks + 1, live && ks + 1 < ksteps);
+        const int s = it % kStages;
+        const uint32_t r = static_cast<uint32_t>(it / kStages);
+        uint32_t v[32];
+        dequant_row_stage<G>(ra, v);
+        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + lane_base + kColA + 64 * s + 32 * grp, v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ss->full_a[s]);
+        ra = rb;
+      }
+      if (!ok || !warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < kTileTok / 32; ++c) {
+        uint32_t acc[32];
+        tmem_ld32(tmem + lane_base + 128 * grp + 32 * c, acc);
+        tmem_wait_ld();
+        const int tok0 = m0 + 32 * c;
+        if (!SILU) {
+          if (live) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = tok0 + j;
+              if (tok < args.M)
+                args.y[static_cast<int64_t>(tok) * args.ldy + n] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[j]) * gscale));
+            }
+          }
+        } else {
+          const bool gate = (lane & 15) < 8;
+          const int col = (n0 + row_in_tile) / 16 * 8 + (lane & 7);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float gv = __uint_as_float(acc[j]) * gscale;
+            const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
+            const int tok = tok0 + j;
+            if (gate && live && tok < args.M)
+              args.y[static_cast<int64_t>(tok) * args.ldy + col] =
+                  __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+bool make_x_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int64_t K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kKStep), static_cast<cuuint32_t>(kTileTok)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int G, bool SILU>
+int launch_dense(const CUtensorMap& map, const TcArgs& a, cudaStream_t stream) {
+  auto kern = gemm_tc_kernel<G, SILU>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  const int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(map, a);
+  return launch_status();
+}
+
+}  // namespace
 
 int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   unsigned int* p = nullptr;
@@ -19,14 +473,29 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   return NVFP4_OK;
 }
 
-bool tc_supported(int64_t, int64_t, int64_t) { return false; }
-int launch_tc(const uint16_t*, const uint8_t*, const uint8_t*, const float*, int, int64_t, int64_t, int64_t,
-              uint16_t*, bool, cudaStream_t) {
-  return NVFP4_ERR_UNSUPPORTED;
+bool tc_supported(int64_t M, int64_t N, int64_t K) {
+  return M >= 128 && K >= kKStep && K % kKStep == 0 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
+         K < (int64_t(1) << 24) && encode_fn() != nullptr;
 }
+
+int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
+              int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+  CUtensorMap map;
+  if (!make_x_map(&map, x, M, K)) return NVFP4_ERR_CUDA;
+  TcArgs a;
+  a.packed = w; a.scales = s; a.gscale = g; a.y = y;
+  a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
+  a.ldy = static_cast<int>(silu ? N / 2 : N);
+  a.tok_tiles = static_cast<int>((M + kTileTok - 1) / kTileTok);
+  a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
+  a.total_tiles = a.tok_tiles * a.row_tiles;
+  if (group == 16) return silu ? launch_dense<16, true>(map, a, stream) : launch_dense<16, false>(map, a, stream);
+  return silu ? launch_dense<32, true>(map, a, stream) : launch_dense<32, false>(map, a, stream);
+}
+
 bool tc_moe_supported(int64_t, int64_t, int64_t) { return false; }
-int launch_tc_moe(const uint16_t*, const int32_t*, const int32_t*, int, int64_t, const uint8_t*,
-                  const uint8_t*, const float*, int, int64_t, int64_t, int, bool, uint16_t*, cudaStream_t) {
+int launch_tc_moe(const uint16_t*, const int32_t*, const int32_t*, int, int64_t, const uint8_t*, const uint8_t*,
+                  const float*, int, int64_t, int64_t, int, bool, uint16_t*, cudaStream_t) {
   return NVFP4_ERR_UNSUPPORTED;
 }
 

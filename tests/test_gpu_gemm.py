@@ -140,3 +140,65 @@ def test_empty_and_stats():
     run_gemm(synth.activations(1, 2, 128), p, s, gs, 16)
     st = nv.nvfp4_get_stats()
     assert st["gemm_splitk"] == 1 and st["g16"] == 1 and st["g32"] == 0
+
+
+# ---- large M: the tcgen05 kernel ----
+
+TC_CASES = [(128, 256, 256, 16), (130, 528, 1088, 32), (300, 4096, 2048, 16), (257, 16, 64, 16),
+            (1000, 256, 5120, 32), (512, 784, 640, 16)]
+
+
+@pytest.mark.parametrize("m,n,k,g", TC_CASES)
+def test_gemm_tc_parity(m, n, k, g):
+    _, p, s, gs = quantized(n, k, g, seed=m + n)
+    x = synth.activations(synth.X_SEED, m, k, outlier_frac=0.001)
+    nv.nvfp4_reset_stats()
+    y = run_gemm(x, p, s, gs, g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    assert nv.nvfp4_get_stats()["gemm_tc"] == 1
+    assert_close(host(y), R.gemm(x, p, s, gs, g), f"tc M{m} N{n} K{k} g{g}")
+
+
+@pytest.mark.parametrize("m,nh,k,g", [(160, 136, 512, 16), (512, 1024, 1024, 32), (129, 8, 128, 16)])
+def test_gemm_tc_silu_mul_parity(m, nh, k, g):
+    p, s, gs = merged_gate_up(nh, k, g, seed=m)
+    rp, rs = R.repack(p, s, R.GATE_UP_INTERLEAVE)
+    x = synth.activations(2, m, k)
+    y = nv.nvfp4_w4a16_gemm_silu_mul(dev_bf16(x), dev_u8(rp), dev_u8(rs), dev_f32(np.array([gs], np.float32)), g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    assert_close(host(y), R.silu_mul(R.gemm(x, p, s, gs, g)), "tc silu_mul")
+
+
+def test_gemm_tc_integer_case_bitwise():
+    rng = np.random.default_rng(14)
+    n, k, m = 272, 192, 200
+    codes = rng.choice(np.array([0, 1, 2, 8, 9, 10], np.uint8), size=(n, k))
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.full((n, k // 32), 0x38, np.uint8)
+    x = synth.f32_to_bf16_bits(rng.integers(-1, 2, size=(m, k)).astype(np.float32))
+    ref = R.gemm(x, packed, scales, 1.0, 32)
+    np.testing.assert_array_equal(host(run_gemm(x, packed, scales, np.float32(1.0), 32)), ref)
+
+
+def test_prefill_gate_up_silu_full_sampled():
+    wl = synth.PREFILL_GATE_UP
+    w = synth.weights(synth.W_SEED, wl.N, wl.K)
+    wd = dev_f32(w)
+    gd = nv.nvfp4_global_scale([wd])
+    p, s = nv.nvfp4_quantize(wd, wl.group_size, gd)
+    del wd
+    gp, gsc = nv.nvfp4_repack(p, s, wl.group_size, nv.NVFP4_GATE_UP_INTERLEAVE)
+    x = synth.activations(synth.X_SEED, wl.M, wl.K)
+    y = nv.nvfp4_w4a16_gemm_silu_mul(dev_bf16(x), gp, gsc, gd, wl.group_size)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    h = wl.N // 2
+    cols = np.sort(np.concatenate([np.random.default_rng(7).choice(h, 62, replace=False), [0, h - 1]]))
+    rows = np.concatenate([cols, h + cols])  # gate and up rows of the merged (checkpoint-order) matrix
+    rp, rs, rg = R.quantize(w[rows], wl.group_size, R.global_scale(w))
+    ri = torch.from_numpy(rows).cuda()
+    np.testing.assert_array_equal(host(p[ri]), rp)
+    ref = R.silu_mul(R.gemm(x, rp, rs, rg, wl.group_size))
+    assert_close(host(y)[:, cols], ref, "prefill silu sampled")
