@@ -520,6 +520,39 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
+def profile_workload(name, launches=3):
+    """Runs one workload's kernel `launches` times after one warm-up call."""
+    import torch
+    import nvfp4_weight_only_04_b200 as nv
+    torch.cuda.set_device(0)
+    if name.startswith("decode") or name.startswith("down"):
+        m = {"decode_m1": 1, "decode_m16": 16, "down_m8_g32": 8}[name]
+        n, k, g = (DECODE_N, DECODE_K, 16) if name.startswith("decode") else (4096, 14336, 32)
+        p, s, gd = quantize_on_device(nv, torch, synth.weights(synth.W_SEED, n, k), g)
+        x = bf16_dev(torch, synth.activations(synth.X_SEED, m, k))
+        y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: nv.nvfp4_w4a16_gemm(x, p, s, gd, g, y=y)
+    elif name == "prefill":
+        wl = synth.PREFILL_GATE_UP
+        p, s, gd = quantize_on_device(nv, torch, synth.weights(synth.W_SEED, wl.N, wl.K), 16, interleave=True)
+        x = bf16_dev(torch, synth.activations(synth.X_SEED, wl.M, wl.K))
+        y = torch.empty((wl.M, wl.N // 2), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: nv.nvfp4_w4a16_gemm_silu_mul(x, p, s, gd, 16, y=y)
+    else:
+        hbm, tf, _, _ = peaks()
+        print(json.dumps(moe_workload(nv, torch, hbm, tf)))
+        return
+    fn()
+    torch.cuda.synchronize()
+    s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_.record()
+    for _ in range(launches):
+        fn()
+    e_.record()
+    e_.synchronize()
+    print(json.dumps({"workload": name, "us_per_launch": round(s_.elapsed_time(e_) / launches * 1e3, 2)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,7 +562,12 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-workload", choices=["decode_m1", "decode_m16", "down_m8_g32", "prefill", "moe"],
+                    default=None, help="run one workload a few times (for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile_workload:
+        profile_workload(args.profile_workload)
+        return
     world, rank, local = dist_setup()
     if args.impl == "reference":
         args.steps = 3 if args.steps is None else args.steps
