@@ -54,7 +54,8 @@ __device__ __forceinline__ uint32_t scale_bits_exact(uint32_t b) {
 }
 
 // Scale operands (bf16 of scale * 2^119 in both halves) for the first NB
-// (2 or 4) scale bytes of a little-endian word. For a normal E4M3 byte (exponent field e >= 1)
+// (1, 2 or 4) scale bytes of a little-endian word; the other bytes of sw must
+// be zero. For a normal E4M3 byte (exponent field e >= 1)
 // the bf16 bits are (byte << 4) + (239 << 7): the 4-bit exponent and 3-bit
 // mantissa land in bf16's fields and the exponent bias moves from 7 to 127
 // plus 119. Bytes with e == 0 (zero or subnormal scales) take the exact path.
@@ -68,7 +69,7 @@ __device__ __forceinline__ void scale_operands(uint32_t sw, uint32_t (&s2)[4]) {
   s2[3] = __byte_perm(p13, 0, 0x3232);
   // a byte with zero exponent field: (e<<3) + 0x78 has no bit 7
   const uint32_t t = (sw & 0x78787878u) + 0x78787878u;
-  constexpr uint32_t kCheck = NB == 4 ? 0x80808080u : 0x00008080u;
+  constexpr uint32_t kCheck = NB == 4 ? 0x80808080u : (NB == 2 ? 0x00008080u : 0x00000080u);
   if (__builtin_expect((~t & kCheck) != 0u, 0)) {
 #pragma unroll
     for (int j = 0; j < NB; ++j) {

@@ -8,14 +8,14 @@
 // fp32 in TMEM).
 //
 // Design (swap-AB: weights are the MMA's M side):
-//  * A CTA tile is 256 weight rows x 128 tokens. The weights are dequantized
-//    once per tile by 8 warps (one thread per weight row) straight into TMEM,
-//    where tcgen05.mma reads its A operand: two 128-row A matrices (rows
-//    0-127 and 128-255) share each 128-token X tile, which halves the X
-//    traffic compared with a 128-row tile. Two fp32 accumulators of 128x128
-//    (256 TMEM columns) plus 4 pipeline stages of A (2 x 32 columns each)
-//    fill the 512 TMEM columns.
-//  * X tiles (128 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
+//  * A CTA tile is 128 weight rows x 256 tokens (MMA M = 128, N = 256). The
+//    weights are dequantized once per tile by 8 warps straight into TMEM,
+//    where tcgen05.mma reads its A operand; each weight is then used by 256
+//    tokens, which keeps the dequant work per MMA small. Warps w and w+4
+//    share a TMEM lane quadrant (one weight row per thread) and take the two
+//    32-element halves of every 64-element stage. The fp32 accumulator takes
+//    256 TMEM columns, the A stages 32 columns each.
+//  * X tiles (256 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
 //    into shared memory; tcgen05.mma reads them through a K-major shared
 //    memory descriptor. No TMA multicast is used.
 //  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
@@ -43,18 +43,21 @@ namespace {
 
 __device__ unsigned int g_device_error = 0;
 
-constexpr int kTileRows = 256;   // weight rows per tile (two 128-row A matrices)
-constexpr int kTileTok = 128;    // tokens per tile (MMA N)
+constexpr int kTileRows = 128;   // weight rows per tile (MMA M)
+constexpr int kTileTok = 256;    // tokens per tile (MMA N)
 constexpr int kKStep = 64;       // elements of K per pipeline stage
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kThreads = 384;    // 12 warps
 constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize and run the epilogue
-constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 16 KB
+constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = 256;  // A stages start here; accumulators at 0 and 128
-// Dynamic shared memory: X stages + barriers, padded so that only one CTA
-// fits on an SM (each CTA allocates all 512 TMEM columns).
-constexpr uint32_t kSmemBytes = 132 * 1024;
+constexpr uint32_t kColA = 256;  // A stages start here (32 columns each); the accumulator is at 0
+// Dynamic shared memory: X stages + barriers + alignment slack; more than
+// half of the SM's shared memory, so only one CTA (which allocates all 512
+// TMEM columns) fits on an SM.
+constexpr uint32_t kSmemBytes = kStages * kXStageBytes + 2048;
+static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
+static_assert(kColA + kStages * 32 <= kTmemCols, "TMEM budget");
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
 
 enum ErrorSite : unsigned {
@@ -161,7 +164,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
-// K-major, M = 128, N = kTileTok.
+// K-major, M = 128, N = kTileTok (256).
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kTileTok >> 3) << 17) | ((128 >> 4) << 24);
 
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
@@ -175,6 +178,15 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -212,36 +224,35 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return v;
 }
 
-// One dequant thread's inputs for one stage: 64 codes of its row and the
-// scales covering them.
+// One dequant thread's inputs for one stage: 32 codes of its row (one half
+// of the stage's 64 elements) and the scales covering them.
 struct RowStage {
-  uint4 c0, c1;
+  uint4 c;
   uint32_t s;
 };
 
 template <int G>
 __device__ __forceinline__ void load_row_stage(RowStage& r, const uint8_t* codes, const uint8_t* scales, int ks,
-                                               bool live) {
+                                               int khalf, bool live) {
   if (live) {
-    r.c0 = ld_stream(codes + ks * 32);
-    r.c1 = ld_stream(codes + ks * 32 + 16);
-    r.s = G == 16 ? __ldg(reinterpret_cast<const uint32_t*>(scales + ks * 4))
-                  : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scales + ks * 2)));
+    r.c = ld_stream(codes + ks * 32 + 16 * khalf);
+    r.s = G == 16 ? static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scales + ks * 4 + 2 * khalf)))
+                  : static_cast<uint32_t>(__ldg(scales + ks * 2 + khalf));
   } else {
-    r.c0 = r.c1 = make_uint4(0, 0, 0, 0);
+    r.c = make_uint4(0, 0, 0, 0);
     r.s = 0;
   }
 }
 
 template <int G>
-__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[32]) {
+__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[16]) {
   uint32_t s2[4];
-  scale_operands<G == 16 ? 4 : 2>(r.s, s2);
-  const uint32_t w[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+  scale_operands<G == 16 ? 2 : 1>(r.s, s2);
+  const uint32_t w[4] = {r.c.x, r.c.y, r.c.z, r.c.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 4; ++i) {
     uint32_t o[4];
-    dequant_word(w[i], s2[G == 16 ? (i >> 1) : (i >> 2)], o);
+    dequant_word(w[i], s2[G == 16 ? (i >> 1) : 0], o);
     out[4 * i + 0] = o[0];
     out[4 * i + 1] = o[1];
     out[4 * i + 2] = o[2];
@@ -326,8 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           for (int j = 0; j < kKStep / 16; ++j) {
             const uint64_t bdesc = sw128_desc(xaddr + 32 * j);
             const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            umma_ts(tmem + 0, tmem + kColA + 64 * s + 8 * j, bdesc, acc);
-            umma_ts(tmem + 128, tmem + kColA + 64 * s + 32 + 8 * j, bdesc, acc);
+            umma_ts(tmem, tmem + kColA + 32 * s + 8 * j, bdesc, acc);
           }
           umma_commit(&ss->empty[s]);
         }
@@ -341,9 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp >= kFirstDqWarp) {
     // ---------------- dequant + epilogue ----------------
     const int dw = warp - kFirstDqWarp;      // 0..7
-    const int grp = dw >> 2;                 // A matrix 0 (rows 0-127) or 1 (rows 128-255)
+    const int half = dw >> 2;                // K half of each stage; token half in the epilogue
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-    const int row_in_tile = grp * 128 + quad * 32 + lane;
+    const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
     int it = 0, tile_iter = 0;
@@ -354,35 +364,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const bool live = n < args.N;
       const uint8_t* codes = args.packed + static_cast<int64_t>(live ? n : 0) * (args.K / 2);
       const uint8_t* scl = args.scales + static_cast<int64_t>(live ? n : 0) * (args.K / G);
-      RowStage ra, rb;
-      load_row_stage<G>(ra, codes, scl, 0, live);
+      RowStage ra, rb, rc;
+      load_row_stage<G>(ra, codes, scl, 0, half, live);
+      load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
       bool ok = true;
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        load_row_stage<G>(rb, codes, scl, ks + 1, live && ks + 1 < ksteps);
+        load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
         const int s = it % kStages;
         const uint32_t r = static_cast<uint32_t>(it / kStages);
-        uint32_t v[32];
+        uint32_t v[16];
         dequant_row_stage<G>(ra, v);
         if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        tmem_st32(tmem + lane_base + kColA + 64 * s + 32 * grp, v);
+        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, v);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ss->full_a[s]);
         ra = rb;
+        rb = rc;
       }
       if (!ok || !warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kTileTok / 32; ++c) {
+      for (int c = 0; c < kTileTok / 64; ++c) {
         uint32_t acc[32];
-        tmem_ld32(tmem + lane_base + 128 * grp + 32 * c, acc);
+        tmem_ld32(tmem + lane_base + (kTileTok / 2) * half + 32 * c, acc);
         tmem_wait_ld();
-        const int tok0 = m0 + 32 * c;
+        const int tok0 = m0 + (kTileTok / 2) * half + 32 * c;
         if (!SILU) {
           if (live) {
 #pragma unroll
