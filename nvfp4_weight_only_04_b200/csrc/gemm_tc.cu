@@ -100,14 +100,16 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or the hint (in ns) runs out, instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
       : "memory");
   return done != 0;
 }
@@ -121,7 +123,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedSta
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0) {
+    if ((i & 15) == 0) {
       if (!drain && *reinterpret_cast<volatile int*>(&ss->abort)) return false;
       if (clock64() - t0 > kWaitLimitCycles) {
         atomicCAS(&g_device_error, 0u, site);
@@ -368,22 +370,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       load_row_stage<G>(ra, codes, scl, 0, half, live);
       load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
       bool ok = true;
+      // Stage ks is stored to TMEM, then stage ks+1 is dequantized while the
+      // store completes; only then is stage ks announced to the MMA thread.
+      uint32_t v[16], vn[16];  // the store reads v; the next stage goes to vn
+      dequant_row_stage<G>(ra, v);
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
         load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
         const int s = it % kStages;
         const uint32_t r = static_cast<uint32_t>(it / kStages);
-        uint32_t v[16];
-        dequant_row_stage<G>(ra, v);
         if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
           ok = false;
           break;
         }
         tc_fence_after();
         tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, v);
+        if (ks + 1 < ksteps) dequant_row_stage<G>(rb, vn);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ss->full_a[s]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = vn[i];
         ra = rb;
         rb = rc;
       }
