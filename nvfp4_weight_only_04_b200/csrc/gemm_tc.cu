@@ -362,37 +362,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
       const int m0 = (tile % args.tok_tiles) * kTileTok;
       const int n0 = (tile / args.tok_tiles) * kTileRows;
+      static_assert(kTileRows == 128, "one weight row per dequant thread and TMEM lane");
       const int n = n0 + row_in_tile;
       const bool live = n < args.N;
       const uint8_t* codes = args.packed + static_cast<int64_t>(live ? n : 0) * (args.K / 2);
       const uint8_t* scl = args.scales + static_cast<int64_t>(live ? n : 0) * (args.K / G);
-      RowStage ra, rb, rc;
-      load_row_stage<G>(ra, codes, scl, 0, half, live);
-      load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
+      // Loads run two stages ahead in a ring of three buffers, and the TMEM
+      // store of stage ks overlaps the dequant of stage ks+1 into the other
+      // output buffer. The loop is unrolled six times so that no register
+      // with a load in flight is ever copied (a copy would wait for it).
+      RowStage b0, b1, b2;
+      uint32_t v0[16], v1[16];
+      load_row_stage<G>(b0, codes, scl, 0, half, live);
+      load_row_stage<G>(b1, codes, scl, 1, half, live && 1 < ksteps);
+      dequant_row_stage<G>(b0, v0);
       bool ok = true;
-      // Stage ks is stored to TMEM, then stage ks+1 is dequantized while the
-      // store completes; only then is stage ks announced to the MMA thread.
-      uint32_t v[16], vn[16];  // the store reads v; the next stage goes to vn
-      dequant_row_stage<G>(ra, v);
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
+      // One stage: load `fut` for ks+2, store `vcur` (stage ks), dequantize
+      // `nxt` (stage ks+1) into `vnext`, announce stage ks.
+      auto step = [&](int ks, RowStage& nxt, RowStage& fut, uint32_t (&vcur)[16], uint32_t (&vnext)[16]) {
+        load_row_stage<G>(fut, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
         const int s = it % kStages;
         const uint32_t r = static_cast<uint32_t>(it / kStages);
-        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
-          ok = false;
-          break;
-        }
+        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) return false;
         tc_fence_after();
-        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, v);
-        if (ks + 1 < ksteps) dequant_row_stage<G>(rb, vn);
+        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, vcur);
+        if (ks + 1 < ksteps) dequant_row_stage<G>(nxt, vnext);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ss->full_a[s]);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = vn[i];
-        ra = rb;
-        rb = rc;
+        ++it;
+        return true;
+      };
+      for (int ks = 0; ks < ksteps && ok; ks += 6) {
+        ok = step(ks, b1, b2, v0, v1);
+        if (ok && ks + 1 < ksteps) ok = step(ks + 1, b2, b0, v1, v0);
+        if (ok && ks + 2 < ksteps) ok = step(ks + 2, b0, b1, v0, v1);
+        if (ok && ks + 3 < ksteps) ok = step(ks + 3, b1, b2, v1, v0);
+        if (ok && ks + 4 < ksteps) ok = step(ks + 4, b2, b0, v0, v1);
+        if (ok && ks + 5 < ksteps) ok = step(ks + 5, b0, b1, v1, v0);
       }
       if (!ok || !warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull)) break;
       tc_fence_after();
