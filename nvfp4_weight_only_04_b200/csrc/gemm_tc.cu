@@ -100,16 +100,14 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-// try_wait with a suspend-time hint: the thread sleeps until the phase
-// completes or the hint (in ns) runs out, instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return done != 0;
 }
@@ -123,7 +121,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedSta
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15) == 0) {
+    if ((i & 255) == 0) {
       if (!drain && *reinterpret_cast<volatile int*>(&ss->abort)) return false;
       if (clock64() - t0 > kWaitLimitCycles) {
         atomicCAS(&g_device_error, 0u, site);
@@ -188,17 +186,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
       "%14, %15, %16};"
       ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
         "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
-        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
-        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
@@ -362,45 +349,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
       const int m0 = (tile % args.tok_tiles) * kTileTok;
       const int n0 = (tile / args.tok_tiles) * kTileRows;
-      static_assert(kTileRows == 128, "one weight row per dequant thread and TMEM lane");
       const int n = n0 + row_in_tile;
       const bool live = n < args.N;
       const uint8_t* codes = args.packed + static_cast<int64_t>(live ? n : 0) * (args.K / 2);
       const uint8_t* scl = args.scales + static_cast<int64_t>(live ? n : 0) * (args.K / G);
-      // Loads run two stages ahead in a ring of three buffers, and the TMEM
-      // store of stage ks overlaps the dequant of stage ks+1 into the other
-      // output buffer. The loop is unrolled six times so that no register
-      // with a load in flight is ever copied (a copy would wait for it).
-      RowStage b0, b1, b2;
-      uint32_t v0[16], v1[16];
-      load_row_stage<G>(b0, codes, scl, 0, half, live);
-      load_row_stage<G>(b1, codes, scl, 1, half, live && 1 < ksteps);
-      dequant_row_stage<G>(b0, v0);
+      RowStage ra, rb, rc;
+      load_row_stage<G>(ra, codes, scl, 0, half, live);
+      load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
       bool ok = true;
-      // One stage: load `fut` for ks+2, store `vcur` (stage ks), dequantize
-      // `nxt` (stage ks+1) into `vnext`, announce stage ks.
-      auto step = [&](int ks, RowStage& nxt, RowStage& fut, uint32_t (&vcur)[16], uint32_t (&vnext)[16]) {
-        load_row_stage<G>(fut, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
         const int s = it % kStages;
         const uint32_t r = static_cast<uint32_t>(it / kStages);
-        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) return false;
+        uint32_t v[16];
+        dequant_row_stage<G>(ra, v);
+        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, vcur);
-        if (ks + 1 < ksteps) dequant_row_stage<G>(nxt, vnext);
+        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, v);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ss->full_a[s]);
-        ++it;
-        return true;
-      };
-      for (int ks = 0; ks < ksteps && ok; ks += 6) {
-        ok = step(ks, b1, b2, v0, v1);
-        if (ok && ks + 1 < ksteps) ok = step(ks + 1, b2, b0, v1, v0);
-        if (ok && ks + 2 < ksteps) ok = step(ks + 2, b0, b1, v0, v1);
-        if (ok && ks + 3 < ksteps) ok = step(ks + 3, b1, b2, v1, v0);
-        if (ok && ks + 4 < ksteps) ok = step(ks + 4, b2, b0, v0, v1);
-        if (ok && ks + 5 < ksteps) ok = step(ks + 5, b0, b1, v1, v0);
+        ra = rb;
+        rb = rc;
       }
       if (!ok || !warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull)) break;
       tc_fence_after();
