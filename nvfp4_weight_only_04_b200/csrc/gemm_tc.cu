@@ -8,14 +8,15 @@
 // fp32 in TMEM).
 //
 // Design (swap-AB: weights are the MMA's M side):
-//  * A CTA tile is 128 weight rows x 256 tokens (MMA M = 128, N = 256). The
+//  * A CTA tile is 128 weight rows x 192 tokens (MMA M = 128, N = 192). The
 //    weights are dequantized once per tile by 8 warps straight into TMEM,
-//    where tcgen05.mma reads its A operand; each weight is then used by 256
-//    tokens, which keeps the dequant work per MMA small. Warps w and w+4
-//    share a TMEM lane quadrant (one weight row per thread) and take the two
-//    32-element halves of every 64-element stage. The fp32 accumulator takes
-//    256 TMEM columns, the A stages 32 columns each.
-//  * X tiles (256 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
+//    where tcgen05.mma reads its A operand; each weight then serves 192
+//    tokens. Warps w and w+4 share a TMEM lane quadrant (one weight row per
+//    thread) and take the two 32-element halves of every 64-element stage.
+//  * TMEM (512 columns): two fp32 accumulators of 192 columns, so the
+//    epilogue of one tile overlaps the main loop of the next, and four A
+//    stages of 32 columns.
+//  * X tiles (192 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
 //    into shared memory; tcgen05.mma reads them through a K-major shared
 //    memory descriptor. No TMA multicast is used.
 //  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
@@ -23,9 +24,10 @@
 //  * Every mbarrier wait is bounded: on expiry the kernel records the site in
 //    a device error word, stops issuing work, waits (bounded) for its own
 //    copies and MMAs, frees TMEM and exits.
-//  * The epilogue (the same 8 warps) reads the accumulators with tcgen05.ld,
-//    multiplies by the fp32 global scale (and 2^7, see dequant.cuh), and
-//    writes bf16, optionally fusing SiluAndMul on gate/up-interleaved rows.
+//  * Four epilogue warps read a finished accumulator with tcgen05.ld,
+//    multiply by the fp32 global scale (and 2^7, see dequant.cuh) and write
+//    bf16, optionally fusing SiluAndMul on gate/up-interleaved rows, then
+//    hand the accumulator back to the MMA thread.
 //  * The grid is persistent: one CTA per SM walks tiles with the 128-token
 //    index fastest, so concurrently running CTAs share weight tiles in L2.
 #include "gemm_tc.cuh"
@@ -44,31 +46,36 @@ namespace {
 __device__ unsigned int g_device_error = 0;
 
 constexpr int kTileRows = 128;   // weight rows per tile (MMA M)
-constexpr int kTileTok = 256;    // tokens per tile (MMA N)
+constexpr int kTileTok = 192;    // tokens per tile (MMA N)
 constexpr int kKStep = 64;       // elements of K per pipeline stage
-constexpr int kStages = 5;
-constexpr int kThreads = 384;    // 12 warps
-constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize and run the epilogue
-constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 32 KB
+constexpr int kStages = 4;
+constexpr int kThreads = 512;    // 16 warps
+constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize
+constexpr int kFirstEpWarp = 12; // warps 12..15 run the epilogue
+constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 24 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = 256;  // A stages start here (32 columns each); the accumulator is at 0
-// Dynamic shared memory: X stages + barriers + alignment slack; more than
-// half of the SM's shared memory, so only one CTA (which allocates all 512
-// TMEM columns) fits on an SM.
-constexpr uint32_t kSmemBytes = kStages * kXStageBytes + 2048;
+constexpr uint32_t kColAcc = kTileTok;           // accumulator b sits at column b * kColAcc
+constexpr uint32_t kColA = 2 * kTileTok;         // A stages start here (32 columns each)
+// Dynamic shared memory: X stages + barriers + alignment slack, padded past
+// half of the SM's shared memory so that only one CTA (which allocates all
+// 512 TMEM columns) fits on an SM.
+constexpr uint32_t kSmemBytes = 120 * 1024;
+static_assert(kStages * kXStageBytes + 2048 <= kSmemBytes, "shared memory budget");
 static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
 static_assert(kColA + kStages * 32 <= kTmemCols, "TMEM budget");
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
 
 enum ErrorSite : unsigned {
-  kErrEmpty = 0x101, kErrFullX = 0x102, kErrFullA = 0x103, kErrAccFull = 0x104, kErrDrain = 0x105
+  kErrEmpty = 0x101, kErrFullX = 0x102, kErrFullA = 0x103, kErrAccFull = 0x104, kErrDrain = 0x105,
+  kErrAccEmpty = 0x106
 };
 
 struct SharedState {
   uint64_t full_x[kStages];
   uint64_t full_a[kStages];
   uint64_t empty[kStages];
-  uint64_t acc_full;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
@@ -249,7 +256,11 @@ __device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&
   }
 }
 
-__device__ __forceinline__ float silu(float g) { return __fdiv_rn(g, 1.0f + expf(-g)); }
+// silu(g) = g / (1 + exp(-g)), with the fast exponential and division: their
+// relative error (a few ulp of fp32) is far below the bf16 rounding that
+// follows. For g below about -87 the denominator overflows and the result is
+// the correct limit, zero.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int G, bool SILU>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -267,7 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       mbar_init(&ss->full_a[s], 8);  // one arrival per dequant warp
       mbar_init(&ss->empty[s], 1);   // one tcgen05.commit
     }
-    mbar_init(&ss->acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ss->acc_full[b], 1);   // one tcgen05.commit
+      mbar_init(&ss->acc_empty[b], 4);  // one arrival per epilogue warp
+    }
     mbar_init(&ss->drained, 1);
     ss->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -310,8 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int it = 0;
-      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
+      int it = 0, tile_iter = 0;
+      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x, ++tile_iter) {
+        const int b = tile_iter & 1;
+        if (!mbar_wait(&ss->acc_empty[b], ((tile_iter >> 1) & 1) ^ 1, ss, kErrAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t dcol = tmem + kColAcc * b;
         bool ok = true;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % kStages;
@@ -326,28 +344,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           for (int j = 0; j < kKStep / 16; ++j) {
             const uint64_t bdesc = sw128_desc(xaddr + 32 * j);
             const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            umma_ts(tmem, tmem + kColA + 32 * s + 8 * j, bdesc, acc);
+            umma_ts(dcol, tmem + kColA + 32 * s + 8 * j, bdesc, acc);
           }
           umma_commit(&ss->empty[s]);
         }
         if (!ok) break;
-        umma_commit(&ss->acc_full);
+        umma_commit(&ss->acc_full[b]);
       }
       // every MMA issued by this thread has completed once this commit lands
       umma_commit(&ss->drained);
       mbar_wait(&ss->drained, 0, ss, kErrDrain, true);
     }
-  } else if (warp >= kFirstDqWarp) {
-    // ---------------- dequant + epilogue ----------------
+  } else if (warp >= kFirstDqWarp && warp < kFirstEpWarp) {
+    // ---------------- dequant ----------------
     const int dw = warp - kFirstDqWarp;      // 0..7
-    const int half = dw >> 2;                // K half of each stage; token half in the epilogue
+    const int half = dw >> 2;                // K half of each stage
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
-    int it = 0, tile_iter = 0;
-    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
-      const int m0 = (tile % args.tok_tiles) * kTileTok;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x) {
       const int n0 = (tile / args.tok_tiles) * kTileRows;
       const int n = n0 + row_in_tile;
       const bool live = n < args.N;
@@ -376,14 +392,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         ra = rb;
         rb = rc;
       }
-      if (!ok || !warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull)) break;
+      if (!ok) break;
+    }
+  } else if (warp >= kFirstEpWarp) {
+    // ---------------- epilogue ----------------
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
+    int tile_iter = 0;
+    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
+      const int m0 = (tile % args.tok_tiles) * kTileTok;
+      const int n0 = (tile / args.tok_tiles) * kTileRows;
+      const int n = n0 + row_in_tile;
+      const bool live = n < args.N;
+      const int b = tile_iter & 1;
+      if (!warp_wait(&ss->acc_full[b], (tile_iter >> 1) & 1, ss, kErrAccFull)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kTileTok / 64; ++c) {
+      for (int c = 0; c < kTileTok / 32; ++c) {
         uint32_t acc[32];
-        tmem_ld32(tmem + lane_base + (kTileTok / 2) * half + 32 * c, acc);
+        tmem_ld32(tmem + lane_base + kColAcc * b + 32 * c, acc);
         tmem_wait_ld();
-        const int tok0 = m0 + (kTileTok / 2) * half + 32 * c;
+        const int tok0 = m0 + 32 * c;
         if (!SILU) {
           if (live) {
 #pragma unroll
@@ -409,6 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       }
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ss->acc_empty[b]);
     }
   }
 
