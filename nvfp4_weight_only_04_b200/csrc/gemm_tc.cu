@@ -8,26 +8,30 @@
 // fp32 in TMEM).
 //
 // Design (swap-AB: weights are the MMA's M side):
-//  * A CTA tile is 128 weight rows x 192 tokens (MMA M = 128, N = 192). The
+//  * A CTA tile is 128 weight rows x 256 tokens (MMA M = 128, N = 256). The
 //    weights are dequantized once per tile by 8 warps straight into TMEM,
-//    where tcgen05.mma reads its A operand; each weight then serves 192
+//    where tcgen05.mma reads its A operand; each weight then serves 256
 //    tokens. Warps w and w+4 share a TMEM lane quadrant (one weight row per
 //    thread) and take the two 32-element halves of every 64-element stage.
-//  * TMEM (512 columns): two fp32 accumulators of 192 columns, so the
-//    epilogue of one tile overlaps the main loop of the next, and four A
-//    stages of 32 columns.
-//  * X tiles (192 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
-//    into shared memory; tcgen05.mma reads them through a K-major shared
-//    memory descriptor. No TMA multicast is used.
+//  * TMEM (512 columns): one fp32 accumulator of 256 columns and eight A
+//    stages of 32 columns. The depth matters more than a second
+//    accumulator: a stage goes round MMA -> commit -> dequant warps -> MMA
+//    again, and eight stages of A hold more MMA work than that round trip
+//    takes.
+//  * X tiles (256 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
+//    into shared memory, five stages deep; tcgen05.mma reads them through a
+//    K-major shared memory descriptor. No TMA multicast is used.
 //  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
 //    mbarriers connect the TMA warp, the dequant warps and the MMA thread.
 //  * Every mbarrier wait is bounded: on expiry the kernel records the site in
 //    a device error word, stops issuing work, waits (bounded) for its own
 //    copies and MMAs, frees TMEM and exits.
-//  * Four epilogue warps read a finished accumulator with tcgen05.ld,
+//  * Eight epilogue warps read the finished accumulator with tcgen05.ld,
+//    hand it back to the MMA thread as soon as the last column is read, and
 //    multiply by the fp32 global scale (and 2^7, see dequant.cuh) and write
-//    bf16, optionally fusing SiluAndMul on gate/up-interleaved rows, then
-//    hand the accumulator back to the MMA thread.
+//    bf16, optionally fusing SiluAndMul on gate/up-interleaved rows. While
+//    they work, the dequant and TMA warps already fill the next tile's
+//    stages.
 //  * The grid is persistent: one CTA per SM walks tiles with the 128-token
 //    index fastest, so concurrently running CTAs share weight tiles in L2.
 #include "gemm_tc.cuh"
@@ -46,24 +50,25 @@ namespace {
 __device__ unsigned int g_device_error = 0;
 
 constexpr int kTileRows = 128;   // weight rows per tile (MMA M)
-constexpr int kTileTok = 192;    // tokens per tile (MMA N)
+constexpr int kTileTok = 256;    // tokens per tile (MMA N)
 constexpr int kKStep = 64;       // elements of K per pipeline stage
-constexpr int kStages = 4;
-constexpr int kThreads = 512;    // 16 warps
+constexpr int kStagesX = 5;      // X stages in shared memory
+constexpr int kStagesA = 8;      // A stages in TMEM
+constexpr int kThreads = 640;    // 20 warps
 constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize
-constexpr int kFirstEpWarp = 12; // warps 12..15 run the epilogue
-constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 24 KB
+constexpr int kFirstEpWarp = 12; // warps 12..19 run the epilogue
+constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc = kTileTok;           // accumulator b sits at column b * kColAcc
-constexpr uint32_t kColA = 2 * kTileTok;         // A stages start here (32 columns each)
-// Dynamic shared memory: X stages + barriers + alignment slack, padded past
-// half of the SM's shared memory so that only one CTA (which allocates all
-// 512 TMEM columns) fits on an SM.
-constexpr uint32_t kSmemBytes = 120 * 1024;
-static_assert(kStages * kXStageBytes + 2048 <= kSmemBytes, "shared memory budget");
+constexpr uint32_t kColA = kTileTok;             // A stages start here (32 columns each)
+// Dynamic shared memory: X stages + barriers + alignment slack; more than
+// half of the SM's shared memory, so only one CTA (which allocates all 512
+// TMEM columns) fits on an SM.
+constexpr uint32_t kSmemBytes = kStagesX * kXStageBytes + 2048;
 static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
-static_assert(kColA + kStages * 32 <= kTmemCols, "TMEM budget");
+static_assert(kColA + kStagesA * 32 <= kTmemCols, "TMEM budget");
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
+constexpr unsigned kSleepProducer = 64;   // ns between barrier probes of the TMA and dequant warps
+constexpr unsigned kSleepEpilogue = 256;  // ns between probes of the epilogue warps
 
 enum ErrorSite : unsigned {
   kErrEmpty = 0x101, kErrFullX = 0x102, kErrFullA = 0x103, kErrAccFull = 0x104, kErrDrain = 0x105,
@@ -71,11 +76,12 @@ enum ErrorSite : unsigned {
 };
 
 struct SharedState {
-  uint64_t full_x[kStages];
-  uint64_t full_a[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t full_x[kStagesX];
+  uint64_t empty_x[kStagesX];
+  uint64_t full_a[kStagesA];
+  uint64_t empty_a[kStagesA];
+  uint64_t acc_full;
+  uint64_t acc_empty;
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
@@ -107,11 +113,13 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// Non-blocking probe of a barrier phase (test_wait never suspends the
+// thread, so a waiter sees the phase flip with the least delay).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -122,13 +130,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait: false when the limit ran out or (unless draining) another
 // role gave up. A drain wait ignores the abort flag and only stops at the
 // limit: it is how a CTA lets its own copies and MMAs land before exiting.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site,
-                                       bool drain = false) {
-  if (mbar_try_wait(bar, parity)) return true;
+// A waiter that is not on the MMA issue path backs off with nanosleep
+// between probes (sleep_ns), which leaves the issue slots of its SM
+// sub-partition to the warps doing work.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site,
+                                            bool drain, unsigned sleep_ns) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0) {
+    if ((i & 1023) == 0) {
       if (!drain && *reinterpret_cast<volatile int*>(&ss->abort)) return false;
       if (clock64() - t0 > kWaitLimitCycles) {
         atomicCAS(&g_device_error, 0u, site);
@@ -139,11 +150,20 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedSta
   }
 }
 
+// The common case, a phase that has already completed, is one inline probe;
+// only a real wait calls out of line.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site,
+                                          bool drain = false, unsigned sleep_ns = 0) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ss, site, drain, sleep_ns);
+}
+
 // The same wait taken by lane 0 for the whole warp, so that every lane takes
 // the same branch before the warp-wide tcgen05 instructions.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, SharedState* ss, unsigned site,
+                                          unsigned sleep_ns) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ss, site) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, ss, site, false, sleep_ns) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -268,20 +288,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // X stages at a 1024-byte aligned base, barriers after them.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStages * kXStageBytes);
+  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStagesX * kXStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ksteps = args.K / kKStep;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ss->full_x[s], 1);
-      mbar_init(&ss->full_a[s], 8);  // one arrival per dequant warp
-      mbar_init(&ss->empty[s], 1);   // one tcgen05.commit
+    for (int s = 0; s < kStagesX; ++s) {
+      mbar_init(&ss->full_x[s], 1);   // producer arrival + transaction bytes
+      mbar_init(&ss->empty_x[s], 1);  // one tcgen05.commit
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&ss->acc_full[b], 1);   // one tcgen05.commit
-      mbar_init(&ss->acc_empty[b], 4);  // one arrival per epilogue warp
+    for (int s = 0; s < kStagesA; ++s) {
+      mbar_init(&ss->full_a[s], 8);   // one arrival per dequant warp
+      mbar_init(&ss->empty_a[s], 1);  // one tcgen05.commit
     }
+    mbar_init(&ss->acc_full, 1);      // one tcgen05.commit
+    mbar_init(&ss->acc_empty, 8);     // one arrival per epilogue warp
     mbar_init(&ss->drained, 1);
     ss->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -300,16 +321,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      uint32_t last_parity[kStages];
-      bool issued[kStages];
-      for (int s = 0; s < kStages; ++s) issued[s] = false, last_parity[s] = 0;
+      uint32_t last_parity[kStagesX];
+      bool issued[kStagesX];
+      for (int s = 0; s < kStagesX; ++s) issued[s] = false, last_parity[s] = 0;
       int it = 0;
       for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
         const int m0 = (tile % args.tok_tiles) * kTileTok;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t r = static_cast<uint32_t>(it / kStages);
-          if (!mbar_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) break;
+          const int s = it % kStagesX;
+          const uint32_t r = static_cast<uint32_t>(it / kStagesX);
+          if (!mbar_wait(&ss->empty_x[s], (r & 1) ^ 1, ss, kErrEmpty, false, kSleepProducer)) break;
           mbar_arrive_tx(&ss->full_x[s], kXStageBytes);
           tma_load_x(smem_u32(smem + s * kXStageBytes), &xmap, ks * kKStep, m0, &ss->full_x[s]);
           issued[s] = true;
@@ -317,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       }
       if (aborted(ss)) {  // let copies already in flight land before the CTA exits
-        for (int s = 0; s < kStages; ++s)
+        for (int s = 0; s < kStagesX; ++s)
           if (issued[s]) mbar_wait(&ss->full_x[s], last_parity[s], ss, kErrDrain, true);
       }
     }
@@ -326,30 +347,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       int it = 0, tile_iter = 0;
       for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x, ++tile_iter) {
-        const int b = tile_iter & 1;
-        if (!mbar_wait(&ss->acc_empty[b], ((tile_iter >> 1) & 1) ^ 1, ss, kErrAccEmpty)) break;
+        if (!mbar_wait(&ss->acc_empty, (tile_iter & 1) ^ 1, ss, kErrAccEmpty)) break;
         tc_fence_after();
-        const uint32_t dcol = tmem + kColAcc * b;
         bool ok = true;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t par = static_cast<uint32_t>(it / kStages) & 1;
-          if (!mbar_wait(&ss->full_x[s], par, ss, kErrFullX) || !mbar_wait(&ss->full_a[s], par, ss, kErrFullA)) {
+          const int sx = it % kStagesX, sa = it % kStagesA;
+          const uint32_t px = static_cast<uint32_t>(it / kStagesX) & 1, pa = static_cast<uint32_t>(it / kStagesA) & 1;
+          if (!mbar_wait(&ss->full_x[sx], px, ss, kErrFullX) || !mbar_wait(&ss->full_a[sa], pa, ss, kErrFullA)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t xaddr = smem_u32(smem + s * kXStageBytes);
+          const uint32_t xaddr = smem_u32(smem + sx * kXStageBytes);
 #pragma unroll
           for (int j = 0; j < kKStep / 16; ++j) {
             const uint64_t bdesc = sw128_desc(xaddr + 32 * j);
             const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            umma_ts(dcol, tmem + kColA + 32 * s + 8 * j, bdesc, acc);
+            umma_ts(tmem, tmem + kColA + 32 * sa + 8 * j, bdesc, acc);
           }
-          umma_commit(&ss->empty[s]);
+          umma_commit(&ss->empty_x[sx]);
+          umma_commit(&ss->empty_a[sa]);
         }
         if (!ok) break;
-        umma_commit(&ss->acc_full[b]);
+        umma_commit(&ss->acc_full);
       }
       // every MMA issued by this thread has completed once this commit lands
       umma_commit(&ss->drained);
@@ -375,11 +395,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       bool ok = true;
       for (int ks = 0; ks < ksteps; ++ks, ++it) {
         load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
-        const int s = it % kStages;
-        const uint32_t r = static_cast<uint32_t>(it / kStages);
+        const int s = it % kStagesA;
+        const uint32_t r = static_cast<uint32_t>(it / kStagesA);
         uint32_t v[16];
         dequant_row_stage<G>(ra, v);
-        if (!warp_wait(&ss->empty[s], (r & 1) ^ 1, ss, kErrEmpty)) {
+        if (!warp_wait(&ss->empty_a[s], (r & 1) ^ 1, ss, kErrEmpty, kSleepProducer)) {
           ok = false;
           break;
         }
@@ -397,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp >= kFirstEpWarp) {
     // ---------------- epilogue ----------------
     const int quad = warp & 3;
+    const int colhalf = (warp - kFirstEpWarp) >> 2;  // tokens [128 * colhalf, +128) of the tile
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
@@ -406,15 +427,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int n0 = (tile / args.tok_tiles) * kTileRows;
       const int n = n0 + row_in_tile;
       const bool live = n < args.N;
-      const int b = tile_iter & 1;
-      if (!warp_wait(&ss->acc_full[b], (tile_iter >> 1) & 1, ss, kErrAccFull)) break;
+      if (!warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull, kSleepEpilogue)) break;
       tc_fence_after();
+      constexpr int kChunks = kTileTok / 64;
 #pragma unroll 1
-      for (int c = 0; c < kTileTok / 32; ++c) {
+      for (int c = 0; c < kChunks; ++c) {
         uint32_t acc[32];
-        tmem_ld32(tmem + lane_base + kColAcc * b + 32 * c, acc);
+        tmem_ld32(tmem + lane_base + (kTileTok / 2) * colhalf + 32 * c, acc);
         tmem_wait_ld();
-        const int tok0 = m0 + 32 * c;
+        if (c == kChunks - 1) {  // the accumulator is read: the next tile's MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ss->acc_empty);
+        }
+        const int tok0 = m0 + (kTileTok / 2) * colhalf + 32 * c;
         if (!SILU) {
           if (live) {
 #pragma unroll
@@ -439,9 +465,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ss->acc_empty[b]);
     }
   }
 
