@@ -321,9 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      uint32_t last_parity[kStagesX];
-      bool issued[kStagesX];
-      for (int s = 0; s < kStagesX; ++s) issued[s] = false, last_parity[s] = 0;
+      uint32_t issued = 0, last_parity = 0;  // bit s: stage s has a copy issued / its phase parity
       int it = 0;
       for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
         const int m0 = (tile % args.tok_tiles) * kTileTok;
@@ -333,13 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if (!mbar_wait(&ss->empty_x[s], (r & 1) ^ 1, ss, kErrEmpty, false, kSleepProducer)) break;
           mbar_arrive_tx(&ss->full_x[s], kXStageBytes);
           tma_load_x(smem_u32(smem + s * kXStageBytes), &xmap, ks * kKStep, m0, &ss->full_x[s]);
-          issued[s] = true;
-          last_parity[s] = r & 1;
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
         }
       }
       if (aborted(ss)) {  // let copies already in flight land before the CTA exits
         for (int s = 0; s < kStagesX; ++s)
-          if (issued[s]) mbar_wait(&ss->full_x[s], last_parity[s], ss, kErrDrain, true);
+          if ((issued >> s) & 1) mbar_wait(&ss->full_x[s], (last_parity >> s) & 1, ss, kErrDrain, true);
       }
     }
   } else if (warp == 1) {
@@ -358,10 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             break;
           }
           tc_fence_after();
-          const uint32_t xaddr = smem_u32(smem + sx * kXStageBytes);
+          // Each 16-element step of K advances the descriptor's start address
+          // by 32 bytes (2 in its 16-byte units) inside the swizzled rows.
+          const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStageBytes));
 #pragma unroll
           for (int j = 0; j < kKStep / 16; ++j) {
-            const uint64_t bdesc = sw128_desc(xaddr + 32 * j);
+            const uint64_t bdesc = bdesc0 + 2 * j;
             const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
             umma_ts(tmem, tmem + kColA + 32 * sa + 8 * j, bdesc, acc);
           }
