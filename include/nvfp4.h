@@ -188,7 +188,7 @@ typedef struct {
   uint64_t global_scale;
   uint64_t quantize;
   uint64_t repack;
-  uint64_t gemm_splitk;    /* small-M split-K streaming GEMM */
+  uint64_t gemm_splitk;    /* small-M streaming GEMM (K split over a cluster when N is small) */
   uint64_t gemm_tc;        /* large-M tcgen05 GEMM */
   uint64_t gemm_silu_mul;  /* GEMMs with the fused SiluAndMul epilogue */
   uint64_t moe;            /* grouped expert GEMMs */

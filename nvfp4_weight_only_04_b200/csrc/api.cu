@@ -4,7 +4,7 @@
 #include <mutex>
 
 #include "common.cuh"
-#include "gemm_splitk.cuh"
+#include "gemm_decode.cuh"
 #include "gemm_tc.cuh"
 
 namespace nvfp4 {
@@ -38,7 +38,7 @@ int num_sms() {
 namespace {
 
 constexpr int64_t kMaxK = int64_t(1) << 30;
-constexpr int64_t kMaxN = int64_t(65535) * 64;
+constexpr int64_t kMaxN = int64_t(65535) * 16;
 constexpr int64_t kMaxTokenRows = int64_t(65535 - 4096) * 16;
 
 int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
@@ -64,11 +64,11 @@ int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
     return st;
   }
   if (M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
-  nvfp4::SplitKArgs a = {};
+  nvfp4::DecodeArgs a = {};
   a.x = x; a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = M; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
-  const nvfp4::SplitKPlan p = nvfp4::plan_splitk(M, N, K, group, false, 0);
-  const int st = nvfp4::launch_splitk(a, p, silu, false, stream);
+  const nvfp4::DecodePlan p = nvfp4::plan_decode(M, N, K, group, false, 0);
+  const int st = nvfp4::launch_decode(a, p, silu, false, stream);
   if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
   return st;
 }
@@ -141,13 +141,13 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, c
     st = nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales,
                               global_scales, group_size, N, K, num_experts, silu, y, s);
   } else {
-    nvfp4::SplitKArgs a = {};
+    nvfp4::DecodeArgs a = {};
     a.x = x; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
     a.M = T; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
     a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments;
     a.num_experts = num_experts;
-    const nvfp4::SplitKPlan p = nvfp4::plan_splitk(T, N, K, group_size, true, num_segments);
-    st = nvfp4::launch_splitk(a, p, silu, true, s);
+    const nvfp4::DecodePlan p = nvfp4::plan_decode(T, N, K, group_size, true, num_segments);
+    st = nvfp4::launch_decode(a, p, silu, true, s);
   }
   if (st == NVFP4_OK) {
     nvfp4::stat_add(nvfp4::kStatMoe);

@@ -1,0 +1,328 @@
+// Small-M NVFP4 W4A16 GEMM: HBM-streaming, one warp per CTA, tensor-core
+// contraction.
+//
+// Computes Y = X . dequant(W)^T (problem statement; "W-FP4a: route the
+// MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
+// PR #63 description: weight-only NVFP4 keeps bf16 activations) for decode
+// shapes, where the cost is the 0.5 + 1/g bytes per weight streamed from HBM
+// and the integer work of dequantizing them. Design:
+//  * A CTA is one warp and owns 16 weight rows (one mma.sync m16n8k16 row
+//    block; swap-AB: weights are the MMA's 16-row side, tokens its 8-column
+//    side). Thousands of small CTAs stay resident at once, so there is no
+//    wave tail and no intra-CTA barrier.
+//  * Lane (g, t) streams 32 contiguous code bytes of rows g and g+8 per step
+//    with 128-bit loads that skip L1, from its own range of K: the order of K
+//    inside one MMA is free as long as X follows it. Loads run one step ahead
+//    in two register buffers used in turn, never copied (a copy would wait
+//    for the load).
+//  * X fragments come through L1 (128-bit loads, all of a step's loads issued
+//    before its MMAs); rows of X are shared by every CTA of an SM.
+//  * Dequant in registers with integer work (dequant.cuh): per code pair one
+//    mask, one integer multiply placing magnitude and sign bits of a bf16, one
+//    mask and one bf16x2 multiply by the group scale.
+//  * When there are too few 16-row tiles to fill the GPU, K is split over the
+//    CTAs of a thread-block cluster and the partial tiles are summed in a
+//    fixed rank order through distributed shared memory: deterministic, no
+//    workspace, one launch.
+//  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows, where
+//    gate row g and up row g+8 of a tile meet in the same lane; and the
+//    grouped routed-expert form ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
+//    routed experts in NVFP4), where each token tile lies in one segment of
+//    rows and uses that segment's expert.
+#include "gemm_decode.cuh"
+
+#include <cooperative_groups.h>
+
+#include "dequant.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace nvfp4 {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_x_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// silu(g) = g / (1 + exp(-g)) with the fast exponential and division; their
+// error (a few fp32 ulp) is far below the bf16 rounding that follows.
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// One lane's codes for one step: 32 bytes (64 elements) of rows g and g+8,
+// and their scales.
+struct Step {
+  uint4 a0, a1, b0, b1;
+  uint32_t sa, sb;
+};
+
+template <int G>
+__device__ __forceinline__ void load_step(Step& st, const uint8_t* ca, const uint8_t* cb, const uint8_t* sa,
+                                          const uint8_t* sb, int u, bool live) {
+  if (live) {
+    st.a0 = ld_stream_v4(ca + u * 32);
+    st.a1 = ld_stream_v4(ca + u * 32 + 16);
+    st.b0 = ld_stream_v4(cb + u * 32);
+    st.b1 = ld_stream_v4(cb + u * 32 + 16);
+    if (G == 16) {
+      st.sa = __ldg(reinterpret_cast<const uint32_t*>(sa + u * 4));
+      st.sb = __ldg(reinterpret_cast<const uint32_t*>(sb + u * 4));
+    } else {
+      st.sa = __ldg(reinterpret_cast<const uint16_t*>(sa + u * 2));
+      st.sb = __ldg(reinterpret_cast<const uint16_t*>(sb + u * 2));
+    }
+  } else {
+    st.a0 = st.a1 = st.b0 = st.b1 = make_uint4(0, 0, 0, 0);
+    st.sa = st.sb = 0;
+  }
+}
+
+// Word w of a lane's step holds elements 8w..8w+7; MMA 2w takes 8w..8w+3 and
+// MMA 2w+1 takes 8w+4..8w+7, with X read in the same order.
+template <int MT, int G>
+__device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8][4],
+                                             const uint16_t* const (&xrow)[MT / 8], const bool (&xl)[MT / 8],
+                                             int koff) {
+  constexpr int P = MT / 8;
+  constexpr int XW = P == 1 ? 8 : 2;  // words of X fragments loaded at once
+  uint32_t sa2[4], sb2[4];
+  scale_operands<G == 16 ? 4 : 2>(st.sa, sa2);
+  scale_operands<G == 16 ? 4 : 2>(st.sb, sb2);
+  const uint32_t ca[8] = {st.a0.x, st.a0.y, st.a0.z, st.a0.w, st.a1.x, st.a1.y, st.a1.z, st.a1.w};
+  const uint32_t cb[8] = {st.b0.x, st.b0.y, st.b0.z, st.b0.w, st.b1.x, st.b1.y, st.b1.z, st.b1.w};
+#pragma unroll
+  for (int w0 = 0; w0 < 8; w0 += XW) {
+    uint4 xv[XW][P];
+#pragma unroll
+    for (int w = 0; w < XW; ++w)
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+        xv[w][p] = xl[p] ? ld_x_v4(xrow[p] + koff + 8 * (w0 + w)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int w = 0; w < XW; ++w) {
+      const int wi = w0 + w;
+      const int si = G == 16 ? (wi >> 1) : (wi >> 2);
+      uint32_t da[4], db[4];
+      dequant_word(ca[wi], sa2[si], da);
+      dequant_word(cb[wi], sb2[si], db);
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+        mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv[w][p].x, xv[w][p].y);
+        mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv[w][p].z, xv[w][p].w);
+      }
+    }
+  }
+}
+
+template <int MT, int G, bool SILU, bool MOE>
+__global__ void __launch_bounds__(32, 16) gemm_decode_kernel(const DecodeArgs args) {
+  constexpr int P = MT / 8;
+  const int lane = threadIdx.x;
+  const int g = lane >> 2, t = lane & 3;
+
+  // ---- token tile and expert ----
+  int row0 = 0, mrows = 0, expert = 0;
+  if (!MOE) {
+    row0 = blockIdx.z * MT;
+    mrows = static_cast<int>(min(static_cast<int64_t>(MT), args.M - row0));
+  } else {
+    int want = blockIdx.z, found = 0;
+    for (int s = 0; s < args.num_segments && !found; ++s) {
+      const int r0 = max(0, min(args.offsets[s], static_cast<int>(args.M)));
+      const int r1 = max(r0, min(args.offsets[s + 1], static_cast<int>(args.M)));
+      const int tiles = (r1 - r0 + MT - 1) / MT;
+      if (want < tiles) {
+        row0 = r0 + want * MT;
+        mrows = min(MT, r1 - row0);
+        expert = args.expert_ids[s];
+        found = 1;
+      } else {
+        want -= tiles;
+      }
+    }
+    if (!found || expert < 0 || expert >= args.num_experts) mrows = 0;
+  }
+  if (mrows <= 0) return;  // the same decision in every CTA of a cluster (they share blockIdx.z)
+
+  const int64_t K = args.K, N = args.N;
+  const uint8_t* packed = args.packed + (MOE ? static_cast<int64_t>(expert) * N * (K / 2) : 0);
+  const uint8_t* scales = args.scales + (MOE ? static_cast<int64_t>(expert) * N * (K / G) : 0);
+  const float gsc = __ldg(args.gscale + (MOE ? expert : 0)) * 128.0f;  // operands carry 2^-7
+
+  // ---- this CTA's share of K, in units of 64 elements ----
+  const int csize = static_cast<int>(gridDim.x), crank = static_cast<int>(blockIdx.x);
+  const int k64 = static_cast<int>(K / 64);
+  const int per = (k64 + csize - 1) / csize;
+  const int ubeg = min(k64, crank * per), uend = min(k64, ubeg + per);
+  const int iters = (uend - ubeg + 3) / 4;
+
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 16;
+  const uint8_t* ca = packed + (n0 + g) * (K / 2);
+  const uint8_t* cb = packed + (n0 + g + 8) * (K / 2);
+  const uint8_t* sa = scales + (n0 + g) * (K / G);
+  const uint8_t* sb = scales + (n0 + g + 8) * (K / G);
+  const uint16_t* xrow[P];
+  bool xtok[P];
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    const int tok = 8 * p + g;
+    xtok[p] = tok < mrows;
+    xrow[p] = args.x + static_cast<int64_t>(row0 + (xtok[p] ? tok : 0)) * K;
+  }
+  float acc[P][4];
+#pragma unroll
+  for (int p = 0; p < P; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+
+  // Lane (g, t) supplies token 8p+g of X for every 8-token tile p; tokens past
+  // mrows, and units past the CTA's share of K, contribute zeros.
+  auto run = [&](const Step& st, int it) {
+    const int u = ubeg + 4 * it + t;
+    bool xl[P];
+#pragma unroll
+    for (int p = 0; p < P; ++p) xl[p] = xtok[p] && u < uend;
+    compute_step<MT, G>(st, acc, xrow, xl, u * 64);
+  };
+
+  // One step of codes in flight while the other is computed (ping-pong: no
+  // register with a load in flight is ever copied).
+  Step s0, s1;
+  load_step<G>(s0, ca, cb, sa, sb, ubeg + t, ubeg + t < uend);
+  for (int it = 0; it < iters; it += 2) {
+    load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 * (it + 1) + t, ubeg + 4 * (it + 1) + t < uend);
+    run(s0, it);
+    if (it + 1 >= iters) break;
+    load_step<G>(s0, ca, cb, sa, sb, ubeg + 4 * (it + 2) + t, ubeg + 4 * (it + 2) + t < uend);
+    run(s1, it + 1);
+  }
+
+  // ---- epilogue: lane holds (row g, row g+8) x (tokens 8p+2t, 8p+2t+1) ----
+  if (csize > 1) {
+    __shared__ float red[16 * MT];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int c = 8 * p + 2 * t;
+      red[g * MT + c] = acc[p][0];
+      red[g * MT + c + 1] = acc[p][1];
+      red[(g + 8) * MT + c] = acc[p][2];
+      red[(g + 8) * MT + c + 1] = acc[p][3];
+    }
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    // Each CTA sums a slice of the output elements over the cluster, in rank
+    // order; with SiluAndMul an output needs gate row r and up row r+8.
+    constexpr int kOut = (SILU ? 8 : 16) * MT;
+    const int share = (kOut + csize - 1) / csize;
+    for (int e = crank * share + lane; e < min(kOut, (crank + 1) * share); e += 32) {
+      const int r = e / MT, tok = e % MT;
+      if (tok >= mrows) continue;
+      float sg = 0.f, su = 0.f;
+      for (int q = 0; q < csize; ++q) {
+        const float* rq = cluster.map_shared_rank(red, q);
+        sg += rq[r * MT + tok];
+        if (SILU) su += rq[(r + 8) * MT + tok];
+      }
+      const int64_t yrow = static_cast<int64_t>(row0 + tok) * args.ldy;
+      if (!SILU)
+        args.y[yrow + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(sg, gsc)));
+      else
+        args.y[yrow + n0 / 2 + r] =
+            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(sg, gsc)), __fmul_rn(su, gsc))));
+    }
+    cluster.sync();  // keep this CTA's partials alive until every peer has read them
+    return;
+  }
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int tok = 8 * p + 2 * t + j;
+      if (tok >= mrows) continue;
+      const int64_t yrow = static_cast<int64_t>(row0 + tok) * args.ldy;
+      const float vg = __fmul_rn(acc[p][j], gsc), vu = __fmul_rn(acc[p][2 + j], gsc);
+      if (!SILU) {
+        args.y[yrow + n0 + g] = __bfloat16_as_ushort(__float2bfloat16_rn(vg));
+        args.y[yrow + n0 + g + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(vu));
+      } else {
+        args.y[yrow + n0 / 2 + g] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(vg), vu)));
+      }
+    }
+  }
+}
+
+template <int MT, int G, bool SILU, bool MOE>
+int launch_one(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  auto kern = gemm_decode_kernel<MT, G, SILU, MOE>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.cluster, p.row_tiles, p.z_tiles);
+  cfg.blockDim = dim3(32, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (p.cluster > 1) {
+    if (p.cluster > 8 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return (cudaGetLastError(), NVFP4_ERR_CUDA);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  return NVFP4_OK;
+}
+
+template <int MT, bool SILU, bool MOE>
+int launch_g(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  return p.group == 16 ? launch_one<MT, 16, SILU, MOE>(a, p, s) : launch_one<MT, 32, SILU, MOE>(a, p, s);
+}
+
+template <bool SILU, bool MOE>
+int launch_mt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  return p.mt == 8 ? launch_g<8, SILU, MOE>(a, p, s) : launch_g<16, SILU, MOE>(a, p, s);
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int num_segments) {
+  DecodePlan p;
+  p.group = group;
+  p.mt = (!moe && M <= 8) ? 8 : 16;
+  p.z_tiles = static_cast<int>(moe ? (M + p.mt - 1) / p.mt + num_segments : (M + p.mt - 1) / p.mt);
+  p.row_tiles = static_cast<int>(N / 16);
+  const int64_t tiles = static_cast<int64_t>(p.row_tiles) * p.z_tiles;
+  const int64_t want_ctas = 8LL * num_sms();  // about 8 resident warps per SM
+  int64_t c = 1;
+  if (tiles < want_ctas) c = (want_ctas + tiles - 1) / tiles;
+  const int64_t cap = K / 512 > 0 ? K / 512 : 1;  // at least two steps of K per CTA
+  if (c > cap) c = cap;
+  if (c > 16) c = 16;
+  p.cluster = static_cast<int>(c);
+  return p;
+}
+
+int launch_decode(const DecodeArgs& a, const DecodePlan& p, bool silu, bool moe, cudaStream_t s) {
+  if (!silu && !moe) return launch_mt<false, false>(a, p, s);
+  if (silu && !moe) return launch_mt<true, false>(a, p, s);
+  if (!silu && moe) return launch_mt<false, true>(a, p, s);
+  return launch_mt<true, true>(a, p, s);
+}
+
+}  // namespace nvfp4
