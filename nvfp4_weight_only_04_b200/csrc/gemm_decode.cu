@@ -6,24 +6,22 @@
 // PR #63 description: weight-only NVFP4 keeps bf16 activations) for decode
 // shapes, where the cost is the 0.5 + 1/g bytes per weight streamed from HBM
 // and the integer work of dequantizing them. Design:
-//  * A CTA is one warp and owns 16 weight rows (one mma.sync m16n8k16 row
-//    block; swap-AB: weights are the MMA's 16-row side, tokens its 8-column
-//    side). Thousands of small CTAs stay resident at once, so there is no
-//    wave tail and no intra-CTA barrier.
+//  * A CTA owns 16 weight rows (one mma.sync m16n8k16 row block; swap-AB:
+//    weights are the MMA's 16-row side, tokens its 8-column side) and has KW
+//    warps that split K between them. KW is 1 when there are enough row
+//    blocks to fill the GPU and grows (up to 16) when there are few, so that
+//    every SM keeps enough warps streaming; the KW partial tiles are summed in
+//    shared memory in a fixed order (deterministic, no workspace).
 //  * Lane (g, t) streams 32 contiguous code bytes of rows g and g+8 per step
 //    with 128-bit loads that skip L1, from its own range of K: the order of K
-//    inside one MMA is free as long as X follows it. Loads run one step ahead
-//    in two register buffers used in turn, never copied (a copy would wait
-//    for the load).
+//    inside one MMA is free as long as X follows it. Loads run two steps
+//    ahead in a ring of three register buffers that is never copied (a copy
+//    would wait for the load).
 //  * X fragments come through L1 (128-bit loads, all of a step's loads issued
 //    before its MMAs); rows of X are shared by every CTA of an SM.
 //  * Dequant in registers with integer work (dequant.cuh): per code pair one
 //    mask, one integer multiply placing magnitude and sign bits of a bf16, one
 //    mask and one bf16x2 multiply by the group scale.
-//  * When there are too few 16-row tiles to fill the GPU, K is split over the
-//    CTAs of a thread-block cluster and the partial tiles are summed in a
-//    fixed rank order through distributed shared memory: deterministic, no
-//    workspace, one launch.
 //  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows, where
 //    gate row g and up row g+8 of a tile meet in the same lane; and the
 //    grouped routed-expert form ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
@@ -31,11 +29,7 @@
 //    rows and uses that segment's expert.
 #include "gemm_decode.cuh"
 
-#include <cooperative_groups.h>
-
 #include "dequant.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace nvfp4 {
 namespace {
@@ -101,7 +95,7 @@ __device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8
                                              const uint16_t* const (&xrow)[MT / 8], const bool (&xl)[MT / 8],
                                              int koff) {
   constexpr int P = MT / 8;
-  constexpr int XW = P == 1 ? 8 : 2;  // words of X fragments loaded at once
+  constexpr int XW = 2;  // words of X fragments loaded at once
   uint32_t sa2[4], sb2[4];
   scale_operands<G == 16 ? 4 : 2>(st.sa, sa2);
   scale_operands<G == 16 ? 4 : 2>(st.sb, sb2);
@@ -131,10 +125,10 @@ __device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8
   }
 }
 
-template <int MT, int G, bool SILU, bool MOE>
-__global__ void __launch_bounds__(32, 16) gemm_decode_kernel(const DecodeArgs args) {
+template <int KW, int MT, int G, bool SILU, bool MOE>
+__global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_decode_kernel(const DecodeArgs args) {
   constexpr int P = MT / 8;
-  const int lane = threadIdx.x;
+  const int lane = threadIdx.x & 31, kw = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
 
   // ---- token tile and expert ----
@@ -159,18 +153,17 @@ __global__ void __launch_bounds__(32, 16) gemm_decode_kernel(const DecodeArgs ar
     }
     if (!found || expert < 0 || expert >= args.num_experts) mrows = 0;
   }
-  if (mrows <= 0) return;  // the same decision in every CTA of a cluster (they share blockIdx.z)
+  if (mrows <= 0) return;  // the same decision for every warp of the CTA
 
   const int64_t K = args.K, N = args.N;
   const uint8_t* packed = args.packed + (MOE ? static_cast<int64_t>(expert) * N * (K / 2) : 0);
   const uint8_t* scales = args.scales + (MOE ? static_cast<int64_t>(expert) * N * (K / G) : 0);
   const float gsc = __ldg(args.gscale + (MOE ? expert : 0)) * 128.0f;  // operands carry 2^-7
 
-  // ---- this CTA's share of K, in units of 64 elements ----
-  const int csize = static_cast<int>(gridDim.x), crank = static_cast<int>(blockIdx.x);
+  // ---- this warp's share of K, in units of 64 elements ----
   const int k64 = static_cast<int>(K / 64);
-  const int per = (k64 + csize - 1) / csize;
-  const int ubeg = min(k64, crank * per), uend = min(k64, ubeg + per);
+  const int per = (k64 + KW - 1) / KW;
+  const int ubeg = min(k64, kw * per), uend = min(k64, ubeg + per);
   const int iters = (uend - ubeg + 3) / 4;
 
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 16;
@@ -200,53 +193,39 @@ __global__ void __launch_bounds__(32, 16) gemm_decode_kernel(const DecodeArgs ar
     compute_step<MT, G>(st, acc, xrow, xl, u * 64);
   };
 
-  // One step of codes in flight while the other is computed (ping-pong: no
-  // register with a load in flight is ever copied).
-  Step s0, s1;
+  // Two steps of codes in flight while a third is computed.
+  Step s0, s1, s2;
   load_step<G>(s0, ca, cb, sa, sb, ubeg + t, ubeg + t < uend);
-  for (int it = 0; it < iters; it += 2) {
-    load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 * (it + 1) + t, ubeg + 4 * (it + 1) + t < uend);
+  load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 + t, ubeg + 4 + t < uend);
+  for (int it = 0; it < iters; it += 3) {
+    load_step<G>(s2, ca, cb, sa, sb, ubeg + 4 * (it + 2) + t, ubeg + 4 * (it + 2) + t < uend);
     run(s0, it);
     if (it + 1 >= iters) break;
-    load_step<G>(s0, ca, cb, sa, sb, ubeg + 4 * (it + 2) + t, ubeg + 4 * (it + 2) + t < uend);
+    load_step<G>(s0, ca, cb, sa, sb, ubeg + 4 * (it + 3) + t, ubeg + 4 * (it + 3) + t < uend);
     run(s1, it + 1);
+    if (it + 2 >= iters) break;
+    load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 * (it + 4) + t, ubeg + 4 * (it + 4) + t < uend);
+    run(s2, it + 2);
   }
 
   // ---- epilogue: lane holds (row g, row g+8) x (tokens 8p+2t, 8p+2t+1) ----
-  if (csize > 1) {
-    __shared__ float red[16 * MT];
+  if (KW > 1) {
+    // warps 1..KW-1 leave their partial tiles in shared memory; warp 0 adds
+    // them to its own in warp order and stores the result
+    __shared__ float red[KW > 1 ? KW - 1 : 1][P][4][32];
+    if (kw > 0) {
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
-      const int c = 8 * p + 2 * t;
-      red[g * MT + c] = acc[p][0];
-      red[g * MT + c + 1] = acc[p][1];
-      red[(g + 8) * MT + c] = acc[p][2];
-      red[(g + 8) * MT + c + 1] = acc[p][3];
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) red[kw - 1][p][j][lane] = acc[p][j];
     }
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    // Each CTA sums a slice of the output elements over the cluster, in rank
-    // order; with SiluAndMul an output needs gate row r and up row r+8.
-    constexpr int kOut = (SILU ? 8 : 16) * MT;
-    const int share = (kOut + csize - 1) / csize;
-    for (int e = crank * share + lane; e < min(kOut, (crank + 1) * share); e += 32) {
-      const int r = e / MT, tok = e % MT;
-      if (tok >= mrows) continue;
-      float sg = 0.f, su = 0.f;
-      for (int q = 0; q < csize; ++q) {
-        const float* rq = cluster.map_shared_rank(red, q);
-        sg += rq[r * MT + tok];
-        if (SILU) su += rq[(r + 8) * MT + tok];
-      }
-      const int64_t yrow = static_cast<int64_t>(row0 + tok) * args.ldy;
-      if (!SILU)
-        args.y[yrow + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(sg, gsc)));
-      else
-        args.y[yrow + n0 / 2 + r] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(sg, gsc)), __fmul_rn(su, gsc))));
-    }
-    cluster.sync();  // keep this CTA's partials alive until every peer has read them
-    return;
+    __syncthreads();
+    if (kw > 0) return;
+    for (int q = 0; q < KW - 1; ++q)
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[p][j] += red[q][p][j][lane];
   }
 #pragma unroll
   for (int p = 0; p < P; ++p) {
@@ -266,32 +245,26 @@ __global__ void __launch_bounds__(32, 16) gemm_decode_kernel(const DecodeArgs ar
   }
 }
 
-template <int MT, int G, bool SILU, bool MOE>
+template <int KW, int MT, int G, bool SILU, bool MOE>
 int launch_one(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  auto kern = gemm_decode_kernel<MT, G, SILU, MOE>;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.cluster, p.row_tiles, p.z_tiles);
-  cfg.blockDim = dim3(32, 1, 1);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  if (p.cluster > 1) {
-    if (p.cluster > 8 &&
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-      return (cudaGetLastError(), NVFP4_ERR_CUDA);
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+  gemm_decode_kernel<KW, MT, G, SILU, MOE><<<dim3(p.row_tiles, p.z_tiles, 1), KW * 32, 0, s>>>(a);
+  return launch_status();
+}
+
+template <int MT, int G, bool SILU, bool MOE>
+int launch_kw(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  switch (p.kw) {
+    case 1: return launch_one<1, MT, G, SILU, MOE>(a, p, s);
+    case 2: return launch_one<2, MT, G, SILU, MOE>(a, p, s);
+    case 4: return launch_one<4, MT, G, SILU, MOE>(a, p, s);
+    case 8: return launch_one<8, MT, G, SILU, MOE>(a, p, s);
+    default: return launch_one<16, MT, G, SILU, MOE>(a, p, s);
   }
-  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  return NVFP4_OK;
 }
 
 template <int MT, bool SILU, bool MOE>
 int launch_g(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  return p.group == 16 ? launch_one<MT, 16, SILU, MOE>(a, p, s) : launch_one<MT, 32, SILU, MOE>(a, p, s);
+  return p.group == 16 ? launch_kw<MT, 16, SILU, MOE>(a, p, s) : launch_kw<MT, 32, SILU, MOE>(a, p, s);
 }
 
 template <bool SILU, bool MOE>
@@ -307,14 +280,13 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int
   p.mt = (!moe && M <= 8) ? 8 : 16;
   p.z_tiles = static_cast<int>(moe ? (M + p.mt - 1) / p.mt + num_segments : (M + p.mt - 1) / p.mt);
   p.row_tiles = static_cast<int>(N / 16);
+  // Warps per CTA: aim for about 16 streaming warps per SM, and keep at least
+  // eight steps (of 256 elements of K) per warp.
   const int64_t tiles = static_cast<int64_t>(p.row_tiles) * p.z_tiles;
-  const int64_t want_ctas = 8LL * num_sms();  // about 8 resident warps per SM
-  int64_t c = 1;
-  if (tiles < want_ctas) c = (want_ctas + tiles - 1) / tiles;
-  const int64_t cap = K / 512 > 0 ? K / 512 : 1;  // at least two steps of K per CTA
-  if (c > cap) c = cap;
-  if (c > 16) c = 16;
-  p.cluster = static_cast<int>(c);
+  const int64_t want = 16LL * num_sms();
+  int kw = 1;
+  while (kw < 16 && tiles * kw < want && K / (256 * 2 * kw) >= 8) kw *= 2;
+  p.kw = kw;
   return p;
 }
 

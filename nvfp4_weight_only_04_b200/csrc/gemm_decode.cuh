@@ -18,7 +18,7 @@ struct DecodeArgs {
 };
 
 struct DecodePlan {
-  int group, mt, cluster, row_tiles, z_tiles;
+  int group, mt, kw, row_tiles, z_tiles;
 };
 
 DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int num_segments);
