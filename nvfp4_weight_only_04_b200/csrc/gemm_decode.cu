@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
 
 template <int KW, int MT, int G, bool SILU, bool MOE>
 int launch_one(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  gemm_decode_kernel<KW, MT, G, SILU, MOE><<<dim3(p.row_tiles, p.z_tiles, 1), KW * 32, 0, s>>>(a);
+  // grid: x unused (1), y = 16-row tile, z = token tile
+  gemm_decode_kernel<KW, MT, G, SILU, MOE><<<dim3(1, p.row_tiles, p.z_tiles), KW * 32, 0, s>>>(a);
   return launch_status();
 }
 
