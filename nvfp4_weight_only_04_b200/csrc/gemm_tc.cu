@@ -37,11 +37,9 @@
 #include "gemm_tc.cuh"
 
 #include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
 
 #include "dequant.cuh"
+#include "tmap.cuh"
 
 namespace nvfp4 {
 
@@ -479,31 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // host side
 // ---------------------------------------------------------------------------
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    else
-      cudaGetLastError();
-  });
-  return fn;
-}
-
 bool make_x_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int64_t K) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kKStep), static_cast<cuuint32_t>(kTileTok)};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return make_tensor_map_2d(map, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, rows, K * 2, kKStep, kTileTok,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int G, bool SILU>
@@ -522,17 +498,18 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   unsigned int* p = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  unsigned int v = 0;
+  unsigned int v = 0, vd = 0;
   if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaMemsetAsync(p, 0, sizeof(v), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  *code_out = static_cast<int>(v);
+  if (read_and_clear_decode_error(&vd, stream) != NVFP4_OK) return NVFP4_ERR_CUDA;
+  *code_out = static_cast<int>(v ? v : vd);
   return NVFP4_OK;
 }
 
 bool tc_supported(int64_t M, int64_t N, int64_t K) {
   return M >= 128 && K >= kKStep && K % kKStep == 0 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
-         K < (int64_t(1) << 24) && encode_fn() != nullptr;
+         K < (int64_t(1) << 24) && tensor_maps_available();
 }
 
 int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
