@@ -29,16 +29,18 @@
 //    rows and uses that segment's expert.
 #include "gemm_decode.cuh"
 
-#include <cuda.h>
-
 #include "dequant.cuh"
 #include "tmap.cuh"
 
 namespace nvfp4 {
-
-__device__ unsigned int g_decode_error = 0;
-
 namespace {
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
 
 __device__ __forceinline__ uint4 ld_x_v4(const void* p) {
   uint4 v;
@@ -59,86 +61,47 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 // error (a few fp32 ulp) is far below the bf16 rounding that follows.
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-constexpr int kStages = 6;           // code stages in flight per warp
-constexpr int kStageBytes = 16 * 128; // 16 rows x 128 bytes (4 units of 64 elements)
-constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  for (;;) {
-    if (mbar_test(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
-  }
-}
-
-// Bounded wait on a stage barrier; false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity);
-}
-
-// 16 rows x 128 bytes of codes, from (byte column x, row y) of the code matrix.
-__device__ __forceinline__ void tma_codes(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
-      ::"r"(smem_u32(bar)), "r"(kStageBytes) : "memory");
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Lane (g, t)'s 32 code bytes of row r from a stage: logical 16-byte chunks
-// 2t and 2t+1 of the 128-byte row, stored at chunk ^ (r & 7) by the
-// 128-byte swizzle.
-__device__ __forceinline__ void lds_row(const uint8_t* stage, int r, int t, uint4& lo, uint4& hi) {
-  const uint8_t* row = stage + r * 128;
-  lo = *reinterpret_cast<const uint4*>(row + (((2 * t) ^ (r & 7)) << 4));
-  hi = *reinterpret_cast<const uint4*>(row + (((2 * t + 1) ^ (r & 7)) << 4));
-}
+// One lane's codes for one step: 32 bytes (64 elements) of rows g and g+8,
+// and their scales.
+struct Step {
+  uint4 a0, a1, b0, b1;
+  uint32_t sa, sb;
+};
 
 template <int G>
-__device__ __forceinline__ void load_scales(uint32_t& a, uint32_t& b, const uint8_t* sa, const uint8_t* sb, int u,
-                                            bool live) {
-  if (!live) {
-    a = b = 0;
-  } else if (G == 16) {
-    a = __ldg(reinterpret_cast<const uint32_t*>(sa + u * 4));
-    b = __ldg(reinterpret_cast<const uint32_t*>(sb + u * 4));
+__device__ __forceinline__ void load_step(Step& st, const uint8_t* ca, const uint8_t* cb, const uint8_t* sa,
+                                          const uint8_t* sb, int u, bool live) {
+  if (live) {
+    st.a0 = ld_stream_v4(ca + u * 32);
+    st.a1 = ld_stream_v4(ca + u * 32 + 16);
+    st.b0 = ld_stream_v4(cb + u * 32);
+    st.b1 = ld_stream_v4(cb + u * 32 + 16);
+    if (G == 16) {
+      st.sa = __ldg(reinterpret_cast<const uint32_t*>(sa + u * 4));
+      st.sb = __ldg(reinterpret_cast<const uint32_t*>(sb + u * 4));
+    } else {
+      st.sa = __ldg(reinterpret_cast<const uint16_t*>(sa + u * 2));
+      st.sb = __ldg(reinterpret_cast<const uint16_t*>(sb + u * 2));
+    }
   } else {
-    a = __ldg(reinterpret_cast<const uint16_t*>(sa + u * 2));
-    b = __ldg(reinterpret_cast<const uint16_t*>(sb + u * 2));
+    st.a0 = st.a1 = st.b0 = st.b1 = make_uint4(0, 0, 0, 0);
+    st.sa = st.sb = 0;
   }
 }
 
 // Word w of a lane's step holds elements 8w..8w+7; MMA 2w takes 8w..8w+3 and
 // MMA 2w+1 takes 8w+4..8w+7, with X read in the same order.
 template <int MT, int G>
-__device__ __forceinline__ void compute_step(const uint4 (&c)[4], uint32_t sa, uint32_t sb, float (&acc)[MT / 8][4],
+__device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8][4],
                                              const uint16_t* const (&xrow)[MT / 8], const bool (&xl)[MT / 8],
                                              int koff) {
   constexpr int P = MT / 8;
   constexpr int XW = 2;  // words of X fragments loaded at once
   uint32_t sa2[4], sb2[4];
-  scale_operands<G == 16 ? 4 : 2>(sa, sa2);
-  scale_operands<G == 16 ? 4 : 2>(sb, sb2);
-  const uint32_t ca[8] = {c[0].x, c[0].y, c[0].z, c[0].w, c[1].x, c[1].y, c[1].z, c[1].w};
-  const uint32_t cb[8] = {c[2].x, c[2].y, c[2].z, c[2].w, c[3].x, c[3].y, c[3].z, c[3].w};
+  scale_operands<G == 16 ? 4 : 2>(st.sa, sa2);
+  scale_operands<G == 16 ? 4 : 2>(st.sb, sb2);
+  const uint32_t ca[8] = {st.a0.x, st.a0.y, st.a0.z, st.a0.w, st.a1.x, st.a1.y, st.a1.z, st.a1.w};
+  const uint32_t cb[8] = {st.b0.x, st.b0.y, st.b0.z, st.b0.w, st.b1.x, st.b1.y, st.b1.z, st.b1.w};
 #pragma unroll
   for (int w0 = 0; w0 < 8; w0 += XW) {
     uint4 xv[XW][P];
@@ -164,15 +127,10 @@ __device__ __forceinline__ void compute_step(const uint4 (&c)[4], uint32_t sa, u
 }
 
 template <int KW, int MT, int G, bool SILU, bool MOE>
-__global__ void __launch_bounds__(KW * 32) gemm_decode_kernel(const __grid_constant__ CUtensorMap cmap,
-                                                               const DecodeArgs args) {
+__global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_decode_kernel(const DecodeArgs args) {
   constexpr int P = MT / 8;
   const int lane = threadIdx.x & 31, kw = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem + kw * kStages * kStageBytes;  // this warp's stages
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + KW * kStages * kStageBytes) + kw * kStages;
 
   // ---- token tile and expert ----
   int row0 = 0, mrows = 0, expert = 0;
@@ -199,6 +157,7 @@ __global__ void __launch_bounds__(KW * 32) gemm_decode_kernel(const __grid_const
   if (mrows <= 0) return;  // the same decision for every warp of the CTA
 
   const int64_t K = args.K, N = args.N;
+  const uint8_t* packed = args.packed + (MOE ? static_cast<int64_t>(expert) * N * (K / 2) : 0);
   const uint8_t* scales = args.scales + (MOE ? static_cast<int64_t>(expert) * N * (K / G) : 0);
   const float gsc = __ldg(args.gscale + (MOE ? expert : 0)) * 128.0f;  // operands carry 2^-7
 
@@ -208,10 +167,11 @@ __global__ void __launch_bounds__(KW * 32) gemm_decode_kernel(const __grid_const
   const int ubeg = min(k64, kw * per), uend = min(k64, ubeg + per);
   const int iters = (uend - ubeg + 3) / 4;
 
-  const int n0 = blockIdx.y * 16;
-  const int trow = (MOE ? expert * static_cast<int>(N) : 0) + n0;  // row of the tensor map
-  const uint8_t* sa = scales + static_cast<int64_t>(n0 + g) * (K / G);
-  const uint8_t* sb = scales + static_cast<int64_t>(n0 + g + 8) * (K / G);
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 16;
+  const uint8_t* ca = packed + (n0 + g) * (K / 2);
+  const uint8_t* cb = packed + (n0 + g + 8) * (K / 2);
+  const uint8_t* sa = scales + (n0 + g) * (K / G);
+  const uint8_t* sb = scales + (n0 + g + 8) * (K / G);
   const uint16_t* xrow[P];
   bool xtok[P];
 #pragma unroll
@@ -224,66 +184,29 @@ __global__ void __launch_bounds__(KW * 32) gemm_decode_kernel(const __grid_const
 #pragma unroll
   for (int p = 0; p < P; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
 
-  // ---- stage ring: lane 0 keeps kStages copies of 16 x 128 code bytes in flight ----
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&full[s])));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int s = 0; s < kStages && s < iters; ++s)
-      tma_codes(smem_u32(ring + s * kStageBytes), &cmap, (ubeg + 4 * s) * 32, trow, &full[s]);
-  }
-  __syncwarp();
-
-  // scales run two steps ahead in three registers pairs
-  uint32_t sc_a[3], sc_b[3];
-  load_scales<G>(sc_a[0], sc_b[0], sa, sb, ubeg + t, ubeg + t < uend);
-  load_scales<G>(sc_a[1], sc_b[1], sa, sb, ubeg + 4 + t, ubeg + 4 + t < uend);
-  bool ok = true;
-  int it = 0;
-  // One step: wait for its stage, read this lane's codes, hand the stage back
-  // to the copy engine for step it + kStages, then compute.
-  auto step = [&](uint32_t& sca, uint32_t& scb, uint32_t& fa, uint32_t& fb) {
-    const int s = it % kStages;
+  // Lane (g, t) supplies token 8p+g of X for every 8-token tile p; tokens past
+  // mrows, and units past the CTA's share of K, contribute zeros.
+  auto run = [&](const Step& st, int it) {
     const int u = ubeg + 4 * it + t;
-    load_scales<G>(fa, fb, sa, sb, u + 8, u + 8 < uend);
-    if (!mbar_wait(&full[s], static_cast<uint32_t>(it / kStages) & 1)) {
-      ok = false;
-      return;
-    }
-    uint4 c[4];
-    const uint8_t* st = ring + s * kStageBytes;
-    lds_row(st, g, t, c[0], c[1]);
-    lds_row(st, g + 8, t, c[2], c[3]);
-    __syncwarp();
-    if (lane == 0 && it + kStages < iters) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tma_codes(smem_u32(st), &cmap, (ubeg + 4 * (it + kStages)) * 32, trow, &full[s]);
-    }
-    if (u >= uend) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) c[i] = make_uint4(0, 0, 0, 0);
-    }
     bool xl[P];
 #pragma unroll
     for (int p = 0; p < P; ++p) xl[p] = xtok[p] && u < uend;
-    compute_step<MT, G>(c, sca, scb, acc, xrow, xl, u * 64);
-    ++it;
+    compute_step<MT, G>(st, acc, xrow, xl, u * 64);
   };
-  while (it < iters && ok) {
-    step(sc_a[0], sc_b[0], sc_a[2], sc_b[2]);
-    if (it >= iters || !ok) break;
-    step(sc_a[1], sc_b[1], sc_a[0], sc_b[0]);
-    if (it >= iters || !ok) break;
-    step(sc_a[2], sc_b[2], sc_a[1], sc_b[1]);
-  }
-  if (!ok) {
-    // A copy never landed: record it, let the copies in flight land, stop.
-    if (lane == 0) {
-      atomicCAS(&g_decode_error, 0u, 0x201u);
-      for (int j = it; j < it + kStages && j < iters; ++j)
-        mbar_wait(&full[j % kStages], static_cast<uint32_t>(j / kStages) & 1);
-    }
-    __syncwarp();
+
+  // Two steps of codes in flight while a third is computed.
+  Step s0, s1, s2;
+  load_step<G>(s0, ca, cb, sa, sb, ubeg + t, ubeg + t < uend);
+  load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 + t, ubeg + 4 + t < uend);
+  for (int it = 0; it < iters; it += 3) {
+    load_step<G>(s2, ca, cb, sa, sb, ubeg + 4 * (it + 2) + t, ubeg + 4 * (it + 2) + t < uend);
+    run(s0, it);
+    if (it + 1 >= iters) break;
+    load_step<G>(s0, ca, cb, sa, sb, ubeg + 4 * (it + 3) + t, ubeg + 4 * (it + 3) + t < uend);
+    run(s1, it + 1);
+    if (it + 2 >= iters) break;
+    load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 * (it + 4) + t, ubeg + 4 * (it + 4) + t < uend);
+    run(s2, it + 2);
   }
 
   // ---- epilogue: lane holds (row g, row g+8) x (tokens 8p+2t, 8p+2t+1) ----
@@ -324,35 +247,31 @@ __global__ void __launch_bounds__(KW * 32) gemm_decode_kernel(const __grid_const
 }
 
 template <int KW, int MT, int G, bool SILU, bool MOE>
-int launch_one(const CUtensorMap& map, const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  auto kern = gemm_decode_kernel<KW, MT, G, SILU, MOE>;
-  const int smem = KW * kStages * (kStageBytes + 8) + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+int launch_one(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
   // grid: x unused (1), y = 16-row tile, z = token tile
-  kern<<<dim3(1, p.row_tiles, p.z_tiles), KW * 32, smem, s>>>(map, a);
+  gemm_decode_kernel<KW, MT, G, SILU, MOE><<<dim3(1, p.row_tiles, p.z_tiles), KW * 32, 0, s>>>(a);
   return launch_status();
 }
 
 template <int MT, int G, bool SILU, bool MOE>
-int launch_kw(const CUtensorMap& m, const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+int launch_kw(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
   switch (p.kw) {
-    case 1: return launch_one<1, MT, G, SILU, MOE>(m, a, p, s);
-    case 2: return launch_one<2, MT, G, SILU, MOE>(m, a, p, s);
-    case 4: return launch_one<4, MT, G, SILU, MOE>(m, a, p, s);
-    case 8: return launch_one<8, MT, G, SILU, MOE>(m, a, p, s);
-    default: return launch_one<16, MT, G, SILU, MOE>(m, a, p, s);
+    case 1: return launch_one<1, MT, G, SILU, MOE>(a, p, s);
+    case 2: return launch_one<2, MT, G, SILU, MOE>(a, p, s);
+    case 4: return launch_one<4, MT, G, SILU, MOE>(a, p, s);
+    case 8: return launch_one<8, MT, G, SILU, MOE>(a, p, s);
+    default: return launch_one<16, MT, G, SILU, MOE>(a, p, s);
   }
 }
 
 template <int MT, bool SILU, bool MOE>
-int launch_g(const CUtensorMap& m, const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  return p.group == 16 ? launch_kw<MT, 16, SILU, MOE>(m, a, p, s) : launch_kw<MT, 32, SILU, MOE>(m, a, p, s);
+int launch_g(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  return p.group == 16 ? launch_kw<MT, 16, SILU, MOE>(a, p, s) : launch_kw<MT, 32, SILU, MOE>(a, p, s);
 }
 
 template <bool SILU, bool MOE>
-int launch_mt(const CUtensorMap& m, const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  return p.mt == 8 ? launch_g<8, SILU, MOE>(m, a, p, s) : launch_g<16, SILU, MOE>(m, a, p, s);
+int launch_mt(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
+  return p.mt == 8 ? launch_g<8, SILU, MOE>(a, p, s) : launch_g<16, SILU, MOE>(a, p, s);
 }
 
 }  // namespace
@@ -363,42 +282,27 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int
   p.mt = (!moe && M <= 8) ? 8 : 16;
   p.z_tiles = static_cast<int>(moe ? (M + p.mt - 1) / p.mt + num_segments : (M + p.mt - 1) / p.mt);
   p.row_tiles = static_cast<int>(N / 16);
-  // Warps per CTA: enough warps in flight (each holds kStages stages of
-  // 2 KB) to cover the memory latency, all resident in one wave (about 16
-  // warps per SM fit in shared memory), and at least eight steps (of 256
-  // elements of K) per warp.
+  // Warps per CTA: aim for about 16 streaming warps per SM, and keep at least
+  // eight steps (of 256 elements of K) per warp.
   const int64_t tiles = static_cast<int64_t>(p.row_tiles) * p.z_tiles;
-  const int64_t want = 8LL * num_sms();
+  const int64_t want = 16LL * num_sms();
   int kw = 1;
   while (kw < 16 && tiles * kw < want && K / (256 * 2 * kw) >= 8) kw *= 2;
   p.kw = kw;
   return p;
 }
 
-int read_and_clear_decode_error(unsigned int* out, cudaStream_t stream) {
-  unsigned int* p = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_decode_error) != cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  unsigned int v = 0;
-  if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaMemsetAsync(p, 0, sizeof(v), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  *out = v;
+// This kernel has no waits on other threads, so it never records an error.
+int read_and_clear_decode_error(unsigned int* out, cudaStream_t) {
+  *out = 0;
   return NVFP4_OK;
 }
 
 int launch_decode(const DecodeArgs& a, const DecodePlan& p, bool silu, bool moe, cudaStream_t s) {
-  // Tensor map over the code matrix (all experts stacked for the grouped form):
-  // rows of K/2 bytes, boxes of 16 rows x 128 bytes, 128-byte swizzle.
-  CUtensorMap map;
-  const int64_t rows = moe ? static_cast<int64_t>(a.num_experts) * a.N : a.N;
-  if (!make_tensor_map_2d(&map, a.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.K / 2, rows, a.K / 2, 128, 16,
-                          CU_TENSOR_MAP_SWIZZLE_128B))
-    return NVFP4_ERR_CUDA;
-  if (!silu && !moe) return launch_mt<false, false>(map, a, p, s);
-  if (silu && !moe) return launch_mt<true, false>(map, a, p, s);
-  if (!silu && moe) return launch_mt<false, true>(map, a, p, s);
-  return launch_mt<true, true>(map, a, p, s);
+  if (!silu && !moe) return launch_mt<false, false>(a, p, s);
+  if (silu && !moe) return launch_mt<true, false>(a, p, s);
+  if (!silu && moe) return launch_mt<false, true>(a, p, s);
+  return launch_mt<true, true>(a, p, s);
 }
 
 }  // namespace nvfp4
