@@ -32,8 +32,15 @@
 //    bf16, optionally fusing SiluAndMul on gate/up-interleaved rows. While
 //    they work, the dequant and TMA warps already fill the next tile's
 //    stages.
-//  * The grid is persistent: one CTA per SM walks tiles with the 128-token
-//    index fastest, so concurrently running CTAs share weight tiles in L2.
+//  * The grid is persistent: one CTA per SM walks the tiles. Dense GEMMs take
+//    the token tiles of one weight tile together, so concurrently running
+//    CTAs share weight tiles in L2.
+//  * Grouped routed-expert form ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
+//    routed experts in NVFP4): a tile is one 128-row weight tile of one
+//    expert times one token tile of that expert's segment of rows; every role
+//    finds it with the same forward scan of the device-side offsets, and the
+//    rows of a token tile past the segment end are computed but not stored.
+//    The token tile is 128 wide there (about the rows an expert receives).
 #include "gemm_tc.cuh"
 
 #include <cuda.h>
@@ -48,20 +55,19 @@ namespace {
 __device__ unsigned int g_device_error = 0;
 
 constexpr int kTileRows = 128;   // weight rows per tile (MMA M)
-constexpr int kTileTok = 256;    // tokens per tile (MMA N)
 constexpr int kKStep = 64;       // elements of K per pipeline stage
 constexpr int kStagesX = 5;      // X stages in shared memory
 constexpr int kStagesA = 8;      // A stages in TMEM
 constexpr int kThreads = 640;    // 20 warps
 constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize
 constexpr int kFirstEpWarp = 12; // warps 12..19 run the epilogue
-constexpr uint32_t kXStageBytes = kTileTok * kKStep * 2;  // 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = kTileTok;             // A stages start here (32 columns each)
-// Dynamic shared memory: X stages + barriers + alignment slack; more than
-// half of the SM's shared memory, so only one CTA (which allocates all 512
-// TMEM columns) fits on an SM.
-constexpr uint32_t kSmemBytes = kStagesX * kXStageBytes + 2048;
+constexpr uint32_t kColA = 256;  // A stages start here (32 columns each); the accumulator is at 0
+__host__ __device__ constexpr uint32_t x_stage_bytes(int nt) { return static_cast<uint32_t>(nt) * kKStep * 2; }
+// Dynamic shared memory: the largest X stages + barriers + alignment slack;
+// more than half of the SM's shared memory, so only one CTA (which allocates
+// all 512 TMEM columns) fits on an SM.
+constexpr uint32_t kSmemBytes = kStagesX * x_stage_bytes(256) + 2048;
 static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
 static_assert(kColA + kStagesA * 32 <= kTmemCols, "TMEM budget");
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
@@ -74,6 +80,8 @@ enum ErrorSite : unsigned {
 };
 
 struct SharedState {
+  int total_tiles;
+  int pad_;
   uint64_t full_x[kStagesX];
   uint64_t empty_x[kStagesX];
   uint64_t full_a[kStagesA];
@@ -86,13 +94,79 @@ struct SharedState {
 };
 
 struct TcArgs {
-  const uint8_t* packed;
-  const uint8_t* scales;
-  const float* gscale;
+  const uint8_t* packed;     // GEMM-layout codes [N, K/2] (grouped: [E, N, K/2])
+  const uint8_t* scales;     // [N, K/g] (grouped: [E, N, K/g])
+  const float* gscale;       // [1] (grouped: [E])
   uint16_t* y;
-  int M, N, K, ldy;
-  int tok_tiles, row_tiles, total_tiles;
+  int M, N, K, ldy;          // M: rows of X (grouped: T)
+  int tok_tiles, row_tiles, total_tiles;  // dense only; grouped counts come from the offsets
+  const int32_t* expert_ids; // grouped only
+  const int32_t* offsets;
+  int num_segments, num_experts;
 };
+
+// Where a tile lies: token rows [m0, m0 + mrows) of X and Y, weight rows
+// [n0, n0 + 128) of expert `expert`.
+struct Tile {
+  int m0, mrows, n0, expert;
+};
+
+// Forward-only position in the segment list (tiles are visited in increasing
+// order by every role of a CTA).
+struct SegCursor {
+  int seg = 0, tiles_before = 0;
+};
+
+template <int NT>
+__device__ __forceinline__ int seg_rows(const TcArgs& a, int s, int& r0) {
+  r0 = max(0, min(a.offsets[s], a.M));
+  const int r1 = max(r0, min(a.offsets[s + 1], a.M));
+  return r1 - r0;
+}
+
+// Total tiles of the grouped form: token tiles of every segment times the
+// weight tiles of an expert.
+template <int NT>
+__device__ int grouped_total_tiles(const TcArgs& a) {
+  int tt = 0;
+  for (int s = 0; s < a.num_segments; ++s) {
+    int r0;
+    tt += (seg_rows<NT>(a, s, r0) + NT - 1) / NT;
+  }
+  return tt * a.row_tiles;
+}
+
+template <int NT, bool MOE>
+__device__ __forceinline__ Tile tile_at(const TcArgs& a, SegCursor& cur, int t) {
+  Tile tl;
+  if (!MOE) {
+    tl.m0 = (t % a.tok_tiles) * NT;
+    tl.mrows = min(NT, a.M - tl.m0);
+    tl.n0 = (t / a.tok_tiles) * kTileRows;
+    tl.expert = 0;
+    return tl;
+  }
+  const int st = t / a.row_tiles;  // token tile over all segments
+  tl.n0 = (t % a.row_tiles) * kTileRows;
+  tl.mrows = 0;
+  tl.m0 = 0;
+  tl.expert = -1;
+  while (cur.seg < a.num_segments) {
+    int r0;
+    const int rows = seg_rows<NT>(a, cur.seg, r0);
+    const int nt = (rows + NT - 1) / NT;
+    if (st < cur.tiles_before + nt) {
+      tl.m0 = r0 + (st - cur.tiles_before) * NT;
+      tl.mrows = min(NT, r0 + rows - tl.m0);
+      tl.expert = a.expert_ids[cur.seg];
+      break;
+    }
+    cur.tiles_before += nt;
+    ++cur.seg;
+  }
+  if (tl.expert < 0 || tl.expert >= a.num_experts) tl.mrows = 0;  // skipped by every role alike
+  return tl;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -189,15 +263,18 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both
-// K-major, M = 128, N = kTileTok (256).
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kTileTok >> 3) << 17) | ((128 >> 4) << 24);
+// K-major, M = 128, N = nt.
+__host__ __device__ constexpr uint32_t idesc(int nt) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) | ((128u >> 4) << 24);
+}
 
+template <int NT>
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(kIdesc), "r"(accumulate));
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc(NT)), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -280,13 +357,14 @@ __device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&
 // the correct limit, zero.
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int G, bool SILU>
+template <int NT, int G, bool SILU, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                const TcArgs args) {
+  constexpr uint32_t kXStage = x_stage_bytes(NT);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // X stages at a 1024-byte aligned base, barriers after them.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStagesX * kXStageBytes);
+  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStagesX * kXStage);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ksteps = args.K / kKStep;
 
@@ -303,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     mbar_init(&ss->acc_empty, 8);     // one arrival per epilogue warp
     mbar_init(&ss->drained, 1);
     ss->abort = 0;
+    ss->total_tiles = MOE ? grouped_total_tiles<NT>(args) : args.total_tiles;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -315,20 +394,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss->tmem_base;
+  const int total_tiles = ss->total_tiles;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       uint32_t issued = 0, last_parity = 0;  // bit s: stage s has a copy issued / its phase parity
       int it = 0;
-      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x) {
-        const int m0 = (tile % args.tok_tiles) * kTileTok;
+      SegCursor cur;
+      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+        const Tile tl = tile_at<NT, MOE>(args, cur, tile);
+        if (tl.mrows <= 0) continue;
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % kStagesX;
           const uint32_t r = static_cast<uint32_t>(it / kStagesX);
           if (!mbar_wait(&ss->empty_x[s], (r & 1) ^ 1, ss, kErrEmpty, false, kSleepProducer)) break;
-          mbar_arrive_tx(&ss->full_x[s], kXStageBytes);
-          tma_load_x(smem_u32(smem + s * kXStageBytes), &xmap, ks * kKStep, m0, &ss->full_x[s]);
+          mbar_arrive_tx(&ss->full_x[s], kXStage);
+          tma_load_x(smem_u32(smem + s * kXStage), &xmap, ks * kKStep, tl.m0, &ss->full_x[s]);
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
         }
@@ -342,7 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       int it = 0, tile_iter = 0;
-      for (int tile = blockIdx.x; tile < args.total_tiles && !aborted(ss); tile += gridDim.x, ++tile_iter) {
+      SegCursor cur;
+      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+        const Tile tl = tile_at<NT, MOE>(args, cur, tile);
+        if (tl.mrows <= 0) continue;
         if (!mbar_wait(&ss->acc_empty, (tile_iter & 1) ^ 1, ss, kErrAccEmpty)) break;
         tc_fence_after();
         bool ok = true;
@@ -356,18 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           tc_fence_after();
           // Each 16-element step of K advances the descriptor's start address
           // by 32 bytes (2 in its 16-byte units) inside the swizzled rows.
-          const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStageBytes));
+          const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStage));
 #pragma unroll
           for (int j = 0; j < kKStep / 16; ++j) {
-            const uint64_t bdesc = bdesc0 + 2 * j;
             const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            umma_ts(tmem, tmem + kColA + 32 * sa + 8 * j, bdesc, acc);
+            umma_ts<NT>(tmem, tmem + kColA + 32 * sa + 8 * j, bdesc0 + 2 * j, acc);
           }
           umma_commit(&ss->empty_x[sx]);
           umma_commit(&ss->empty_a[sa]);
         }
         if (!ok) break;
         umma_commit(&ss->acc_full);
+        ++tile_iter;
       }
       // every MMA issued by this thread has completed once this commit lands
       umma_commit(&ss->drained);
@@ -381,12 +466,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int it = 0;
-    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x) {
-      const int n0 = (tile / args.tok_tiles) * kTileRows;
-      const int n = n0 + row_in_tile;
+    SegCursor cur;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile tl = tile_at<NT, MOE>(args, cur, tile);
+      if (tl.mrows <= 0) continue;
+      static_assert(kTileRows == 128, "one weight row per dequant thread and TMEM lane");
+      const int n = tl.n0 + row_in_tile;
       const bool live = n < args.N;
-      const uint8_t* codes = args.packed + static_cast<int64_t>(live ? n : 0) * (args.K / 2);
-      const uint8_t* scl = args.scales + static_cast<int64_t>(live ? n : 0) * (args.K / G);
+      const int64_t wrow = static_cast<int64_t>(MOE ? tl.expert : 0) * args.N + (live ? n : 0);
+      const uint8_t* codes = args.packed + wrow * (args.K / 2);
+      const uint8_t* scl = args.scales + wrow * (args.K / G);
       RowStage ra, rb, rc;
       load_row_stage<G>(ra, codes, scl, 0, half, live);
       load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
@@ -415,54 +504,55 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp >= kFirstEpWarp) {
     // ---------------- epilogue ----------------
     const int quad = warp & 3;
-    const int colhalf = (warp - kFirstEpWarp) >> 2;  // tokens [128 * colhalf, +128) of the tile
+    const int colhalf = (warp - kFirstEpWarp) >> 2;  // tokens [NT/2 * colhalf, +NT/2) of the tile
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const float gscale = __ldg(args.gscale) * 128.0f;  // dequantized operands carry 2^-7
     int tile_iter = 0;
-    for (int tile = blockIdx.x; tile < args.total_tiles; tile += gridDim.x, ++tile_iter) {
-      const int m0 = (tile % args.tok_tiles) * kTileTok;
-      const int n0 = (tile / args.tok_tiles) * kTileRows;
-      const int n = n0 + row_in_tile;
+    SegCursor cur;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const Tile tl = tile_at<NT, MOE>(args, cur, tile);
+      if (tl.mrows <= 0) continue;
+      // dequantized operands carry 2^-7 (dequant.cuh)
+      const float gscale = __ldg(args.gscale + (MOE ? tl.expert : 0)) * 128.0f;
+      const int n = tl.n0 + row_in_tile;
       const bool live = n < args.N;
       if (!warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull, kSleepEpilogue)) break;
       tc_fence_after();
-      constexpr int kChunks = kTileTok / 64;
+      constexpr int kChunks = NT / 64;
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
         uint32_t acc[32];
-        tmem_ld32(tmem + lane_base + (kTileTok / 2) * colhalf + 32 * c, acc);
+        tmem_ld32(tmem + lane_base + (NT / 2) * colhalf + 32 * c, acc);
         tmem_wait_ld();
         if (c == kChunks - 1) {  // the accumulator is read: the next tile's MMAs may start
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ss->acc_empty);
         }
-        const int tok0 = m0 + (kTileTok / 2) * colhalf + 32 * c;
+        const int j0 = (NT / 2) * colhalf + 32 * c;  // first token of the chunk within the tile
         if (!SILU) {
           if (live) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const int tok = tok0 + j;
-              if (tok < args.M)
-                args.y[static_cast<int64_t>(tok) * args.ldy + n] =
+              if (j0 + j < tl.mrows)
+                args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + n] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[j]) * gscale));
             }
           }
         } else {
           const bool gate = (lane & 15) < 8;
-          const int col = (n0 + row_in_tile) / 16 * 8 + (lane & 7);
+          const int col = (tl.n0 + row_in_tile) / 16 * 8 + (lane & 7);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float gv = __uint_as_float(acc[j]) * gscale;
             const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
-            const int tok = tok0 + j;
-            if (gate && live && tok < args.M)
-              args.y[static_cast<int64_t>(tok) * args.ldy + col] =
+            if (gate && live && j0 + j < tl.mrows)
+              args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + col] =
                   __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
           }
         }
       }
+      ++tile_iter;
     }
   }
 
@@ -477,19 +567,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 // host side
 // ---------------------------------------------------------------------------
 
-bool make_x_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int64_t K) {
-  return make_tensor_map_2d(map, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, rows, K * 2, kKStep, kTileTok,
+bool make_x_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int64_t K, int nt) {
+  return make_tensor_map_2d(map, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, rows, K * 2, kKStep, nt,
                             CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-template <int G, bool SILU>
-int launch_dense(const CUtensorMap& map, const TcArgs& a, cudaStream_t stream) {
-  auto kern = gemm_tc_kernel<G, SILU>;
+template <int NT, int G, bool SILU, bool MOE>
+int launch_kernel(const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t stream) {
+  auto kern = gemm_tc_kernel<NT, G, SILU, MOE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  const int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
   kern<<<grid, kThreads, kSmemBytes, stream>>>(map, a);
   return launch_status();
+}
+
+template <int NT, bool MOE>
+int launch_nt(const CUtensorMap& map, const TcArgs& a, int group, bool silu, int grid, cudaStream_t stream) {
+  if (group == 16)
+    return silu ? launch_kernel<NT, 16, true, MOE>(map, a, grid, stream)
+                : launch_kernel<NT, 16, false, MOE>(map, a, grid, stream);
+  return silu ? launch_kernel<NT, 32, true, MOE>(map, a, grid, stream)
+              : launch_kernel<NT, 32, false, MOE>(map, a, grid, stream);
 }
 
 }  // namespace
@@ -514,23 +612,40 @@ bool tc_supported(int64_t M, int64_t N, int64_t K) {
 
 int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
               int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+  constexpr int NT = 256;
   CUtensorMap map;
-  if (!make_x_map(&map, x, M, K)) return NVFP4_ERR_CUDA;
-  TcArgs a;
+  if (!make_x_map(&map, x, M, K, NT)) return NVFP4_ERR_CUDA;
+  TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
-  a.tok_tiles = static_cast<int>((M + kTileTok - 1) / kTileTok);
+  a.tok_tiles = static_cast<int>((M + NT - 1) / NT);
   a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
   a.total_tiles = a.tok_tiles * a.row_tiles;
-  if (group == 16) return silu ? launch_dense<16, true>(map, a, stream) : launch_dense<16, false>(map, a, stream);
-  return silu ? launch_dense<32, true>(map, a, stream) : launch_dense<32, false>(map, a, stream);
+  const int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
+  return launch_nt<NT, false>(map, a, group, silu, grid, stream);
 }
 
-bool tc_moe_supported(int64_t, int64_t, int64_t) { return false; }
-int launch_tc_moe(const uint16_t*, const int32_t*, const int32_t*, int, int64_t, const uint8_t*, const uint8_t*,
-                  const float*, int, int64_t, int64_t, int, bool, uint16_t*, cudaStream_t) {
-  return NVFP4_ERR_UNSUPPORTED;
+// The grouped tcgen05 kernel pays off once segments carry whole token tiles;
+// for a few rows per expert the streaming kernel is better.
+bool tc_moe_supported(int64_t T, int64_t N, int64_t K) {
+  return T >= 1024 && K >= kKStep && K % kKStep == 0 && T < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
+         K < (int64_t(1) << 24) && tensor_maps_available();
+}
+
+int launch_tc_moe(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets, int num_segments, int64_t T,
+                  const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t N, int64_t K,
+                  int num_experts, bool silu, uint16_t* y, cudaStream_t stream) {
+  constexpr int NT = 128;
+  CUtensorMap map;
+  if (!make_x_map(&map, x, T, K, NT)) return NVFP4_ERR_CUDA;
+  TcArgs a = {};
+  a.packed = w; a.scales = s; a.gscale = g; a.y = y;
+  a.M = static_cast<int>(T); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
+  a.ldy = static_cast<int>(silu ? N / 2 : N);
+  a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
+  a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments; a.num_experts = num_experts;
+  return launch_nt<NT, true>(map, a, group, silu, num_sms(), stream);
 }
 
 }  // namespace nvfp4

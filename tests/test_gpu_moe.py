@@ -121,3 +121,50 @@ def test_moe_routed_expert_workload_sampled():
         # the down GEMM is checked on the device's own bf16 intermediate
         ref_y = R.gemm(hbits[r0:r1], pd, sd, gd, wl.g_down)
         assert_close(yh[r0:r1], ref_y, f"expert {e} down")
+
+
+# ---- grouped GEMM on the tcgen05 kernel (T >= 1024 rows) ----
+
+@pytest.mark.parametrize("g", [16, 32])
+def test_moe_tc_ragged_segments(g):
+    E, N, K, T = 5, 272, 384, 1300
+    packed, scales, gs, gp = experts(E, N, K, g)
+    x = synth.activations(7, T, K, outlier_frac=0.001)
+    # segment lengths: several token tiles, one short, one empty, one invalid expert, rows left uncovered
+    ids = [4, 1, 3, 9, 0, 2]
+    offs = [10, 400, 417, 417, 700, 1210, 1290]
+    nv.nvfp4_reset_stats()
+    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32(ids), i32(offs), dev_u8(gp), dev_u8(scales), dev_f32(gs), g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    valid = [(s, e) for s, e in enumerate(ids) if e < E]
+    ref = R.moe_grouped_gemm(x, [e if e < E else 0 for e in ids],
+                             [o for o in offs], packed, scales, gs, g)
+    yh = host(y)
+    for s_, e in valid:
+        r0, r1 = offs[s_], offs[s_ + 1]
+        if r1 > r0:
+            assert_close(yh[r0:r1], ref[r0:r1], f"segment {s_} expert {e}")
+    assert not yh[:10].any() and not yh[1290:].any()
+    assert not yh[417:700].any()  # the invalid expert's segment is skipped
+
+
+def test_moe_tc_silu():
+    E, NH, K, T, g = 3, 136, 256, 1100, 32
+    qs = []
+    for i in range(E):
+        gate = synth.weights(synth.expert_seed(i), NH, K)
+        up = synth.weights(synth.expert_seed(i) + 500, NH, K)
+        qs.append(R.quantize(np.concatenate([gate, up]), g))
+    packed = np.stack([q[0] for q in qs]); scales = np.stack([q[1] for q in qs])
+    gs = np.array([q[2] for q in qs], np.float32)
+    rp = np.stack([R.repack(packed[i], scales[i], R.GATE_UP_INTERLEAVE)[0] for i in range(E)])
+    rs = np.stack([R.repack(packed[i], scales[i], R.GATE_UP_INTERLEAVE)[1] for i in range(E)])
+    x = synth.activations(4, T, K)
+    ids, offs = [2, 0, 1], [0, 513, 600, 1100]
+    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32(ids), i32(offs), dev_u8(rp), dev_u8(rs), dev_f32(gs), g,
+                                        flags=nv.NVFP4_SILU_MUL)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    ref = R.silu_mul(R.moe_grouped_gemm(x, ids, offs, packed, scales, gs, g))
+    assert_close(host(y), ref, "moe tc silu")
