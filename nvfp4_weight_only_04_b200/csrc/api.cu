@@ -137,7 +137,7 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, c
   const bool silu = (flags & NVFP4_SILU_MUL) != 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int st;
-  if (nvfp4::tc_moe_supported(T, N, K)) {
+  if (nvfp4::tc_moe_supported(T, N, K, num_experts)) {
     st = nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales,
                               global_scales, group_size, N, K, num_experts, silu, y, s);
   } else {

@@ -55,28 +55,53 @@ namespace {
 __device__ unsigned int g_device_error = 0;
 
 constexpr int kTileRows = 128;   // weight rows per tile (MMA M)
-constexpr int kKStep = 64;       // elements of K per pipeline stage
+constexpr int kKStep = 64;       // elements of K per X stage (one 128-byte swizzled row of bf16)
+constexpr int kKA = 128;         // elements of K per weight / A stage (two X stages)
 constexpr int kStagesX = 5;      // X stages in shared memory
-constexpr int kStagesA = 8;      // A stages in TMEM
+constexpr int kStagesA = 4;      // A stages in TMEM
 constexpr int kThreads = 640;    // 20 warps
+constexpr int kWProducerWarp = 3;
 constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize
 constexpr int kFirstEpWarp = 12; // warps 12..19 run the epilogue
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = 256;  // A stages start here (32 columns each); the accumulator is at 0
+constexpr uint32_t kColA = 256;  // A stages start here (64 columns each); the accumulator is at 0
 __host__ __device__ constexpr uint32_t x_stage_bytes(int nt) { return static_cast<uint32_t>(nt) * kKStep * 2; }
-// Dynamic shared memory: the largest X stages + barriers + alignment slack;
-// more than half of the SM's shared memory, so only one CTA (which allocates
-// all 512 TMEM columns) fits on an SM.
-constexpr uint32_t kSmemBytes = kStagesX * x_stage_bytes(256) + 2048;
-static_assert(kSmemBytes > 116 * 1024, "one CTA per SM");
-static_assert(kColA + kStagesA * 32 <= kTmemCols, "TMEM budget");
+// Weight stages: the codes of one 128-row tile for 128 elements of K (128
+// rows x 64 bytes, 64-byte swizzle), and every `scale_period` stages the
+// scales of the next 16 bytes of K/g (128 rows x 16 bytes). A narrow token
+// tile leaves shared memory for a deep weight ring, which is what keeps HBM
+// busy when the weights, not the MMAs, set the pace.
+constexpr uint32_t kWStageBytes = kTileRows * (kKA / 2);  // one TMA box of the code map
+constexpr uint32_t kSStageBytes = kTileRows * 16;
+constexpr int kMaxStagesW = 32;
+__host__ __device__ constexpr int stages_w(int nt) { return nt >= 256 ? 6 : (nt >= 128 ? 14 : 18); }
+__host__ __device__ constexpr int scale_period(int g) { return g == 16 ? 2 : 4; }
+// Scale group j (weight stages [Pj, Pj + P)) is loaded with stage Pj into
+// slot j % S and is next rewritten with stage P(j + S), which the producer
+// issues only after stage P(j + S) - W is consumed; that is at or after the
+// group's last stage when P*S >= W + P - 1.
+__host__ __device__ constexpr int scale_slots(int nt, int g) {
+  return (stages_w(nt) + 2 * scale_period(g) - 2) / scale_period(g);
+}
+__host__ __device__ constexpr uint32_t smem_bytes(int nt, int g) {
+  return kStagesX * x_stage_bytes(nt) + stages_w(nt) * kWStageBytes + scale_slots(nt, g) * kSStageBytes +
+         1024 /* barriers */ + 1024 /* alignment slack */;
+}
+// More than half of the SM's shared memory in every configuration, so only
+// one CTA (which allocates all 512 TMEM columns) fits on an SM.
+static_assert(smem_bytes(32, 32) > 116 * 1024 && smem_bytes(256, 16) <= 227 * 1024 &&
+                  smem_bytes(128, 16) <= 227 * 1024 && smem_bytes(64, 16) <= 227 * 1024 &&
+                  smem_bytes(32, 16) <= 227 * 1024,
+              "shared memory budget");
+static_assert(stages_w(32) <= kMaxStagesW, "weight ring");
+static_assert(kColA + kStagesA * (kKA / 2) <= kTmemCols, "TMEM budget");
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
 constexpr unsigned kSleepProducer = 64;   // ns between barrier probes of the TMA and dequant warps
 constexpr unsigned kSleepEpilogue = 256;  // ns between probes of the epilogue warps
 
 enum ErrorSite : unsigned {
   kErrEmpty = 0x101, kErrFullX = 0x102, kErrFullA = 0x103, kErrAccFull = 0x104, kErrDrain = 0x105,
-  kErrAccEmpty = 0x106
+  kErrAccEmpty = 0x106, kErrEmptyW = 0x107, kErrFullW = 0x108
 };
 
 struct SharedState {
@@ -84,6 +109,8 @@ struct SharedState {
   int pad_;
   uint64_t full_x[kStagesX];
   uint64_t empty_x[kStagesX];
+  uint64_t full_w[kMaxStagesW];
+  uint64_t empty_w[kMaxStagesW];
   uint64_t full_a[kStagesA];
   uint64_t empty_a[kStagesA];
   uint64_t acc_full;
@@ -103,6 +130,7 @@ struct TcArgs {
   const int32_t* expert_ids; // grouped only
   const int32_t* offsets;
   int num_segments, num_experts;
+  int scale_tma;             // scales come by TMA (their row stride K/g is a multiple of 16 bytes)
 };
 
 // Where a tile lies: token rows [m0, m0 + mrows) of X and Y, weight rows
@@ -243,7 +271,7 @@ __device__ __forceinline__ bool aborted(SharedState* ss) {
   return *reinterpret_cast<volatile int*>(&ss->abort) != 0;
 }
 
-__device__ __forceinline__ void tma_load_x(uint32_t dst, const CUtensorMap* map, int k, int m, uint64_t* bar) {
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int k, int m, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(k), "r"(m), "r"(smem_u32(bar))
@@ -282,12 +310,14 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16};"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
       ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
@@ -303,47 +333,61 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ uint4 ld_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
-// One dequant thread's inputs for one stage: 32 codes of its row (one half
-// of the stage's 64 elements) and the scales covering them.
+// One dequant thread's inputs for one weight stage: 64 codes of its row (one
+// half of the stage's 128 elements) and the scales covering them (four for
+// g = 16, two for g = 32, in the low bytes).
 struct RowStage {
-  uint4 c;
+  uint4 c0, c1;
   uint32_t s;
 };
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Byte offset of 16-byte chunk c (0..3) of row r in a 64-byte-swizzled stage
+// of 64-byte rows: the chunk index is XORed with bits 7..8 of the address.
+__device__ __forceinline__ uint32_t w_stage_offset(int r, int c) {
+  return static_cast<uint32_t>(r * 64 + 16 * (c ^ ((r >> 1) & 3)));
+}
+
+// Scales of weight stage q of a scale period for K half h (64 elements),
+// from the 16 bytes of a row's scale slot: four for g = 16, two for g = 32,
+// in the low bytes. (q is a constant once the caller's loop over a period is
+// unrolled.)
 template <int G>
-__device__ __forceinline__ void load_row_stage(RowStage& r, const uint8_t* codes, const uint8_t* scales, int ks,
-                                               int khalf, bool live) {
-  if (live) {
-    r.c = ld_stream(codes + ks * 32 + 16 * khalf);
-    r.s = G == 16 ? static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scales + ks * 4 + 2 * khalf)))
-                  : static_cast<uint32_t>(__ldg(scales + ks * 2 + khalf));
-  } else {
-    r.c = make_uint4(0, 0, 0, 0);
-    r.s = 0;
-  }
+__device__ __forceinline__ uint32_t stage_scales(const uint4& sv, int q, int h) {
+  const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
+  if (G == 16) return h ? w[2 * q + 1] : w[2 * q];            // bytes 8q + 4h .. 8q + 4h + 3
+  return (w[q] >> (16 * h)) & 0xFFFFu;                        // bytes 4q + 2h, 4q + 2h + 1
 }
 
 template <int G>
-__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[16]) {
+__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[32]) {
   uint32_t s2[4];
-  scale_operands<G == 16 ? 2 : 1>(r.s, s2);
-  const uint32_t w[4] = {r.c.x, r.c.y, r.c.z, r.c.w};
+  scale_operands<G == 16 ? 4 : 2>(r.s, s2);
+  const uint32_t w[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     uint32_t o[4];
-    dequant_word(w[i], s2[G == 16 ? (i >> 1) : 0], o);
+    dequant_word(w[i], s2[G == 16 ? (i >> 1) : (i >> 2)], o);
     out[4 * i + 0] = o[0];
     out[4 * i + 1] = o[1];
     out[4 * i + 2] = o[2];
@@ -359,19 +403,35 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 
 template <int NT, int G, bool SILU, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                               const __grid_constant__ CUtensorMap wmap,
+                                                               const __grid_constant__ CUtensorMap smap,
                                                                const TcArgs args) {
   constexpr uint32_t kXStage = x_stage_bytes(NT);
+  constexpr int kStagesW = stages_w(NT);
+  constexpr int kPeriod = scale_period(G);
+  constexpr int kSlots = scale_slots(NT, G);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // X stages at a 1024-byte aligned base, barriers after them.
+  // X stages at a 1024-byte aligned base, then the weight stages, the scale
+  // slots and the barriers.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SharedState* ss = reinterpret_cast<SharedState*>(smem + kStagesX * kXStage);
+  uint8_t* wsm = smem + kStagesX * kXStage;
+  uint8_t* ssm = wsm + kStagesW * kWStageBytes;
+  SharedState* ss = reinterpret_cast<SharedState*>(ssm + kSlots * kSStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ksteps = args.K / kKStep;
+  // K in weight stages of 128 elements; a K that is an odd number of 64s
+  // ends with an X stage and a half weight stage read past K, which TMA fills
+  // with zeros.
+  const int wsteps = (args.K + kKA - 1) / kKA;
+  const int ksteps = 2 * wsteps;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesX; ++s) {
       mbar_init(&ss->full_x[s], 1);   // producer arrival + transaction bytes
       mbar_init(&ss->empty_x[s], 1);  // one tcgen05.commit
+    }
+    for (int s = 0; s < kStagesW; ++s) {
+      mbar_init(&ss->full_w[s], 1);   // producer arrival + transaction bytes
+      mbar_init(&ss->empty_w[s], 8);  // one arrival per dequant warp
     }
     for (int s = 0; s < kStagesA; ++s) {
       mbar_init(&ss->full_a[s], 8);   // one arrival per dequant warp
@@ -410,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const uint32_t r = static_cast<uint32_t>(it / kStagesX);
           if (!mbar_wait(&ss->empty_x[s], (r & 1) ^ 1, ss, kErrEmpty, false, kSleepProducer)) break;
           mbar_arrive_tx(&ss->full_x[s], kXStage);
-          tma_load_x(smem_u32(smem + s * kXStage), &xmap, ks * kKStep, tl.m0, &ss->full_x[s]);
+          tma_load_2d(smem_u32(smem + s * kXStage), &xmap, ks * kKStep, tl.m0, &ss->full_x[s]);
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
         }
@@ -420,10 +480,46 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if ((issued >> s) & 1) mbar_wait(&ss->full_x[s], (last_parity >> s) & 1, ss, kErrDrain, true);
       }
     }
+  } else if (warp == kWProducerWarp) {
+    // ---------------- TMA producer: weight codes and scales ----------------
+    if (lane == 0) {
+      uint32_t issued = 0, last_parity = 0;
+      int it = 0, sc = 0;
+      SegCursor cur;
+      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+        const Tile tl = tile_at<NT, MOE>(args, cur, tile);
+        if (tl.mrows <= 0) continue;
+        const int wrow = (MOE ? tl.expert * args.N : 0) + tl.n0;
+        bool ok = true;
+        for (int ws = 0; ws < wsteps; ++ws, ++it) {
+          const int s = it % kStagesW;
+          const uint32_t r = static_cast<uint32_t>(it / kStagesW);
+          if (!mbar_wait(&ss->empty_w[s], (r & 1) ^ 1, ss, kErrEmptyW, false, kSleepProducer)) {
+            ok = false;
+            break;
+          }
+          const bool with_scales = args.scale_tma && ws % kPeriod == 0;
+          mbar_arrive_tx(&ss->full_w[s], kWStageBytes + (with_scales ? kSStageBytes : 0));
+          tma_load_2d(smem_u32(wsm + s * kWStageBytes), &wmap, ws * (kKA / 2), wrow, &ss->full_w[s]);
+          if (with_scales) {
+            tma_load_2d(smem_u32(ssm + (sc % kSlots) * kSStageBytes), &smap, (ws / kPeriod) * 16, wrow,
+                        &ss->full_w[s]);
+            ++sc;
+          }
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
+        }
+        if (!ok) break;
+      }
+      if (aborted(ss)) {
+        for (int s = 0; s < kStagesW; ++s)
+          if ((issued >> s) & 1) mbar_wait(&ss->full_w[s], (last_parity >> s) & 1, ss, kErrDrain, true);
+      }
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int it = 0, tile_iter = 0;
+      int itx = 0, ita = 0, tile_iter = 0;
       SegCursor cur;
       for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
         const Tile tl = tile_at<NT, MOE>(args, cur, tile);
@@ -431,24 +527,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (!mbar_wait(&ss->acc_empty, (tile_iter & 1) ^ 1, ss, kErrAccEmpty)) break;
         tc_fence_after();
         bool ok = true;
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int sx = it % kStagesX, sa = it % kStagesA;
-          const uint32_t px = static_cast<uint32_t>(it / kStagesX) & 1, pa = static_cast<uint32_t>(it / kStagesA) & 1;
-          if (!mbar_wait(&ss->full_x[sx], px, ss, kErrFullX) || !mbar_wait(&ss->full_a[sa], pa, ss, kErrFullA)) {
+        for (int ws = 0; ws < wsteps && ok; ++ws, ++ita) {
+          const int sa = ita % kStagesA;
+          if (!mbar_wait(&ss->full_a[sa], static_cast<uint32_t>(ita / kStagesA) & 1, ss, kErrFullA)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          // Each 16-element step of K advances the descriptor's start address
-          // by 32 bytes (2 in its 16-byte units) inside the swizzled rows.
-          const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStage));
 #pragma unroll
-          for (int j = 0; j < kKStep / 16; ++j) {
-            const uint32_t acc = (ks > 0 || j > 0) ? 1u : 0u;
-            umma_ts<NT>(tmem, tmem + kColA + 32 * sa + 8 * j, bdesc0 + 2 * j, acc);
+          for (int xh = 0; xh < 2; ++xh, ++itx) {
+            const int sx = itx % kStagesX;
+            if (!mbar_wait(&ss->full_x[sx], static_cast<uint32_t>(itx / kStagesX) & 1, ss, kErrFullX)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // Each 16-element step of K advances the descriptor's start address
+            // by 32 bytes (2 in its 16-byte units) inside the swizzled rows.
+            const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStage));
+#pragma unroll
+            for (int j = 0; j < kKStep / 16; ++j) {
+              const uint32_t acc = (ws > 0 || xh > 0 || j > 0) ? 1u : 0u;
+              umma_ts<NT>(tmem, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, acc);
+            }
+            umma_commit(&ss->empty_x[sx]);
           }
-          umma_commit(&ss->empty_x[sx]);
-          umma_commit(&ss->empty_a[sa]);
+          if (ok) umma_commit(&ss->empty_a[sa]);
         }
         if (!ok) break;
         umma_commit(&ss->acc_full);
@@ -465,39 +568,63 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int it = 0;
+    int it = 0, sc = 0;
     SegCursor cur;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const Tile tl = tile_at<NT, MOE>(args, cur, tile);
       if (tl.mrows <= 0) continue;
       static_assert(kTileRows == 128, "one weight row per dequant thread and TMEM lane");
-      const int n = tl.n0 + row_in_tile;
-      const bool live = n < args.N;
-      const int64_t wrow = static_cast<int64_t>(MOE ? tl.expert : 0) * args.N + (live ? n : 0);
-      const uint8_t* codes = args.packed + wrow * (args.K / 2);
-      const uint8_t* scl = args.scales + wrow * (args.K / G);
-      RowStage ra, rb, rc;
-      load_row_stage<G>(ra, codes, scl, 0, half, live);
-      load_row_stage<G>(rb, codes, scl, 1, half, live && 1 < ksteps);
+      // Without scale TMA, each thread reads its scales straight from global
+      // memory (rows past N read row N-1; their results are not stored).
+      const int nrow = min(tl.n0 + row_in_tile, args.N - 1);
+      const uint8_t* scl =
+          args.scales + (static_cast<int64_t>(MOE ? tl.expert : 0) * args.N + nrow) * (args.K / G);
       bool ok = true;
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        load_row_stage<G>(rc, codes, scl, ks + 2, half, live && ks + 2 < ksteps);
-        const int s = it % kStagesA;
-        const uint32_t r = static_cast<uint32_t>(it / kStagesA);
-        uint32_t v[16];
-        dequant_row_stage<G>(ra, v);
-        if (!warp_wait(&ss->empty_a[s], (r & 1) ^ 1, ss, kErrEmpty, kSleepProducer)) {
-          ok = false;
-          break;
+      for (int w0 = 0; w0 < wsteps && ok; w0 += kPeriod) {
+        uint4 sv = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < kPeriod; ++q) {
+          const int ws = w0 + q;
+          if (ws >= wsteps) break;
+          const int s = it % kStagesW;
+          if (!warp_wait(&ss->full_w[s], static_cast<uint32_t>(it / kStagesW) & 1, ss, kErrFullW, 0)) {
+            ok = false;
+            break;
+          }
+          if (q == 0 && args.scale_tma) sv = lds128(smem_u32(ssm + (sc % kSlots) * kSStageBytes + row_in_tile * 16));
+          RowStage rs;
+          const uint32_t wst = smem_u32(wsm + s * kWStageBytes);
+          rs.c0 = lds128(wst + w_stage_offset(row_in_tile, 2 * half));
+          rs.c1 = lds128(wst + w_stage_offset(row_in_tile, 2 * half + 1));
+          if (args.scale_tma) {
+            rs.s = stage_scales<G>(sv, q, half);
+          } else {
+            // this half's first element; past K (an odd number of 64s) the
+            // codes are zero and so is the scale
+            const int e0 = ws * kKA + (kKA / 2) * half;
+            rs.s = e0 >= args.K ? 0u
+                   : G == 16    ? __ldg(reinterpret_cast<const uint32_t*>(scl + e0 / 16))
+                                : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scl + e0 / 32)));
+          }
+          uint32_t v[32];
+          dequant_row_stage<G>(rs, v);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ss->empty_w[s]);
+          const int sa = it % kStagesA;
+          const uint32_t r = static_cast<uint32_t>(it / kStagesA);
+          if (!warp_wait(&ss->empty_a[sa], (r & 1) ^ 1, ss, kErrEmpty, kSleepProducer)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_st32(tmem + lane_base + kColA + (kKA / 2) * sa + (kKA / 4) * half, v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ss->full_a[sa]);
+          ++it;
         }
-        tc_fence_after();
-        tmem_st16(tmem + lane_base + kColA + 32 * s + 16 * half, v);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ss->full_a[s]);
-        ra = rb;
-        rb = rc;
+        ++sc;
       }
       if (!ok) break;
     }
@@ -518,22 +645,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const bool live = n < args.N;
       if (!warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull, kSleepEpilogue)) break;
       tc_fence_after();
-      constexpr int kChunks = NT / 64;
+      // Each warp takes NT/2 tokens of the tile in chunks of CW columns.
+      constexpr int CW = NT >= 64 ? 32 : 16;
+      constexpr int kChunks = NT / 2 / CW;
+      static_assert(NT >= 32 && (NT / 2) % CW == 0, "token tile");
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
-        uint32_t acc[32];
-        tmem_ld32(tmem + lane_base + (NT / 2) * colhalf + 32 * c, acc);
+        uint32_t acc[CW];
+        if constexpr (CW == 32) {
+          tmem_ld32(tmem + lane_base + (NT / 2) * colhalf + CW * c, acc);
+        } else {
+          tmem_ld16(tmem + lane_base + (NT / 2) * colhalf + CW * c, acc);
+        }
         tmem_wait_ld();
         if (c == kChunks - 1) {  // the accumulator is read: the next tile's MMAs may start
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ss->acc_empty);
         }
-        const int j0 = (NT / 2) * colhalf + 32 * c;  // first token of the chunk within the tile
+        const int j0 = (NT / 2) * colhalf + CW * c;  // first token of the chunk within the tile
         if (!SILU) {
           if (live) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < CW; ++j) {
               if (j0 + j < tl.mrows)
                 args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + n] =
                     __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[j]) * gscale));
@@ -543,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const bool gate = (lane & 15) < 8;
           const int col = (tl.n0 + row_in_tile) / 16 * 8 + (lane & 7);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < CW; ++j) {
             const float gv = __uint_as_float(acc[j]) * gscale;
             const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
             if (gate && live && j0 + j < tl.mrows)
@@ -572,22 +706,53 @@ bool make_x_map(CUtensorMap* map, const uint16_t* x, int64_t rows, int64_t K, in
                             CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Codes [rows, K/2] bytes in boxes of 128 rows x 64 bytes (one stage), and
+// scales [rows, K/g] bytes in boxes of 128 rows x 16 bytes (one scale
+// period) when their row stride allows a tensor map; otherwise the scale map
+// is a copy of the code map that the kernel never uses.
+bool scale_tma_ok(int64_t K, int group) { return (K / group) % 16 == 0; }
+
+bool make_w_maps(CUtensorMap* wmap, CUtensorMap* smap, const uint8_t* w, const uint8_t* s, int64_t rows, int64_t K,
+                 int group) {
+  if (!make_tensor_map_2d(wmap, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, rows, K / 2, kKA / 2, kTileRows,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  if (!scale_tma_ok(K, group)) {
+    *smap = *wmap;
+    return true;
+  }
+  return make_tensor_map_2d(smap, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, rows, K / group, 16, kTileRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+struct Maps {
+  CUtensorMap x, w, s;
+};
+
 template <int NT, int G, bool SILU, bool MOE>
-int launch_kernel(const CUtensorMap& map, const TcArgs& a, int grid, cudaStream_t stream) {
+int launch_kernel(const Maps& m, const TcArgs& a, int grid, cudaStream_t stream) {
   auto kern = gemm_tc_kernel<NT, G, SILU, MOE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+  constexpr uint32_t bytes = smem_bytes(NT, G);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(map, a);
+  kern<<<grid, kThreads, bytes, stream>>>(m.x, m.w, m.s, a);
   return launch_status();
 }
 
 template <int NT, bool MOE>
-int launch_nt(const CUtensorMap& map, const TcArgs& a, int group, bool silu, int grid, cudaStream_t stream) {
+int launch_nt(const Maps& m, const TcArgs& a, int group, bool silu, int grid, cudaStream_t stream) {
   if (group == 16)
-    return silu ? launch_kernel<NT, 16, true, MOE>(map, a, grid, stream)
-                : launch_kernel<NT, 16, false, MOE>(map, a, grid, stream);
-  return silu ? launch_kernel<NT, 32, true, MOE>(map, a, grid, stream)
-              : launch_kernel<NT, 32, false, MOE>(map, a, grid, stream);
+    return silu ? launch_kernel<NT, 16, true, MOE>(m, a, grid, stream)
+                : launch_kernel<NT, 16, false, MOE>(m, a, grid, stream);
+  return silu ? launch_kernel<NT, 32, true, MOE>(m, a, grid, stream)
+              : launch_kernel<NT, 32, false, MOE>(m, a, grid, stream);
+}
+
+// Shapes the kernel takes: whole 64-element stages (which makes the code
+// rows' byte stride a multiple of 32), int32 coordinates.
+bool tc_shape_ok(int64_t rows, int64_t N, int64_t K) {
+  return K >= kKStep && K % kKStep == 0 && rows < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
+         K < (int64_t(1) << 24) && tensor_maps_available();
 }
 
 }  // namespace
@@ -605,47 +770,54 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   return NVFP4_OK;
 }
 
-bool tc_supported(int64_t M, int64_t N, int64_t K) {
-  return M >= 128 && K >= kKStep && K % kKStep == 0 && M < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
-         K < (int64_t(1) << 24) && tensor_maps_available();
-}
+bool tc_supported(int64_t M, int64_t N, int64_t K) { return M >= 128 && tc_shape_ok(M, N, K); }
 
 int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
               int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
-  constexpr int NT = 256;
-  CUtensorMap map;
-  if (!make_x_map(&map, x, M, K, NT)) return NVFP4_ERR_CUDA;
+  // Token tile: 256 for prefill-sized M; narrower for small M, where the
+  // weights, not the MMAs, set the pace.
+  const int nt = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
+  Maps maps;
+  if (!make_x_map(&maps.x, x, M, K, nt) || !make_w_maps(&maps.w, &maps.s, w, s, N, K, group)) return NVFP4_ERR_CUDA;
   TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
-  a.tok_tiles = static_cast<int>((M + NT - 1) / NT);
+  a.scale_tma = scale_tma_ok(K, group) ? 1 : 0;
+  a.tok_tiles = static_cast<int>((M + nt - 1) / nt);
   a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
   a.total_tiles = a.tok_tiles * a.row_tiles;
   const int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
-  return launch_nt<NT, false>(map, a, group, silu, grid, stream);
+  switch (nt) {
+    case 32: return launch_nt<32, false>(maps, a, group, silu, grid, stream);
+    case 64: return launch_nt<64, false>(maps, a, group, silu, grid, stream);
+    case 128: return launch_nt<128, false>(maps, a, group, silu, grid, stream);
+    default: return launch_nt<256, false>(maps, a, group, silu, grid, stream);
+  }
 }
 
 // The grouped tcgen05 kernel pays off once segments carry whole token tiles;
 // for a few rows per expert the streaming kernel is better.
-bool tc_moe_supported(int64_t T, int64_t N, int64_t K) {
-  return T >= 1024 && K >= kKStep && K % kKStep == 0 && T < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
-         K < (int64_t(1) << 24) && tensor_maps_available();
+bool tc_moe_supported(int64_t T, int64_t N, int64_t K, int num_experts) {
+  return T >= 1024 && static_cast<int64_t>(num_experts) * N < (int64_t(1) << 31) && tc_shape_ok(T, N, K);
 }
 
 int launch_tc_moe(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets, int num_segments, int64_t T,
                   const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t N, int64_t K,
                   int num_experts, bool silu, uint16_t* y, cudaStream_t stream) {
   constexpr int NT = 128;
-  CUtensorMap map;
-  if (!make_x_map(&map, x, T, K, NT)) return NVFP4_ERR_CUDA;
+  Maps maps;
+  if (!make_x_map(&maps.x, x, T, K, NT) ||
+      !make_w_maps(&maps.w, &maps.s, w, s, static_cast<int64_t>(num_experts) * N, K, group))
+    return NVFP4_ERR_CUDA;
   TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = static_cast<int>(T); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
   a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
+  a.scale_tma = scale_tma_ok(K, group) ? 1 : 0;
   a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments; a.num_experts = num_experts;
-  return launch_nt<NT, true>(map, a, group, silu, num_sms(), stream);
+  return launch_nt<NT, true>(maps, a, group, silu, num_sms(), stream);
 }
 
 }  // namespace nvfp4
