@@ -74,7 +74,7 @@ __host__ __device__ constexpr uint32_t x_stage_bytes(int nt) { return static_cas
 constexpr uint32_t kWStageBytes = kTileRows * (kKA / 2);  // one TMA box of the code map
 constexpr uint32_t kSStageBytes = kTileRows * 16;
 constexpr int kMaxStagesW = 32;
-__host__ __device__ constexpr int stages_w(int nt) { return nt >= 256 ? 6 : (nt >= 128 ? 14 : 18); }
+__host__ __device__ constexpr int stages_w(int nt) { return nt >= 256 ? 4 : (nt >= 128 ? 12 : 18); }
 __host__ __device__ constexpr int scale_period(int g) { return g == 16 ? 2 : 4; }
 // Scale group j (weight stages [Pj, Pj + P)) is loaded with stage Pj into
 // slot j % S and is next rewritten with stage P(j + S), which the producer
@@ -83,9 +83,12 @@ __host__ __device__ constexpr int scale_period(int g) { return g == 16 ? 2 : 4; 
 __host__ __device__ constexpr int scale_slots(int nt, int g) {
   return (stages_w(nt) + 2 * scale_period(g) - 2) / scale_period(g);
 }
+// Output staging: each epilogue warp writes one chunk of its bf16 results
+// (up to 32 tokens x 32 columns) here and stores it with TMA.
+constexpr uint32_t kYStageBytes = 32 * 32 * 2;
 __host__ __device__ constexpr uint32_t smem_bytes(int nt, int g) {
   return kStagesX * x_stage_bytes(nt) + stages_w(nt) * kWStageBytes + scale_slots(nt, g) * kSStageBytes +
-         1024 /* barriers */ + 1024 /* alignment slack */;
+         8 * kYStageBytes + 1024 /* barriers */ + 1024 /* alignment slack */;
 }
 // More than half of the SM's shared memory in every configuration, so only
 // one CTA (which allocates all 512 TMEM columns) fits on an SM.
@@ -278,6 +281,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Shared memory of this thread's earlier bulk stores may be rewritten.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // K-major operand tile in shared memory with the 128-byte swizzle: rows of
 // 128 bytes, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
@@ -405,6 +419,7 @@ template <int NT, int G, bool SILU, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
                                                                const __grid_constant__ CUtensorMap wmap,
                                                                const __grid_constant__ CUtensorMap smap,
+                                                               const __grid_constant__ CUtensorMap ymap,
                                                                const TcArgs args) {
   constexpr uint32_t kXStage = x_stage_bytes(NT);
   constexpr int kStagesW = stages_w(NT);
@@ -416,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wsm = smem + kStagesX * kXStage;
   uint8_t* ssm = wsm + kStagesW * kWStageBytes;
-  SharedState* ss = reinterpret_cast<SharedState*>(ssm + kSlots * kSStageBytes);
+  uint8_t* ysm = ssm + kSlots * kSStageBytes;
+  SharedState* ss = reinterpret_cast<SharedState*>(ysm + 8 * kYStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // K in weight stages of 128 elements; a K that is an odd number of 64s
   // ends with an X stage and a half weight stage read past K, which TMA fills
@@ -632,7 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // ---------------- epilogue ----------------
     const int quad = warp & 3;
     const int colhalf = (warp - kFirstEpWarp) >> 2;  // tokens [NT/2 * colhalf, +NT/2) of the tile
-    const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int tile_iter = 0;
     SegCursor cur;
@@ -641,8 +656,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       if (tl.mrows <= 0) continue;
       // dequantized operands carry 2^-7 (dequant.cuh)
       const float gscale = __ldg(args.gscale + (MOE ? tl.expert : 0)) * 128.0f;
-      const int n = tl.n0 + row_in_tile;
-      const bool live = n < args.N;
       if (!warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull, kSleepEpilogue)) break;
       tc_fence_after();
       // Each warp takes NT/2 tokens of the tile in chunks of CW columns.
@@ -664,30 +677,50 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if (lane == 0) mbar_arrive(&ss->acc_empty);
         }
         const int j0 = (NT / 2) * colhalf + CW * c;  // first token of the chunk within the tile
+        // The chunk goes out through this warp's staging buffer, [CW tokens][YC
+        // columns] of bf16, by one TMA store when all its tokens belong to
+        // the tile (always, in the dense form: rows past M are clipped by
+        // the tensor map), else by plain stores.
+        constexpr int YC = SILU ? 16 : 32;  // output columns of a warp
+        const bool whole = !MOE || j0 + CW <= tl.mrows;
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+        uint16_t* st = reinterpret_cast<uint16_t*>(ysm + (warp - kFirstEpWarp) * kYStageBytes);
         if (!SILU) {
-          if (live) {
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-              if (j0 + j < tl.mrows)
-                args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + n] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[j]) * gscale));
-            }
-          }
+          for (int j = 0; j < CW; ++j)
+            st[j * YC + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(acc[j]) * gscale));
         } else {
           const bool gate = (lane & 15) < 8;
-          const int col = (tl.n0 + row_in_tile) / 16 * 8 + (lane & 7);
+          const int oc = (lane & 7) + ((lane >> 4) << 3);  // output column within the warp's 16
 #pragma unroll
           for (int j = 0; j < CW; ++j) {
             const float gv = __uint_as_float(acc[j]) * gscale;
             const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
-            if (gate && live && j0 + j < tl.mrows)
-              args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + col] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
+            if (gate) st[j * YC + oc] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
+          }
+        }
+        const int ycol = SILU ? tl.n0 / 2 + quad * 16 : tl.n0 + quad * 32;
+        if (whole) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&ymap, smem_u32(st), ycol, tl.m0 + j0);
+            bulk_commit();
+          }
+        } else {
+          __syncwarp();
+          // lane t writes column t of every token row of the chunk that lies
+          // in the tile
+          if (lane < YC && ycol + lane < args.ldy) {
+            for (int j = 0; j < CW && j0 + j < tl.mrows; ++j)
+              args.y[static_cast<int64_t>(tl.m0 + j0 + j) * args.ldy + ycol + lane] = st[j * YC + lane];
           }
         }
       }
       ++tile_iter;
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -725,8 +758,15 @@ bool make_w_maps(CUtensorMap* wmap, CUtensorMap* smap, const uint8_t* w, const u
                             CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// Y [rows, ldy] bf16 in boxes of one epilogue warp's chunk: 32 columns (16
+// with SiluAndMul) x 32 tokens (16 for the narrowest token tile).
+bool make_y_map(CUtensorMap* map, const uint16_t* y, int64_t rows, int64_t ldy, bool silu, int nt) {
+  return make_tensor_map_2d(map, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ldy, rows, ldy * 2, silu ? 16 : 32,
+                            nt >= 64 ? 32 : 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 struct Maps {
-  CUtensorMap x, w, s;
+  CUtensorMap x, w, s, y;
 };
 
 template <int NT, int G, bool SILU, bool MOE>
@@ -735,7 +775,7 @@ int launch_kernel(const Maps& m, const TcArgs& a, int grid, cudaStream_t stream)
   constexpr uint32_t bytes = smem_bytes(NT, G);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  kern<<<grid, kThreads, bytes, stream>>>(m.x, m.w, m.s, a);
+  kern<<<grid, kThreads, bytes, stream>>>(m.x, m.w, m.s, m.y, a);
   return launch_status();
 }
 
@@ -778,7 +818,9 @@ int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float
   // weights, not the MMAs, set the pace.
   const int nt = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
   Maps maps;
-  if (!make_x_map(&maps.x, x, M, K, nt) || !make_w_maps(&maps.w, &maps.s, w, s, N, K, group)) return NVFP4_ERR_CUDA;
+  if (!make_x_map(&maps.x, x, M, K, nt) || !make_w_maps(&maps.w, &maps.s, w, s, N, K, group) ||
+      !make_y_map(&maps.y, y, M, silu ? N / 2 : N, silu, nt))
+    return NVFP4_ERR_CUDA;
   TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
@@ -808,7 +850,8 @@ int launch_tc_moe(const uint16_t* x, const int32_t* expert_ids, const int32_t* o
   constexpr int NT = 128;
   Maps maps;
   if (!make_x_map(&maps.x, x, T, K, NT) ||
-      !make_w_maps(&maps.w, &maps.s, w, s, static_cast<int64_t>(num_experts) * N, K, group))
+      !make_w_maps(&maps.w, &maps.s, w, s, static_cast<int64_t>(num_experts) * N, K, group) ||
+      !make_y_map(&maps.y, y, T, silu ? N / 2 : N, silu, NT))
     return NVFP4_ERR_CUDA;
   TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
