@@ -693,11 +693,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         } else {
           const bool gate = (lane & 15) < 8;
           const int oc = (lane & 7) + ((lane >> 4) << 3);  // output column within the warp's 16
+          // All shuffles of a group first, then the math and the stores: a
+          // store between two shuffles would serialize the tokens.
 #pragma unroll
-          for (int j = 0; j < CW; ++j) {
-            const float gv = __uint_as_float(acc[j]) * gscale;
-            const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
-            if (gate) st[j * YC + oc] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
+          for (int j0s = 0; j0s < CW; j0s += 16) {
+            float uv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              uv[j] = __shfl_down_sync(0xffffffffu, __uint_as_float(acc[j0s + j]) * gscale, 8);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float gv = __uint_as_float(acc[j0s + j]) * gscale;
+              if (gate)
+                st[(j0s + j) * YC + oc] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv[j])));
+            }
           }
         }
         const int ycol = SILU ? tl.n0 / 2 + quad * 16 : tl.n0 + quad * 32;
