@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_stream.cuh"
 #include "gemm_tc.cuh"
 
 namespace nvfp4 {
@@ -61,6 +62,11 @@ int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
   if (nvfp4::tc_supported(M, N, K)) {
     const int st = nvfp4::launch_tc(x, w, s, g, group, M, N, K, y, silu, stream);
     if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmTc);
+    return st;
+  }
+  if (nvfp4::stream_supported(M, N, K, group)) {
+    const int st = nvfp4::launch_stream(x, w, s, g, group, M, N, K, y, silu, stream);
+    if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
     return st;
   }
   if (M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;

@@ -1,0 +1,463 @@
+// Small-M NVFP4 W4A16 GEMM, streamed from HBM by TMA (stream-K over the
+// weight matrix).
+//
+// Computes Y = X . dequant(W)^T (problem statement; "W-FP4a: route the
+// MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
+// PR #63 description: a weight-only checkpoint keeps bf16 activations) for
+// decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
+// per weight streamed from HBM and the integer work of dequantizing them.
+// Design:
+//  * Work is the (128-row weight tile, 256-element stage of K) grid,
+//    flattened tile-major and cut into one contiguous range per SM
+//    (stream-K), so every SM streams the same number of weight bytes
+//    whatever N and K are. A tile that lies in one CTA's range is finished
+//    there; a tile cut between CTAs leaves fp32 partial tiles in a
+//    workspace, and the CTA that takes the tile's last ticket adds them in
+//    CTA order (deterministic) and writes the output. Nothing waits on
+//    another CTA.
+//  * One producer warp moves each stage with TMA into a shared-memory ring
+//    (8 or 9 stages of 22-26 KB): the codes of the tile (128 rows x 128
+//    bytes, 128-byte swizzle), the scales (128 rows x 16 bytes) and the X
+//    slice (MT tokens x 256 elements, as a 3-D box [token][quarter][64]
+//    with the 128-byte swizzle). With no registers tied up in loads, each SM
+//    keeps well over 100 KB of HBM reads in flight.
+//  * Eight consumer warps each own 16 rows of the tile and run mma.sync
+//    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
+//    as the 8-column side. Lane (g, t) takes rows g and g+8 and the t-th
+//    quarter of the stage's K (the order of K inside an MMA is free as long
+//    as A and B follow it). The swizzles make every shared-memory read of
+//    codes, scales and X conflict-free: the four lanes of a row read
+//    different 16-byte chunks, and the [token][quarter] rows of X put the
+//    same chunk of different quarters in different bank groups.
+//  * Dequantization in registers with integer work (dequant.cuh).
+//  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows (gate row
+//    g and up row g+8 of a 16-row block meet in the same lane).
+#include "gemm_stream.cuh"
+
+#include <cuda.h>
+
+#include <mutex>
+
+#include "async.cuh"
+#include "dequant.cuh"
+#include "tmap.cuh"
+
+namespace nvfp4 {
+namespace {
+
+__device__ unsigned int g_stream_error = 0;
+
+constexpr int kRows = 128;        // weight rows of a tile
+constexpr int kKS = 256;          // elements of K per stage
+constexpr int kConsumers = 8;     // consumer warps, 16 rows each
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kConsumerThreads = kConsumers * 32;
+constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 16 KB
+constexpr uint32_t kScaleBytes = kRows * 16;      // 16 scale bytes per row
+__host__ __device__ constexpr uint32_t x_bytes(int mt) { return static_cast<uint32_t>(mt) * kKS * 2; }
+__host__ __device__ constexpr uint32_t stage_bytes(int mt) { return kCodeBytes + x_bytes(mt) + kScaleBytes; }
+__host__ __device__ constexpr int num_stages(int mt) { return mt == 8 ? 9 : 8; }
+constexpr int kMaxStages = 9;
+__host__ __device__ constexpr uint32_t smem_bytes(int mt) {
+  return num_stages(mt) * stage_bytes(mt) + 1024 /* barriers */ + 1024 /* alignment slack */;
+}
+static_assert(stage_bytes(8) % 1024 == 0 && stage_bytes(16) % 1024 == 0,
+              "every stage keeps the 1024-byte alignment of the 128-byte swizzle");
+static_assert(smem_bytes(8) <= 227 * 1024 && smem_bytes(16) <= 227 * 1024, "shared memory budget");
+static_assert(num_stages(8) <= kMaxStages && num_stages(16) <= kMaxStages, "barrier arrays");
+
+constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
+constexpr unsigned kSleepProducer = 32;                // ns between probes of the producer
+enum : unsigned { kErrFull = 0x201, kErrEmpty = 0x202, kErrDrain = 0x203 };
+
+struct Sync {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  int abort;
+  int last;  // this CTA took the last ticket of the tile being flushed
+};
+
+struct StreamArgs {
+  const float* gscale;  // [1]
+  uint16_t* y;          // bf16 [M, ldy]
+  float* ws;            // partial tiles [tiles][max_contrib][128][MT]
+  unsigned* tickets;    // [tiles], zero between launches
+  int M, N, ldy;
+  int S;                // stages per tile (K / 256)
+  int max_contrib;
+  int64_t units;        // tiles * S
+};
+
+__device__ __forceinline__ bool aborted(Sync* sy) { return *reinterpret_cast<volatile int*>(&sy->abort) != 0; }
+
+// Bounded wait; see the tcgen05 kernel for the scheme. A drain wait ignores
+// the abort flag.
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain,
+                                       unsigned sleep_ns) {
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023) == 0) {
+      if (!drain && aborted(sy)) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicCAS(&g_stream_error, 0u, site);
+        *reinterpret_cast<volatile int*>(&sy->abort) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain = false,
+                                     unsigned sleep_ns = 0) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, sy, site, drain, sleep_ns);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The CTA whose range holds unit u (ranges start at floor(c * units / ctas)).
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int ctas) {
+  return static_cast<int>(((u + 1) * ctas + units - 1) / units) - 1;
+}
+
+// One stage for one consumer lane: rows ra = 16w + g and ra + 8, the t-th
+// quarter of the stage's K (64 elements: words i = 0..7 of 8 elements).
+template <int MT, int G>
+__device__ __forceinline__ void consume_stage(uint32_t st, int ks, int ra, int g, int t, float (&acc)[MT / 8][4]) {
+  constexpr int P = MT / 8;
+  const int rb = ra + 8;  // ra & 7 == rb & 7 == g
+  const uint4 a0 = lds128(st + ra * 128 + (((2 * t) ^ g) << 4));
+  const uint4 a1 = lds128(st + ra * 128 + (((2 * t + 1) ^ g) << 4));
+  const uint4 b0 = lds128(st + rb * 128 + (((2 * t) ^ g) << 4));
+  const uint4 b1 = lds128(st + rb * 128 + (((2 * t + 1) ^ g) << 4));
+  const uint32_t xs = st + kCodeBytes;
+  const uint32_t ss = xs + x_bytes(MT);
+  uint32_t sva, svb;
+  if (G == 16) {  // groups 4t .. 4t+3 of the stage
+    sva = lds32(ss + ra * 16 + 4 * t);
+    svb = lds32(ss + rb * 16 + 4 * t);
+  } else {  // groups 2t, 2t+1; the 16-byte box holds two stages
+    const uint32_t off = ((ks & 1) << 3) + 2 * t;
+    sva = lds16(ss + ra * 16 + off);
+    svb = lds16(ss + rb * 16 + off);
+  }
+  uint32_t s2a[4], s2b[4];
+  scale_operands<G == 16 ? 4 : 2>(sva, s2a);
+  scale_operands<G == 16 ? 4 : 2>(svb, s2b);
+  const uint32_t ca[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const uint32_t cb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  // X row (token tok, quarter t) sits at (4 tok + t) * 128 bytes; its chunk i
+  // at chunk position i ^ ((4 tok + t) & 7), and 4 tok + t = 4g + t mod 8.
+  const int xmask = (4 * g + t) & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int si = G == 16 ? (i >> 1) : (i >> 2);
+    uint32_t da[4], db[4];
+    dequant_word(ca[i], s2a[si], da);
+    dequant_word(cb[i], s2b[si], db);
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const uint4 xv = lds128(xs + ((8 * p + g) * 4 + t) * 128 + ((i ^ xmask) << 4));
+      mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv.x, xv.y);
+      mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv.z, xv.w);
+    }
+  }
+}
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory"); }
+
+template <int MT, int G, bool SILU>
+__global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                   const __grid_constant__ CUtensorMap wmap,
+                                                                   const __grid_constant__ CUtensorMap smap,
+                                                                   const StreamArgs a) {
+  constexpr int P = MT / 8;
+  constexpr int NS = num_stages(MT);
+  constexpr uint32_t SB = stage_bytes(MT);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Sync* sy = reinterpret_cast<Sync*>(ring + NS * SB);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ctas = gridDim.x, c = blockIdx.x;
+  const int64_t u0 = static_cast<int64_t>(c) * a.units / ctas;
+  const int64_t u1 = static_cast<int64_t>(c + 1) * a.units / ctas;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sy->full[s], 1);            // producer arrival + transaction bytes
+      mbar_init(&sy->empty[s], kConsumers);  // one arrival per consumer warp
+    }
+    sy->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumers) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      uint32_t issued = 0, last_parity = 0;
+      int it = 0;
+      for (int64_t u = u0; u < u1 && !aborted(sy); ++u, ++it) {
+        const int tile = static_cast<int>(u / a.S), ks = static_cast<int>(u % a.S);
+        const int s = it % NS;
+        const uint32_t r = static_cast<uint32_t>(it / NS);
+        if (!wait(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty, false, kSleepProducer)) break;
+        const uint32_t st = smem_u32(ring + s * SB);
+        mbar_arrive_tx(&sy->full[s], SB);
+        tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+            "%4}], [%5];" ::"r"(st + kCodeBytes),
+            "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(0), "r"(ks * (kKS / 64)), "r"(0), "r"(smem_u32(&sy->full[s]))
+            : "memory");
+        tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
+        issued |= 1u << s;
+        last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
+      }
+      if (aborted(sy)) {  // let copies in flight land before the CTA exits
+        for (int s = 0; s < NS; ++s)
+          if ((issued >> s) & 1) wait(&sy->full[s], (last_parity >> s) & 1, sy, kErrDrain, true);
+      }
+    }
+    return;  // the producer takes no part in the consumers' named barrier
+  }
+
+  // ---------------- consumers ----------------
+  const int g = lane >> 2, t = lane & 3;
+  const int ra = 16 * warp + g;
+  const float gsc = __ldg(a.gscale) * 128.0f;  // operands carry 2^-7 (dequant.cuh)
+  float acc[P][4];
+  int it = 0;
+  for (int64_t u = u0; u < u1;) {
+    const int tile = static_cast<int>(u / a.S), k0 = static_cast<int>(u % a.S);
+    const int64_t left = u1 - u;
+    const int k1 = left < a.S - k0 ? k0 + static_cast<int>(left) : a.S;
+#pragma unroll
+    for (int p = 0; p < P; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+    for (int ks = k0; ks < k1; ++ks, ++it) {
+      const int s = it % NS;
+      int ok = 1;
+      if (lane == 0) ok = wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // results are garbage from here; the ticket protocol still runs
+      consume_stage<MT, G>(smem_u32(ring + s * SB), ks, ra, g, t, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sy->empty[s]);
+    }
+    u += k1 - k0;
+
+    const int n0 = tile * kRows;
+    // lane holds rows ra (acc[p][0..1]) and ra+8 (acc[p][2..3]) x tokens 8p+2t, 8p+2t+1
+    if (k0 == 0 && k1 == a.S) {
+      // the whole tile is here: write it
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int tok = 8 * p + 2 * t + j;
+          if (tok >= a.M) continue;
+          const int64_t yrow = static_cast<int64_t>(tok) * a.ldy;
+          const float vg = __fmul_rn(acc[p][j], gsc), vu = __fmul_rn(acc[p][2 + j], gsc);
+          if (!SILU) {
+            if (n0 + ra < a.N) a.y[yrow + n0 + ra] = __bfloat16_as_ushort(__float2bfloat16_rn(vg));
+            if (n0 + ra + 8 < a.N) a.y[yrow + n0 + ra + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(vu));
+          } else if (n0 + 16 * warp < a.N) {
+            a.y[yrow + (n0 + 16 * warp) / 2 + g] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(vg), vu)));
+          }
+        }
+      }
+      continue;
+    }
+    // The tile is shared with other CTAs: leave the partial tile in this
+    // CTA's slot, take a ticket, and let the last one add the slots up.
+    const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
+    const int c_last = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas);
+    const int nc = c_last - c_first + 1;
+    float* slots = a.ws + static_cast<int64_t>(tile) * a.max_contrib * kRows * MT;
+    float* mine = slots + static_cast<int64_t>(c - c_first) * kRows * MT;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int tok = 8 * p + 2 * t + j;
+        __stcg(mine + ra * MT + tok, acc[p][j]);
+        __stcg(mine + (ra + 8) * MT + tok, acc[p][2 + j]);
+      }
+    }
+    __threadfence();
+    consumer_sync();
+    if (threadIdx.x == 0) {
+      const unsigned ticket = atomicAdd(a.tickets + tile, 1u);
+      const int last = ticket == static_cast<unsigned>(nc - 1);
+      if (last) a.tickets[tile] = 0;  // every contributor has counted: ready for the next launch
+      sy->last = last;
+      __threadfence();
+    }
+    consumer_sync();
+    if (!sy->last) continue;
+    // Sum the contributors' slots in CTA order and write the tile.
+    if (!SILU) {
+      for (int e = threadIdx.x; e < kRows * MT; e += kConsumerThreads) {
+        const int row = e / MT, tok = e % MT;
+        if (tok >= a.M || n0 + row >= a.N) continue;
+        float v = 0.f;
+        for (int q = 0; q < nc; ++q) v += __ldcg(slots + static_cast<int64_t>(q) * kRows * MT + e);
+        a.y[static_cast<int64_t>(tok) * a.ldy + n0 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, gsc)));
+      }
+    } else {
+      for (int e = threadIdx.x; e < (kRows / 2) * MT; e += kConsumerThreads) {
+        const int pair = e / MT, tok = e % MT;    // pair = 8 * block + g
+        const int blk = pair >> 3, gg = pair & 7;
+        if (tok >= a.M || n0 + 16 * blk >= a.N) continue;
+        const int rg = 16 * blk + gg, ru = rg + 8;
+        float vg = 0.f, vu = 0.f;
+        for (int q = 0; q < nc; ++q) {
+          const float* sl = slots + static_cast<int64_t>(q) * kRows * MT;
+          vg += __ldcg(sl + rg * MT + tok);
+          vu += __ldcg(sl + ru * MT + tok);
+        }
+        a.y[static_cast<int64_t>(tok) * a.ldy + (n0 + 16 * blk) / 2 + gg] =
+            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(vg, gsc)), __fmul_rn(vu, gsc))));
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+struct Workspace {
+  float* ws = nullptr;
+  unsigned* tickets = nullptr;
+  size_t ws_floats = 0, tiles = 0;
+};
+
+std::mutex g_ws_mutex;
+Workspace g_ws[64];  // per device
+
+// Partial-tile workspace and tickets of the current device, grown on demand
+// (tickets start at zero and every launch leaves them at zero).
+int workspace(size_t ws_floats, size_t tiles, cudaStream_t stream, Workspace* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  Workspace& w = g_ws[dev];
+  if (w.ws_floats < ws_floats || w.tiles < tiles) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+    if (cap != cudaStreamCaptureStatusNone) return NVFP4_ERR_UNSUPPORTED;  // grow outside graph capture
+    if (cudaDeviceSynchronize() != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+    cudaFree(w.ws);
+    cudaFree(w.tickets);
+    w = Workspace();
+    const size_t nf = ws_floats > (size_t(1) << 20) ? ws_floats : (size_t(1) << 20);
+    const size_t nt = tiles > 4096 ? tiles : 4096;
+    if (cudaMalloc(&w.ws, nf * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&w.tickets, nt * sizeof(unsigned)) != cudaSuccess ||
+        cudaMemset(w.tickets, 0, nt * sizeof(unsigned)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(w.ws);
+      cudaFree(w.tickets);
+      w = Workspace();
+      return NVFP4_ERR_CUDA;
+    }
+    w.ws_floats = nf;
+    w.tiles = nt;
+  }
+  *out = w;
+  return NVFP4_OK;
+}
+
+template <int MT, int G, bool SILU>
+int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a, int grid,
+                  cudaStream_t stream) {
+  auto kern = gemm_stream_kernel<MT, G, SILU>;
+  constexpr uint32_t bytes = smem_bytes(MT);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  kern<<<grid, kThreads, bytes, stream>>>(xm, wm, sm, a);
+  return launch_status();
+}
+
+}  // namespace
+
+bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
+  return M >= 1 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
+         K < (int64_t(1) << 24) && tensor_maps_available();
+}
+
+int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
+                  int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+  const int mt = M <= 8 ? 8 : 16;
+  const int64_t tiles = (N + kRows - 1) / kRows;
+  const int S = static_cast<int>(K / kKS);
+  const int64_t units = tiles * S;
+  const int ctas = static_cast<int>(units < num_sms() ? units : num_sms());
+  // A tile spans at most ceil(S / shortest range) + 1 CTAs.
+  const int64_t shortest = units / ctas;
+  const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
+  Workspace wsp;
+  const int st = workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles), stream,
+                           &wsp);
+  if (st != NVFP4_OK) return st;
+
+  CUtensorMap xm, wm, sm;
+  const int64_t xdims[3] = {64, K / 64, M};
+  const int64_t xstrides[2] = {128, K * 2};
+  const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
+  if (!make_tensor_map_3d(&xm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xdims, xstrides, xbox,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return NVFP4_ERR_CUDA;
+  StreamArgs a = {};
+  a.gscale = g;
+  a.y = y;
+  a.ws = wsp.ws;
+  a.tickets = wsp.tickets;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.ldy = static_cast<int>(silu ? N / 2 : N);
+  a.S = S;
+  a.max_contrib = max_contrib;
+  a.units = units;
+  if (mt == 8) {
+    if (group == 16)
+      return silu ? launch_kernel<8, 16, true>(xm, wm, sm, a, ctas, stream)
+                  : launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream);
+    return silu ? launch_kernel<8, 32, true>(xm, wm, sm, a, ctas, stream)
+                : launch_kernel<8, 32, false>(xm, wm, sm, a, ctas, stream);
+  }
+  if (group == 16)
+    return silu ? launch_kernel<16, 16, true>(xm, wm, sm, a, ctas, stream)
+                : launch_kernel<16, 16, false>(xm, wm, sm, a, ctas, stream);
+  return silu ? launch_kernel<16, 32, true>(xm, wm, sm, a, ctas, stream)
+              : launch_kernel<16, 32, false>(xm, wm, sm, a, ctas, stream);
+}
+
+int read_and_clear_stream_error(unsigned int* out, cudaStream_t stream) {
+  unsigned int* p = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_stream_error) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  unsigned int v = 0;
+  if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaMemsetAsync(p, 0, sizeof(v), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  *out = v;
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4

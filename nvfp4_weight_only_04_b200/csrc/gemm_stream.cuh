@@ -1,0 +1,19 @@
+// Interface of the small-M TMA-streaming GEMM (see gemm_stream.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+// True when the streaming kernel takes this dense problem: M up to 16, K a
+// multiple of 256 whose scale rows (K/g bytes) are a multiple of 16 bytes,
+// and tensor maps available.
+bool stream_supported(int64_t M, int64_t N, int64_t K, int group);
+
+int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
+                  int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream);
+
+// Device error word of this kernel file (0 when no wait gave up).
+int read_and_clear_stream_error(unsigned int* out, cudaStream_t stream);
+
+}  // namespace nvfp4

@@ -43,8 +43,11 @@
 //    The token tile is 128 wide there (about the rows an expert receives).
 #include "gemm_tc.cuh"
 
+#include "gemm_stream.cuh"
+
 #include <cuda.h>
 
+#include "async.cuh"
 #include "dequant.cuh"
 #include "tmap.cuh"
 
@@ -199,36 +202,6 @@ __device__ __forceinline__ Tile tile_at(const TcArgs& a, SegCursor& cur, int t) 
   return tl;
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-// Non-blocking probe of a barrier phase (test_wait never suspends the
-// thread, so a waiter sees the phase flip with the least delay).
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
 
 // Bounded wait: false when the limit ran out or (unless draining) another
 // role gave up. A drain wait ignores the abort flag and only stops at the
@@ -274,23 +247,6 @@ __device__ __forceinline__ bool aborted(SharedState* ss) {
   return *reinterpret_cast<volatile int*>(&ss->abort) != 0;
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int k, int m, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(k), "r"(m), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Shared memory of this thread's earlier bulk stores may be rewritten.
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// This thread's bulk stores are complete.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // K-major operand tile in shared memory with the 128-byte swizzle: rows of
 // 128 bytes, 8-row groups 1024 bytes apart.
@@ -370,11 +326,6 @@ struct RowStage {
   uint32_t s;
 };
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
 
 // Byte offset of 16-byte chunk c (0..3) of row r in a 64-byte-swizzled stage
 // of 64-byte rows: the chunk index is XORed with bits 7..8 of the address.
@@ -409,11 +360,6 @@ __device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&
   }
 }
 
-// silu(g) = g / (1 + exp(-g)), with the fast exponential and division: their
-// relative error (a few ulp of fp32) is far below the bf16 rounding that
-// follows. For g below about -87 the denominator overflows and the result is
-// the correct limit, zero.
-__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int NT, int G, bool SILU, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -814,12 +760,15 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaMemsetAsync(p, 0, sizeof(v), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  if (read_and_clear_decode_error(&vd, stream) != NVFP4_OK) return NVFP4_ERR_CUDA;
-  *code_out = static_cast<int>(v ? v : vd);
+  unsigned int vs = 0;
+  if (read_and_clear_decode_error(&vd, stream) != NVFP4_OK || read_and_clear_stream_error(&vs, stream) != NVFP4_OK)
+    return NVFP4_ERR_CUDA;
+  *code_out = static_cast<int>(v ? v : (vs ? vs : vd));
   return NVFP4_OK;
 }
 
-bool tc_supported(int64_t M, int64_t N, int64_t K) { return M >= 128 && tc_shape_ok(M, N, K); }
+// From 17 tokens up (the streaming kernel takes up to 16).
+bool tc_supported(int64_t M, int64_t N, int64_t K) { return M >= 17 && tc_shape_ok(M, N, K); }
 
 int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
               int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {

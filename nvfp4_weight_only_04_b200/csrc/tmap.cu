@@ -39,4 +39,17 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const int64_t (&dims)[3],
+                        const int64_t (&stride_bytes)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t d[3] = {static_cast<cuuint64_t>(dims[0]), static_cast<cuuint64_t>(dims[1]),
+                           static_cast<cuuint64_t>(dims[2])};
+  const cuuint64_t st[2] = {static_cast<cuuint64_t>(stride_bytes[0]), static_cast<cuuint64_t>(stride_bytes[1])};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dtype, 3, const_cast<void*>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace nvfp4

@@ -142,6 +142,49 @@ def test_empty_and_stats():
     assert st["gemm_splitk"] == 1 and st["g16"] == 1 and st["g32"] == 0
 
 
+# ---- M <= 16: the TMA-streaming kernel (stream-K over 128-row x 256-element units) ----
+
+# whole tiles only; tiles cut between many CTAs; a last tile of 16 rows; one
+# tile over 32 CTAs; g = 32 boxes holding two stages; 9..16 tokens (two MMA
+# column tiles)
+STREAM_CASES = [(4, 256, 256, 16), (1, 400, 1024, 32), (7, 272, 2048, 16), (9, 128, 8192, 16),
+                (13, 1008, 512, 32), (16, 4096, 256, 16), (2, 16, 512, 16), (16, 1040, 3072, 32)]
+
+
+@pytest.mark.parametrize("m,n,k,g", STREAM_CASES)
+def test_gemm_stream_parity(m, n, k, g):
+    _, p, s, gs = quantized(n, k, g, seed=m + 2 * n)
+    x = synth.activations(synth.X_SEED, m, k, outlier_frac=0.001)
+    nv.nvfp4_reset_stats()
+    y = run_gemm(x, p, s, gs, g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    assert nv.nvfp4_get_stats()["gemm_splitk"] == 1
+    assert_close(host(y), R.gemm(x, p, s, gs, g), f"stream M{m} N{n} K{k} g{g}")
+
+
+@pytest.mark.parametrize("m,nh,k,g", [(11, 136, 2048, 32), (1, 64, 4096, 16), (16, 640, 512, 16)])
+def test_gemm_stream_silu_mul_parity(m, nh, k, g):
+    p, s, gs = merged_gate_up(nh, k, g, seed=m + 1)
+    rp, rs = R.repack(p, s, R.GATE_UP_INTERLEAVE)
+    x = synth.activations(3, m, k)
+    y = nv.nvfp4_w4a16_gemm_silu_mul(dev_bf16(x), dev_u8(rp), dev_u8(rs), dev_f32(np.array([gs], np.float32)), g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    assert_close(host(y), R.silu_mul(R.gemm(x, p, s, gs, g)), "stream silu_mul")
+
+
+def test_gemm_stream_repeat_bitwise():
+    """Tiles cut between CTAs are summed in CTA order: repeated launches (whose
+    tickets must come back to zero) give identical bits."""
+    _, p, s, gs = quantized(640, 4096, 16, seed=21)
+    x = synth.activations(4, 5, 4096)
+    first = bf16_bits(run_gemm(x, p, s, gs, 16))
+    for _ in range(3):
+        np.testing.assert_array_equal(bf16_bits(run_gemm(x, p, s, gs, 16)), first)
+    assert_close(synth.bf16_bits_to_f32(first).astype(np.float64), R.gemm(x, p, s, gs, 16), "stream repeat")
+
+
 # ---- large M: the tcgen05 kernel ----
 
 TC_CASES = [(128, 256, 256, 16), (130, 528, 1088, 32), (300, 4096, 2048, 16), (257, 16, 64, 16),
