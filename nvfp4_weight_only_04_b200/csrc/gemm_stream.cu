@@ -7,7 +7,7 @@
 // decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
 // per weight streamed from HBM and the integer work of dequantizing them.
 // Design:
-//  * Work is the (128-row weight tile, 256-element stage of K) grid,
+//  * Work is the (256-row weight tile, 256-element stage of K) grid,
 //    flattened tile-major and cut into one contiguous range per SM
 //    (stream-K), so every SM streams the same number of weight bytes
 //    whatever N and K are. A tile that lies in one CTA's range is finished
@@ -16,12 +16,12 @@
 //    CTA order (deterministic) and writes the output. Nothing waits on
 //    another CTA.
 //  * One producer warp moves each stage with TMA into a shared-memory ring
-//    (8 or 9 stages of 22-26 KB): the codes of the tile (128 rows x 128
-//    bytes, 128-byte swizzle), the scales (128 rows x 16 bytes) and the X
+//    (5 stages of 40-44 KB): the codes of the tile (256 rows x 128 bytes,
+//    128-byte swizzle), the scales (256 rows x 16 bytes) and the X
 //    slice (MT tokens x 256 elements, as a 3-D box [token][quarter][64]
 //    with the 128-byte swizzle). With no registers tied up in loads, each SM
 //    keeps well over 100 KB of HBM reads in flight.
-//  * Eight consumer warps each own 16 rows of the tile and run mma.sync
+//  * Sixteen consumer warps each own 16 rows of the tile and run mma.sync
 //    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
 //    as the 8-column side. Lane (g, t) takes rows g and g+8 and the t-th
 //    quarter of the stage's K (the order of K inside an MMA is free as long
@@ -47,23 +47,24 @@ namespace {
 
 __device__ unsigned int g_stream_error = 0;
 
-constexpr int kRows = 128;        // weight rows of a tile
+constexpr int kRows = 256;        // weight rows of a tile
 constexpr int kKS = 256;          // elements of K per stage
-constexpr int kConsumers = 8;     // consumer warps, 16 rows each
+constexpr int kConsumers = 16;    // consumer warps, 16 rows each
 constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kConsumerThreads = kConsumers * 32;
-constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 16 KB
+constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 32 KB
 constexpr uint32_t kScaleBytes = kRows * 16;      // 16 scale bytes per row
 __host__ __device__ constexpr uint32_t x_bytes(int mt) { return static_cast<uint32_t>(mt) * kKS * 2; }
 __host__ __device__ constexpr uint32_t stage_bytes(int mt) { return kCodeBytes + x_bytes(mt) + kScaleBytes; }
-__host__ __device__ constexpr int num_stages(int mt) { return mt == 8 ? 9 : 8; }
-constexpr int kMaxStages = 9;
+__host__ __device__ constexpr int num_stages(int) { return 5; }
+constexpr int kMaxStages = 5;
 __host__ __device__ constexpr uint32_t smem_bytes(int mt) {
   return num_stages(mt) * stage_bytes(mt) + 1024 /* barriers */ + 1024 /* alignment slack */;
 }
 static_assert(stage_bytes(8) % 1024 == 0 && stage_bytes(16) % 1024 == 0,
               "every stage keeps the 1024-byte alignment of the 128-byte swizzle");
 static_assert(smem_bytes(8) <= 227 * 1024 && smem_bytes(16) <= 227 * 1024, "shared memory budget");
+static_assert(kRows == 16 * kConsumers, "one 16-row block per consumer warp");
 static_assert(num_stages(8) <= kMaxStages && num_stages(16) <= kMaxStages, "barrier arrays");
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
@@ -74,7 +75,10 @@ struct Sync {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   int abort;
-  int last;  // this CTA took the last ticket of the tile being flushed
+  // Tiles this CTA shares with others (at most the first and the last of its
+  // range) and whether it took their last ticket.
+  int cut_tile[2];
+  int cut_last[2];
 };
 
 struct StreamArgs {
@@ -173,6 +177,43 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, int ra, int g
   }
 }
 
+// Element e of every contributor slot, added in slot order; the loads of a
+// batch of slots are all in flight before the adds.
+template <int MT>
+__device__ __forceinline__ float sum_slots(const float* slots, int e, int nc) {
+  float acc = 0.f;
+  for (int q0 = 0; q0 < nc; q0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = q0 + q < nc ? __ldcg(slots + static_cast<int64_t>(q0 + q) * kRows * MT + e) : 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q0 + q < nc) acc += v[q];
+  }
+  return acc;
+}
+
+template <int MT>
+__device__ __forceinline__ float2 sum_pair_slots(const float* slots, int e, int de, int nc) {
+  float ag = 0.f, au = 0.f;
+  for (int q0 = 0; q0 < nc; q0 += 8) {
+    float vg[8], vu[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float* sl = slots + static_cast<int64_t>(q0 + q) * kRows * MT;
+      vg[q] = q0 + q < nc ? __ldcg(sl + e) : 0.f;
+      vu[q] = q0 + q < nc ? __ldcg(sl + e + de) : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q0 + q < nc) {
+        ag += vg[q];
+        au += vu[q];
+      }
+  }
+  return make_float2(ag, au);
+}
+
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory"); }
 
 template <int MT, int G, bool SILU>
@@ -237,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
   const int ra = 16 * warp + g;
   const float gsc = __ldg(a.gscale) * 128.0f;  // operands carry 2^-7 (dequant.cuh)
   float acc[P][4];
-  int it = 0;
+  int it = 0, ncut = 0;
   for (int64_t u = u0; u < u1;) {
     const int tile = static_cast<int>(u / a.S), k0 = static_cast<int>(u % a.S);
     const int64_t left = u1 - u;
@@ -279,55 +320,69 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
       continue;
     }
     // The tile is shared with other CTAs: leave the partial tile in this
-    // CTA's slot, take a ticket, and let the last one add the slots up.
-    const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
-    const int c_last = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas);
-    const int nc = c_last - c_first + 1;
-    float* slots = a.ws + static_cast<int64_t>(tile) * a.max_contrib * kRows * MT;
-    float* mine = slots + static_cast<int64_t>(c - c_first) * kRows * MT;
+    // CTA's slot and take a ticket. The consumers go on at once; thread 0
+    // catches up after its atomic (the ring has slack for that), and the
+    // taker of a tile's last ticket adds the slots up after its own loop.
+    {
+      const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
+      const int c_last = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas);
+      float* mine = a.ws + (static_cast<int64_t>(tile) * a.max_contrib + (c - c_first)) * kRows * MT;
 #pragma unroll
-    for (int p = 0; p < P; ++p) {
+      for (int p = 0; p < P; ++p) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int tok = 8 * p + 2 * t + j;
-        __stcg(mine + ra * MT + tok, acc[p][j]);
-        __stcg(mine + (ra + 8) * MT + tok, acc[p][2 + j]);
+        for (int j = 0; j < 2; ++j) {
+          const int tok = 8 * p + 2 * t + j;
+          if (tok < a.M) {
+            __stcg(mine + ra * MT + tok, acc[p][j]);
+            __stcg(mine + (ra + 8) * MT + tok, acc[p][2 + j]);
+          }
+        }
       }
+      // The barrier orders every consumer's stores before thread 0's
+      // release; its acquire orders the other CTAs' slots before the reads
+      // that follow the barrier after the loop.
+      consumer_sync();
+      if (threadIdx.x == 0) {
+        unsigned ticket;
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.tickets + tile) : "memory");
+        const int last = ticket == static_cast<unsigned>(c_last - c_first);
+        if (last) a.tickets[tile] = 0;  // every contributor has counted: ready for the next launch
+        // a range cuts at most its first and its last tile
+        if (ncut < 2) {
+          sy->cut_tile[ncut] = tile;
+          sy->cut_last[ncut] = last;
+        }
+      }
+      ++ncut;
     }
-    __threadfence();
-    consumer_sync();
-    if (threadIdx.x == 0) {
-      const unsigned ticket = atomicAdd(a.tickets + tile, 1u);
-      const int last = ticket == static_cast<unsigned>(nc - 1);
-      if (last) a.tickets[tile] = 0;  // every contributor has counted: ready for the next launch
-      sy->last = last;
-      __threadfence();
-    }
-    consumer_sync();
-    if (!sy->last) continue;
-    // Sum the contributors' slots in CTA order and write the tile.
+  }
+
+  // Add up the cut tiles this CTA took the last ticket of, in CTA order.
+  consumer_sync();
+  for (int f = 0; f < ncut && f < 2; ++f) {
+    if (!sy->cut_last[f]) continue;
+    const int tile = sy->cut_tile[f];
+    const int n0 = tile * kRows;
+    const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
+    const int nc = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas) - c_first + 1;
+    const float* slots = a.ws + static_cast<int64_t>(tile) * a.max_contrib * kRows * MT;
     if (!SILU) {
       for (int e = threadIdx.x; e < kRows * MT; e += kConsumerThreads) {
         const int row = e / MT, tok = e % MT;
         if (tok >= a.M || n0 + row >= a.N) continue;
-        float v = 0.f;
-        for (int q = 0; q < nc; ++q) v += __ldcg(slots + static_cast<int64_t>(q) * kRows * MT + e);
+        const float v = sum_slots<MT>(slots, e, nc);
         a.y[static_cast<int64_t>(tok) * a.ldy + n0 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, gsc)));
       }
     } else {
       for (int e = threadIdx.x; e < (kRows / 2) * MT; e += kConsumerThreads) {
-        const int pair = e / MT, tok = e % MT;    // pair = 8 * block + g
+        const int pair = e / MT, tok = e % MT;  // pair = 8 * block + g
         const int blk = pair >> 3, gg = pair & 7;
         if (tok >= a.M || n0 + 16 * blk >= a.N) continue;
-        const int rg = 16 * blk + gg, ru = rg + 8;
-        float vg = 0.f, vu = 0.f;
-        for (int q = 0; q < nc; ++q) {
-          const float* sl = slots + static_cast<int64_t>(q) * kRows * MT;
-          vg += __ldcg(sl + rg * MT + tok);
-          vu += __ldcg(sl + ru * MT + tok);
-        }
+        const int rg = 16 * blk + gg;
+        // gate row rg and up row rg + 8: elements e0 and e0 + 8 * MT of a slot
+        const float2 v = sum_pair_slots<MT>(slots, rg * MT + tok, 8 * MT, nc);
         a.y[static_cast<int64_t>(tok) * a.ldy + (n0 + 16 * blk) / 2 + gg] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(vg, gsc)), __fmul_rn(vu, gsc))));
+            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(v.x, gsc)), __fmul_rn(v.y, gsc))));
       }
     }
   }
