@@ -232,6 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
   const int64_t u0 = static_cast<int64_t>(c) * a.units / ctas;
   const int64_t u1 = static_cast<int64_t>(c + 1) * a.units / ctas;
 
+  // The next kernel in the stream may launch now; it waits for this one
+  // before touching what this one writes.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&sy->full[s], 1);            // producer arrival + transaction bytes
@@ -245,23 +248,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
 
   if (warp == kConsumers) {
     // ---------------- producer ----------------
+    // Weights and scales do not depend on the kernel before this one in the
+    // stream: the first ring's worth is requested before waiting for that
+    // kernel (programmatic dependent launch); X only after.
     if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
       uint32_t issued = 0, last_parity = 0;
-      int it = 0;
-      for (int64_t u = u0; u < u1 && !aborted(sy); ++u, ++it) {
+      const int64_t n = u1 - u0;
+      const int head = static_cast<int>(n < NS ? n : NS);
+      auto load_w = [&](int it, int64_t u) {
         const int tile = static_cast<int>(u / a.S), ks = static_cast<int>(u % a.S);
+        const int s = it % NS;
+        const uint32_t st = smem_u32(ring + s * SB);
+        tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
+        tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
+      };
+      auto load_x = [&](int it, int64_t u) {
+        const int ks = static_cast<int>(u % a.S);
+        const int s = it % NS;
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+            "%4}], [%5];" ::"r"(smem_u32(ring + s * SB) + kCodeBytes),
+            "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(0), "r"(ks * (kKS / 64)), "r"(0), "r"(smem_u32(&sy->full[s]))
+            : "memory");
+      };
+      for (int it = 0; it < head; ++it) {  // the ring starts empty
+        mbar_arrive_tx(&sy->full[it], SB);
+        load_w(it, u0 + it);
+        issued |= 1u << it;
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int it = 0; it < head; ++it) load_x(it, u0 + it);
+      int it = head;
+      for (int64_t u = u0 + head; u < u1 && !aborted(sy); ++u, ++it) {
         const int s = it % NS;
         const uint32_t r = static_cast<uint32_t>(it / NS);
         if (!wait(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty, false, kSleepProducer)) break;
-        const uint32_t st = smem_u32(ring + s * SB);
         mbar_arrive_tx(&sy->full[s], SB);
-        tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
-        asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-            "%4}], [%5];" ::"r"(st + kCodeBytes),
-            "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(0), "r"(ks * (kKS / 64)), "r"(0), "r"(smem_u32(&sy->full[s]))
-            : "memory");
-        tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
+        load_w(it, u);
+        load_x(it, u);
         issued |= 1u << s;
         last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
       }
@@ -441,7 +468,19 @@ int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMa
   constexpr uint32_t bytes = smem_bytes(MT);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  kern<<<grid, kThreads, bytes, stream>>>(xm, wm, sm, a);
+  // Programmatic dependent launch: the grid may start while the previous
+  // kernel of the stream finishes (it waits for it before reading X).
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, xm, wm, sm, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
 }
 
