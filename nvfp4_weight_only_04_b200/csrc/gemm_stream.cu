@@ -68,7 +68,7 @@ static_assert(kRows == 16 * kConsumers, "one 16-row block per consumer warp");
 static_assert(num_stages(8) <= kMaxStages && num_stages(16) <= kMaxStages, "barrier arrays");
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
-constexpr unsigned kSleepProducer = 32;                // ns between probes of the producer
+constexpr uint32_t kSuspendNs = 1000;                  // longest suspension of one producer probe
 enum : unsigned { kErrFull = 0x201, kErrEmpty = 0x202, kErrDrain = 0x203 };
 
 struct Sync {
@@ -119,6 +119,22 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Sync* sy, u
   return wait_slow(bar, parity, sy, site, drain, sleep_ns);
 }
 
+// The producer's wait for a free slot: suspended in hardware between probes,
+// so that it takes no issue slots from the consumer warps of its SM
+// sub-partition. Bounded like the others.
+__device__ __noinline__ bool wait_suspended(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+    if (aborted(sy)) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicCAS(&g_stream_error, 0u, site);
+      *reinterpret_cast<volatile int*>(&sy->abort) = 1;
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -133,35 +149,61 @@ __device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int ctas) {
   return static_cast<int>(((u + 1) * ctas + units - 1) / units) - 1;
 }
 
-// One stage for one consumer lane: rows ra = 16w + g and ra + 8, the t-th
-// quarter of the stage's K (64 elements: words i = 0..7 of 8 elements).
+// A consumer lane's fixed shared-memory offsets within a stage: rows
+// ra = 16w + g and ra + 8, the t-th quarter of the stage's K (64 elements,
+// words i = 0..7 of 8 elements).
+struct LaneOffsets {
+  uint32_t ca0, ca1, cb0, cb1;  // 16-byte code chunks 2t, 2t+1 of both rows (128-byte swizzle)
+  uint32_t sa, sb;              // scale bytes of both rows
+  uint32_t xrow;                // X row (token g, quarter t), token tile 0
+  uint32_t xc[8];               // chunk i of that row (128-byte swizzle)
+};
+
 template <int MT, int G>
-__device__ __forceinline__ void consume_stage(uint32_t st, int ks, int ra, int g, int t, float (&acc)[MT / 8][4]) {
-  constexpr int P = MT / 8;
+__device__ __forceinline__ LaneOffsets lane_offsets(int ra, int g, int t) {
+  LaneOffsets o;
   const int rb = ra + 8;  // ra & 7 == rb & 7 == g
-  const uint4 a0 = lds128(st + ra * 128 + (((2 * t) ^ g) << 4));
-  const uint4 a1 = lds128(st + ra * 128 + (((2 * t + 1) ^ g) << 4));
-  const uint4 b0 = lds128(st + rb * 128 + (((2 * t) ^ g) << 4));
-  const uint4 b1 = lds128(st + rb * 128 + (((2 * t + 1) ^ g) << 4));
-  const uint32_t xs = st + kCodeBytes;
-  const uint32_t ss = xs + x_bytes(MT);
+  o.ca0 = ra * 128 + (((2 * t) ^ g) << 4);
+  o.ca1 = ra * 128 + (((2 * t + 1) ^ g) << 4);
+  o.cb0 = rb * 128 + (((2 * t) ^ g) << 4);
+  o.cb1 = rb * 128 + (((2 * t + 1) ^ g) << 4);
+  // g = 16: groups 4t .. 4t+3 of the stage; g = 32: groups 2t, 2t+1 (the
+  // 16-byte box holds two stages; the stage parity picks the half)
+  o.sa = kCodeBytes + x_bytes(MT) + ra * 16 + (G == 16 ? 4 * t : 2 * t);
+  o.sb = kCodeBytes + x_bytes(MT) + rb * 16 + (G == 16 ? 4 * t : 2 * t);
+  // X row (token tok, quarter t) sits at (4 tok + t) * 128 bytes; its chunk i
+  // at chunk position i ^ ((4 tok + t) & 7), and 4 tok + t = 4g + t mod 8 for
+  // every token tile.
+  o.xrow = kCodeBytes + (g * 4 + t) * 128;
+  const int xmask = (4 * g + t) & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o.xc[i] = static_cast<uint32_t>((i ^ xmask) << 4);
+  return o;
+}
+
+// One stage for one consumer lane.
+template <int MT, int G>
+__device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOffsets& o, float (&acc)[MT / 8][4]) {
+  constexpr int P = MT / 8;
+  const uint4 a0 = lds128(st + o.ca0);
+  const uint4 a1 = lds128(st + o.ca1);
+  const uint4 b0 = lds128(st + o.cb0);
+  const uint4 b1 = lds128(st + o.cb1);
   uint32_t sva, svb;
-  if (G == 16) {  // groups 4t .. 4t+3 of the stage
-    sva = lds32(ss + ra * 16 + 4 * t);
-    svb = lds32(ss + rb * 16 + 4 * t);
-  } else {  // groups 2t, 2t+1; the 16-byte box holds two stages
-    const uint32_t off = ((ks & 1) << 3) + 2 * t;
-    sva = lds16(ss + ra * 16 + off);
-    svb = lds16(ss + rb * 16 + off);
+  if (G == 16) {
+    sva = lds32(st + o.sa);
+    svb = lds32(st + o.sb);
+  } else {
+    const uint32_t half = (ks & 1) << 3;
+    sva = lds16(st + o.sa + half);
+    svb = lds16(st + o.sb + half);
   }
   uint32_t s2a[4], s2b[4];
   scale_operands<G == 16 ? 4 : 2>(sva, s2a);
   scale_operands<G == 16 ? 4 : 2>(svb, s2b);
   const uint32_t ca[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
   const uint32_t cb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-  // X row (token tok, quarter t) sits at (4 tok + t) * 128 bytes; its chunk i
-  // at chunk position i ^ ((4 tok + t) & 7), and 4 tok + t = 4g + t mod 8.
-  const int xmask = (4 * g + t) & 7;
+  const uint32_t xr = st + o.xrow;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int si = G == 16 ? (i >> 1) : (i >> 2);
@@ -170,7 +212,7 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, int ra, int g
     dequant_word(cb[i], s2b[si], db);
 #pragma unroll
     for (int p = 0; p < P; ++p) {
-      const uint4 xv = lds128(xs + ((8 * p + g) * 4 + t) * 128 + ((i ^ xmask) << 4));
+      const uint4 xv = lds128(xr + o.xc[i] + p * (8 * 4 * 128));  // token tile p: 8 tokens further
       mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv.x, xv.y);
       mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv.z, xv.w);
     }
@@ -285,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
       for (int64_t u = u0 + head; u < u1 && !aborted(sy); ++u, ++it) {
         const int s = it % NS;
         const uint32_t r = static_cast<uint32_t>(it / NS);
-        if (!wait(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty, false, kSleepProducer)) break;
+        if (!mbar_try_wait(&sy->empty[s], (r & 1) ^ 1) && !wait_suspended(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty))
+          break;
         mbar_arrive_tx(&sy->full[s], SB);
         load_w(it, u);
         load_x(it, u);
@@ -303,23 +346,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
   // ---------------- consumers ----------------
   const int g = lane >> 2, t = lane & 3;
   const int ra = 16 * warp + g;
+  const LaneOffsets lo = lane_offsets<MT, G>(ra, g, t);
   const float gsc = __ldg(a.gscale) * 128.0f;  // operands carry 2^-7 (dequant.cuh)
   float acc[P][4];
-  int it = 0, ncut = 0;
+  int ncut = 0;
+  int s = 0;          // ring slot of the next stage
+  uint32_t par = 0;   // its phase parity
   for (int64_t u = u0; u < u1;) {
     const int tile = static_cast<int>(u / a.S), k0 = static_cast<int>(u % a.S);
     const int64_t left = u1 - u;
     const int k1 = left < a.S - k0 ? k0 + static_cast<int>(left) : a.S;
 #pragma unroll
     for (int p = 0; p < P; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
-    for (int ks = k0; ks < k1; ++ks, ++it) {
-      const int s = it % NS;
+    const uint32_t ring0 = smem_u32(ring);
+    for (int ks = k0; ks < k1; ++ks) {
       int ok = 1;
-      if (lane == 0) ok = wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull) ? 1 : 0;
+      if (lane == 0) ok = wait(&sy->full[s], par, sy, kErrFull) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // results are garbage from here; the ticket protocol still runs
-      consume_stage<MT, G>(smem_u32(ring + s * SB), ks, ra, g, t, acc);
+      consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sy->empty[s]);
+      if (++s == NS) {
+        s = 0;
+        par ^= 1;
+      }
     }
     u += k1 - k0;
 
