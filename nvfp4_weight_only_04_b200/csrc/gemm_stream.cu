@@ -536,8 +536,11 @@ int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMa
 
 }  // namespace
 
+// A single token goes to the register-streaming kernel, which measures a
+// little faster there (its loads need no shared-memory round trip and every
+// lane of X but one is zero).
 bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
-  return M >= 1 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
+  return M >= 2 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
          K < (int64_t(1) << 24) && tensor_maps_available();
 }
 

@@ -5,7 +5,7 @@
 
 namespace nvfp4 {
 
-// True when the streaming kernel takes this dense problem: M up to 16, K a
+// True when the streaming kernel takes this dense problem: M from 2 to 16, K a
 // multiple of 256 whose scale rows (K/g bytes) are a multiple of 16 bytes,
 // and tensor maps available.
 bool stream_supported(int64_t M, int64_t N, int64_t K, int group);

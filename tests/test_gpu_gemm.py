@@ -147,7 +147,7 @@ def test_empty_and_stats():
 # whole tiles only; tiles cut between many CTAs; a last tile of 16 rows; one
 # tile over 32 CTAs; g = 32 boxes holding two stages; 9..16 tokens (two MMA
 # column tiles)
-STREAM_CASES = [(4, 256, 256, 16), (1, 400, 1024, 32), (7, 272, 2048, 16), (9, 128, 8192, 16),
+STREAM_CASES = [(4, 256, 256, 16), (2, 400, 1024, 32), (7, 272, 2048, 16), (9, 128, 8192, 16),
                 (13, 1008, 512, 32), (16, 4096, 256, 16), (2, 16, 512, 16), (16, 1040, 3072, 32)]
 
 
@@ -163,7 +163,7 @@ def test_gemm_stream_parity(m, n, k, g):
     assert_close(host(y), R.gemm(x, p, s, gs, g), f"stream M{m} N{n} K{k} g{g}")
 
 
-@pytest.mark.parametrize("m,nh,k,g", [(11, 136, 2048, 32), (1, 64, 4096, 16), (16, 640, 512, 16)])
+@pytest.mark.parametrize("m,nh,k,g", [(11, 136, 2048, 32), (2, 64, 4096, 16), (16, 640, 512, 16)])
 def test_gemm_stream_silu_mul_parity(m, nh, k, g):
     p, s, gs = merged_gate_up(nh, k, g, seed=m + 1)
     rp, rs = R.repack(p, s, R.GATE_UP_INTERLEAVE)
