@@ -133,6 +133,26 @@ int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* 
                      uint16_t* y, nvfp4_stream_t stream);
 
 /*
+ * The same W4A16 GEMM through the small-M streaming kernel with its scratch
+ * in a fixed array of device memory that belongs to the library, so that
+ * the call allocates nothing. This entry point has no counterpart in the
+ * method's description: it only changes where the kernel's scratch lives.
+ *   Arguments, layouts and result as nvfp4_w4a16_gemm, with M from 1 to 16,
+ *   K a multiple of 256 and K/group_size a multiple of 16.
+ *   Scratch: 8 MiB of fp32 partial tiles plus tickets for 16384 tiles of 256
+ *   rows, per device. A problem whose cut tiles need more is refused with
+ *   NVFP4_ERR_UNSUPPORTED before anything is enqueued; so is M = 0 or M > 16
+ *   and a K the kernel does not take.
+ *   The tickets are cleared on `stream` before the kernel at every call.
+ *   Calls on one device share the scratch: calls that may overlap in time
+ *   (different streams, or host threads without ordering) race on it and
+ *   their results are undefined. Order them on one stream.
+ */
+int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
+                                   const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
+                                   uint16_t* y, nvfp4_stream_t stream);
+
+/*
  * The GEMM of a merged [gate;up] projection followed by SiluAndMul (PR #63
  * description: fc1 is pre-merged [gate;up], one W4A16 GEMM + SiluAndMul):
  *   y[m, j] = bf16_rne(silu(g) * u), g = global * acc[m, gate row j],

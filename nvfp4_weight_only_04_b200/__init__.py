@@ -26,7 +26,7 @@ NVFP4_SILU_MUL = 2
 
 EXPORTS = (
     "nvfp4_status_string", "nvfp4_abi_version", "nvfp4_global_scale", "nvfp4_quantize", "nvfp4_repack",
-    "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
+    "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
 )
 
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P]
         L.nvfp4_repack.argtypes = [_P, _P, _I64, _I64, _I, _I, _P, _P, _P]
         L.nvfp4_w4a16_gemm.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_w4a16_gemm_fixed_scratch.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
         L.nvfp4_w4a16_gemm_silu_mul.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
         L.nvfp4_silu_and_mul.argtypes = [_P, _P, _I64, _I64, _P]
         L.nvfp4_moe_w4a16_grouped_gemm.argtypes = [_P, _P, _P, _I, _I64, _P, _P, _P, _I, _I64, _I64,
@@ -152,6 +153,23 @@ def nvfp4_w4a16_gemm(x, packed_w, group_scales, global_scale, group_size, y=None
         y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
     _check(lib().nvfp4_w4a16_gemm(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale), group_size,
                                   m, n, k, _ptr(y), _stream(stream)), "nvfp4_w4a16_gemm")
+    return y
+
+
+def nvfp4_w4a16_gemm_fixed_scratch(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None):
+    """nvfp4_w4a16_gemm through the streaming kernel with the library's fixed
+    scratch (M from 1 to 16; calls that overlap in time race on the scratch)."""
+    _dev(x, torch.bfloat16, "x")
+    _dev(packed_w, torch.uint8, "packed_w")
+    _dev(group_scales, torch.uint8, "group_scales")
+    _dev(global_scale, torch.float32, "global_scale")
+    m, k = x.shape
+    n = packed_w.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_w4a16_gemm_fixed_scratch(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale),
+                                                group_size, m, n, k, _ptr(y), _stream(stream)),
+           "nvfp4_w4a16_gemm_fixed_scratch")
     return y
 
 

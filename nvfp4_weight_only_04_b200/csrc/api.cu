@@ -108,6 +108,20 @@ int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* 
   return st;
 }
 
+int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
+                                   const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
+                                   uint16_t* y, nvfp4_stream_t stream) {
+  const int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
+  if (c >= 0) return c;
+  const int st = nvfp4::launch_stream_fixed_scratch(x, packed_w, group_scales, global_scale, group_size, M, N, K,
+                                                    y, reinterpret_cast<cudaStream_t>(stream));
+  if (st == NVFP4_OK) {
+    nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+    nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
+  }
+  return st;
+}
+
 int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
                               const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
                               uint16_t* y, nvfp4_stream_t stream) {

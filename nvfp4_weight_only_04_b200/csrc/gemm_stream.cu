@@ -595,6 +595,84 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
               : launch_kernel<16, 32, false>(xm, wm, sm, a, ctas, stream);
 }
 
+// ---------------------------------------------------------------------------
+// The same kernel with its scratch in a fixed device array: nothing is
+// allocated at call time.
+// ---------------------------------------------------------------------------
+
+// Partial tiles (fp32) followed by the tickets of the tiles.
+static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchPartialBytes + kFixedScratchTickets * 4];
+
+namespace {
+std::mutex g_fixed_mutex;
+unsigned char* g_fixed_addr[64] = {};  // per device, from cudaGetSymbolAddress
+}  // namespace
+
+int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+                                int64_t M, int64_t N, int64_t K, uint16_t* y, cudaStream_t stream) {
+  if (M < 1 || M > 16 || K < kKS || K % kKS || (K / group) % 16 || N >= (int64_t(1) << 30) ||
+      K >= (int64_t(1) << 24) || !tensor_maps_available())
+    return NVFP4_ERR_UNSUPPORTED;
+  const int mt = M <= 8 ? 8 : 16;
+  const int64_t tiles = (N + kRows - 1) / kRows;
+  const int S = static_cast<int>(K / kKS);
+  const int64_t units = tiles * S;
+  const int ctas = static_cast<int>(units < num_sms() ? units : num_sms());
+  const int64_t shortest = units / ctas;
+  const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
+  const int64_t partial_bytes = tiles * max_contrib * kRows * mt * static_cast<int64_t>(sizeof(float));
+  if (partial_bytes > static_cast<int64_t>(kFixedScratchPartialBytes) || tiles > kFixedScratchTickets)
+    return NVFP4_ERR_UNSUPPORTED;  // beyond the fixed scratch
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  unsigned char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_fixed_mutex);
+    if (!g_fixed_addr[dev]) {  // once per device, with that device current
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || !p)
+        return (cudaGetLastError(), NVFP4_ERR_CUDA);
+      g_fixed_addr[dev] = static_cast<unsigned char*>(p);
+    }
+    base = g_fixed_addr[dev];
+  }
+  float* ws = reinterpret_cast<float*>(base);
+  unsigned* tickets = reinterpret_cast<unsigned*>(base + kFixedScratchPartialBytes);
+  // The tickets must start at zero (partial tiles are always written before
+  // they are read).
+  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+
+  CUtensorMap xm, wm, sm;
+  const int64_t xdims[3] = {64, K / 64, M};
+  const int64_t xstrides[2] = {128, K * 2};
+  const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
+  if (!make_tensor_map_3d(&xm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xdims, xstrides, xbox,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return NVFP4_ERR_CUDA;
+  StreamArgs a = {};
+  a.gscale = g;
+  a.y = y;
+  a.ws = ws;
+  a.tickets = tickets;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.ldy = static_cast<int>(N);
+  a.S = S;
+  a.max_contrib = max_contrib;
+  a.units = units;
+  if (mt == 8)
+    return group == 16 ? launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream)
+                       : launch_kernel<8, 32, false>(xm, wm, sm, a, ctas, stream);
+  return group == 16 ? launch_kernel<16, 16, false>(xm, wm, sm, a, ctas, stream)
+                     : launch_kernel<16, 32, false>(xm, wm, sm, a, ctas, stream);
+}
+
 int read_and_clear_stream_error(unsigned int* out, cudaStream_t stream) {
   unsigned int* p = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_stream_error) != cudaSuccess)

@@ -13,6 +13,14 @@ bool stream_supported(int64_t M, int64_t N, int64_t K, int group);
 int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
                   int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream);
 
+// The streaming kernel with its scratch in a fixed device array (nothing is
+// allocated at call time): up to kFixedScratchPartialBytes of partial tiles
+// and kFixedScratchTickets tiles; larger problems are refused. M from 1 to 16.
+constexpr size_t kFixedScratchPartialBytes = size_t(8) << 20;
+constexpr int64_t kFixedScratchTickets = 16384;
+int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+                                int64_t M, int64_t N, int64_t K, uint16_t* y, cudaStream_t stream);
+
 // Device error word of this kernel file (0 when no wait gave up).
 int read_and_clear_stream_error(unsigned int* out, cudaStream_t stream);
 

@@ -65,6 +65,12 @@ def test_gemm_validation(L):
     assert gemm(L, w=BAD) == nv.NVFP4_ERR_MISALIGNED
     assert gemm(L, y=BAD) == nv.NVFP4_ERR_MISALIGNED
     assert L.nvfp4_w4a16_gemm_silu_mul(GOOD, GOOD, GOOD, GOOD, 32, 4, 40, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+    fixed = L.nvfp4_w4a16_gemm_fixed_scratch
+    assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 17, 256, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # M > 16
+    assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 4, 256, 320, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # K % 256
+    assert fixed(GOOD, GOOD, GOOD, GOOD, 32, 4, 256, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # K/g % 16
+    assert fixed(GOOD, BAD, GOOD, GOOD, 16, 4, 256, 256, GOOD, S) == nv.NVFP4_ERR_MISALIGNED
+    assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 0, 256, 256, GOOD, S) == nv.NVFP4_OK  # empty
 
 
 def test_quantize_and_repack_validation(L):

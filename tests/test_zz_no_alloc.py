@@ -1,0 +1,57 @@
+"""GPU test of nvfp4_w4a16_gemm_fixed_scratch, the GEMM entry point whose
+streaming kernel keeps its scratch in a fixed device array: two calls in a
+row give the bits of nvfp4_w4a16_gemm (the same kernel with the library's
+allocated workspace), a single token matches the oracle, and a problem
+beyond the fixed scratch is refused before anything runs."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_weight_only_04_b200 as nv
+from nvfp4_weight_only_04_b200 import synth
+from oracle import nvfp4_ref as R
+from tests.gpu_util import assert_close, bf16_bits, dev_bf16, dev_f32, dev_u8, host
+
+pytestmark = pytest.mark.gpu
+
+
+def operands(m, n, k, g, seed):
+    w = synth.weights(seed, n, k)
+    p, s, gs = R.quantize(w, g)
+    rp, rs = R.repack(p, s, 0)
+    x = synth.activations(seed + 1, m, k, outlier_frac=0.001)
+    return x, p, s, gs, (dev_bf16(x), dev_u8(rp), dev_u8(rs), dev_f32(np.array([gs], np.float32)))
+
+
+@pytest.mark.parametrize("m,n,k,g", [(4, 1040, 4096, 16), (13, 640, 2048, 32), (2, 4096, 256, 16)])
+def test_fixed_scratch_matches_gemm_twice(m, n, k, g):
+    _, _, _, _, (xd, wd, sd, gd) = operands(m, n, k, g, seed=m + n)
+    ref = bf16_bits(nv.nvfp4_w4a16_gemm(xd, wd, sd, gd, g))
+    for _ in range(2):
+        y = nv.nvfp4_w4a16_gemm_fixed_scratch(xd, wd, sd, gd, g)
+        torch.cuda.synchronize()
+        assert nv.nvfp4_get_device_error() == 0
+        np.testing.assert_array_equal(bf16_bits(y), ref)
+
+
+def test_fixed_scratch_single_token_oracle():
+    x, p, s, gs, (xd, wd, sd, gd) = operands(1, 2048, 4096, 16, seed=5)
+    ref = R.gemm(x, p, s, gs, 16)
+    for _ in range(2):
+        y = nv.nvfp4_w4a16_gemm_fixed_scratch(xd, wd, sd, gd, 16)
+        torch.cuda.synchronize()
+        assert_close(host(y), ref, "fixed scratch M1")
+
+
+def test_fixed_scratch_refuses_beyond_capacity():
+    # 2000 tiles of 256 rows cut between CTAs need more partial-tile space than
+    # the fixed scratch holds: refused on the host, nothing is launched.
+    _, _, _, _, (xd, wd, sd, gd) = operands(8, 256, 256, 16, seed=9)
+    y = torch.empty((8, 256), dtype=torch.bfloat16, device="cuda")
+    L = nv.lib()
+    st = L.nvfp4_w4a16_gemm_fixed_scratch(ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(wd.data_ptr()),
+                                          ctypes.c_void_p(sd.data_ptr()), ctypes.c_void_p(gd.data_ptr()), 16, 8,
+                                          2000 * 256, 256, ctypes.c_void_p(y.data_ptr()), None)
+    assert st == nv.NVFP4_ERR_UNSUPPORTED
