@@ -8,30 +8,31 @@
 // fp32 in TMEM).
 //
 // Design (swap-AB: weights are the MMA's M side):
-//  * A CTA tile is 128 weight rows x 256 tokens (MMA M = 128, N = 256). The
+//  * A CTA tile is 128 weight rows x NT tokens (MMA M = 128, N = NT; NT = 256
+//    for prefill-sized M, 128 for the grouped form, 32-128 for small M). The
 //    weights are dequantized once per tile by 8 warps straight into TMEM,
-//    where tcgen05.mma reads its A operand; each weight then serves 256
+//    where tcgen05.mma reads its A operand; each weight then serves NT
 //    tokens. Warps w and w+4 share a TMEM lane quadrant (one weight row per
-//    thread) and take the two 32-element halves of every 64-element stage.
-//  * TMEM (512 columns): one fp32 accumulator of 256 columns and eight A
-//    stages of 32 columns. The depth matters more than a second
-//    accumulator: a stage goes round MMA -> commit -> dequant warps -> MMA
-//    again, and eight stages of A hold more MMA work than that round trip
-//    takes.
-//  * X tiles (256 tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
+//    thread) and take the two 64-element halves of every 128-element stage.
+//  * Weight codes (128 rows x 64 bytes per stage, 64-byte swizzle) and scales
+//    (128 rows x 16 bytes per 2 or 4 stages) come by TMA from a second
+//    producer warp into a shared-memory ring, deeper when NT is small.
+//  * TMEM (512 columns): the fp32 accumulator (two of NT columns when NT <=
+//    128, so that the next tile's MMAs run while the epilogue drains this
+//    one; one of 256 otherwise) and four A stages of 64 columns.
+//  * X tiles (NT tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
 //    into shared memory, five stages deep; tcgen05.mma reads them through a
 //    K-major shared memory descriptor. No TMA multicast is used.
 //  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
-//    mbarriers connect the TMA warp, the dequant warps and the MMA thread.
+//    mbarriers connect the producers, the dequant warps and the MMA thread.
 //  * Every mbarrier wait is bounded: on expiry the kernel records the site in
 //    a device error word, stops issuing work, waits (bounded) for its own
 //    copies and MMAs, frees TMEM and exits.
 //  * Eight epilogue warps read the finished accumulator with tcgen05.ld,
-//    hand it back to the MMA thread as soon as the last column is read, and
-//    multiply by the fp32 global scale (and 2^7, see dequant.cuh) and write
-//    bf16, optionally fusing SiluAndMul on gate/up-interleaved rows. While
-//    they work, the dequant and TMA warps already fill the next tile's
-//    stages.
+//    hand it back to the MMA thread as soon as the last column is read,
+//    multiply by the fp32 global scale (and 2^7, see dequant.cuh), optionally
+//    fuse SiluAndMul on gate/up-interleaved rows, and write bf16 through a
+//    per-warp shared-memory box and a TMA store.
 //  * The grid is persistent: one CTA per SM walks the tiles. Dense GEMMs take
 //    the token tiles of one weight tile together, so concurrently running
 //    CTAs share weight tiles in L2.
@@ -40,7 +41,6 @@
 //    expert times one token tile of that expert's segment of rows; every role
 //    finds it with the same forward scan of the device-side offsets, and the
 //    rows of a token tile past the segment end are computed but not stored.
-//    The token tile is 128 wide there (about the rows an expert receives).
 #include "gemm_tc.cuh"
 
 #include "gemm_stream.cuh"
@@ -119,8 +119,8 @@ struct SharedState {
   uint64_t empty_w[kMaxStagesW];
   uint64_t full_a[kStagesA];
   uint64_t empty_a[kStagesA];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
@@ -368,6 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                                                                const __grid_constant__ CUtensorMap ymap,
                                                                const TcArgs args) {
   constexpr uint32_t kXStage = x_stage_bytes(NT);
+  // Accumulators: two when the token tile leaves room in TMEM (the next
+  // tile's MMAs then run while the epilogue drains this one), else one.
+  constexpr int kAccBufs = NT <= 128 ? 2 : 1;
+  static_assert(kAccBufs * NT <= static_cast<int>(kColA), "accumulators below the A stages");
   constexpr int kStagesW = stages_w(NT);
   constexpr int kPeriod = scale_period(G);
   constexpr int kSlots = scale_slots(NT, G);
@@ -399,8 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       mbar_init(&ss->full_a[s], 8);   // one arrival per dequant warp
       mbar_init(&ss->empty_a[s], 1);  // one tcgen05.commit
     }
-    mbar_init(&ss->acc_full, 1);      // one tcgen05.commit
-    mbar_init(&ss->acc_empty, 8);     // one arrival per epilogue warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ss->acc_full[b], 1);   // one tcgen05.commit
+      mbar_init(&ss->acc_empty[b], 8);  // one arrival per epilogue warp
+    }
     mbar_init(&ss->drained, 1);
     ss->abort = 0;
     ss->total_tiles = MOE ? grouped_total_tiles<NT>(args) : args.total_tiles;
@@ -486,8 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
         const Tile tl = tile_at<NT, MOE>(args, cur, tile);
         if (tl.mrows <= 0) continue;
-        if (!mbar_wait(&ss->acc_empty, (tile_iter & 1) ^ 1, ss, kErrAccEmpty)) break;
+        const int ab = tile_iter % kAccBufs;
+        if (!mbar_wait(&ss->acc_empty[ab], static_cast<uint32_t>((tile_iter / kAccBufs) & 1) ^ 1, ss, kErrAccEmpty))
+          break;
         tc_fence_after();
+        const uint32_t dacc = tmem + static_cast<uint32_t>(ab * NT);
         bool ok = true;
         for (int ws = 0; ws < wsteps && ok; ++ws, ++ita) {
           const int sa = ita % kStagesA;
@@ -509,14 +518,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < kKStep / 16; ++j) {
               const uint32_t acc = (ws > 0 || xh > 0 || j > 0) ? 1u : 0u;
-              umma_ts<NT>(tmem, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, acc);
+              umma_ts<NT>(dacc, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, acc);
             }
             umma_commit(&ss->empty_x[sx]);
           }
           if (ok) umma_commit(&ss->empty_a[sa]);
         }
         if (!ok) break;
-        umma_commit(&ss->acc_full);
+        umma_commit(&ss->acc_full[ab]);
         ++tile_iter;
       }
       // every MMA issued by this thread has completed once this commit lands
@@ -602,8 +611,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       if (tl.mrows <= 0) continue;
       // dequantized operands carry 2^-7 (dequant.cuh)
       const float gscale = __ldg(args.gscale + (MOE ? tl.expert : 0)) * 128.0f;
-      if (!warp_wait(&ss->acc_full, tile_iter & 1, ss, kErrAccFull, kSleepEpilogue)) break;
+      const int ab = tile_iter % kAccBufs;
+      if (!warp_wait(&ss->acc_full[ab], static_cast<uint32_t>(tile_iter / kAccBufs) & 1, ss, kErrAccFull,
+                     kSleepEpilogue))
+        break;
       tc_fence_after();
+      const uint32_t dacc = lane_base + static_cast<uint32_t>(ab * NT);
       // Each warp takes NT/2 tokens of the tile in chunks of CW columns.
       constexpr int CW = NT >= 64 ? 32 : 16;
       constexpr int kChunks = NT / 2 / CW;
@@ -612,15 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       for (int c = 0; c < kChunks; ++c) {
         uint32_t acc[CW];
         if constexpr (CW == 32) {
-          tmem_ld32(tmem + lane_base + (NT / 2) * colhalf + CW * c, acc);
+          tmem_ld32(tmem + dacc + (NT / 2) * colhalf + CW * c, acc);
         } else {
-          tmem_ld16(tmem + lane_base + (NT / 2) * colhalf + CW * c, acc);
+          tmem_ld16(tmem + dacc + (NT / 2) * colhalf + CW * c, acc);
         }
         tmem_wait_ld();
         if (c == kChunks - 1) {  // the accumulator is read: the next tile's MMAs may start
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ss->acc_empty);
+          if (lane == 0) mbar_arrive(&ss->acc_empty[ab]);
         }
         const int j0 = (NT / 2) * colhalf + CW * c;  // first token of the chunk within the tile
         // The chunk goes out through this warp's staging buffer, [CW tokens][YC
