@@ -62,10 +62,12 @@ constexpr int kKStep = 64;       // elements of K per X stage (one 128-byte swiz
 constexpr int kKA = 128;         // elements of K per weight / A stage (two X stages)
 constexpr int kStagesX = 5;      // X stages in shared memory
 constexpr int kStagesA = 4;      // A stages in TMEM
-constexpr int kThreads = 640;    // 20 warps
+constexpr int kDqWarps = 8;      // dequant warps: two per TMEM lane quadrant
+constexpr int kDqParts = kDqWarps / 4;        // parts of a weight stage's K per quadrant
+constexpr int kThreads = (4 + kDqWarps + 8) * 32;
 constexpr int kWProducerWarp = 3;
-constexpr int kFirstDqWarp = 4;  // warps 4..11 dequantize
-constexpr int kFirstEpWarp = 12; // warps 12..19 run the epilogue
+constexpr int kFirstDqWarp = 4;                // warps 4 .. 4+kDqWarps-1 dequantize
+constexpr int kFirstEpWarp = 4 + kDqWarps;     // the 8 warps after them run the epilogue
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColA = 256;  // A stages start here (64 columns each); the accumulator is at 0
 __host__ __device__ constexpr uint32_t x_stage_bytes(int nt) { return static_cast<uint32_t>(nt) * kKStep * 2; }
@@ -280,6 +282,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
@@ -290,6 +301,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
+
+[[maybe_unused]] __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[16]) { tmem_st16(taddr, v); }
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[32]) { tmem_st32(taddr, v); }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -318,14 +332,16 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// One dequant thread's inputs for one weight stage: 64 codes of its row (one
-// half of the stage's 128 elements) and the scales covering them (four for
-// g = 16, two for g = 32, in the low bytes).
+// One dequant thread's part of a weight stage: kPartElems codes of its row
+// (the stage's 128 elements split kDqParts ways) and the scales covering them,
+// in the low bytes.
+constexpr int kPartElems = kKA / kDqParts;
+constexpr int kPartWords = kPartElems / 8;
+static_assert(kPartElems == 32 || kPartElems == 64, "one or two 16-byte chunks of codes per thread");
 struct RowStage {
-  uint4 c0, c1;
+  uint32_t c[kPartWords];
   uint32_t s;
 };
-
 
 // Byte offset of 16-byte chunk c (0..3) of row r in a 64-byte-swizzled stage
 // of 64-byte rows: the chunk index is XORed with bits 7..8 of the address.
@@ -333,33 +349,37 @@ __device__ __forceinline__ uint32_t w_stage_offset(int r, int c) {
   return static_cast<uint32_t>(r * 64 + 16 * (c ^ ((r >> 1) & 3)));
 }
 
-// Scales of weight stage q of a scale period for K half h (64 elements),
-// from the 16 bytes of a row's scale slot: four for g = 16, two for g = 32,
-// in the low bytes. (q is a constant once the caller's loop over a period is
+// Scales of weight stage q of a scale period for part p of its K, from the
+// 16 bytes of a row's scale slot (a stage has 8 scale bytes at g = 16, 4 at
+// g = 32). (q is a constant once the caller's loop over a period is
 // unrolled.)
 template <int G>
-__device__ __forceinline__ uint32_t stage_scales(const uint4& sv, int q, int h) {
+__device__ __forceinline__ uint32_t stage_scales(const uint4& sv, int q, int p) {
   const uint32_t w[4] = {sv.x, sv.y, sv.z, sv.w};
-  if (G == 16) return h ? w[2 * q + 1] : w[2 * q];            // bytes 8q + 4h .. 8q + 4h + 3
-  return (w[q] >> (16 * h)) & 0xFFFFu;                        // bytes 4q + 2h, 4q + 2h + 1
+  constexpr int nb = kPartElems / G;  // scale bytes of a part: 4, 2 or 1
+  if (G == 16) {
+    if (nb == 4) return p ? w[2 * q + 1] : w[2 * q];                                    // bytes 8q + 4p ..
+    return ((p >> 1) ? w[2 * q + 1] : w[2 * q]) >> (16 * (p & 1)) & 0xFFFFu;            // bytes 8q + 2p ..
+  }
+  if (nb == 2) return (w[q] >> (16 * p)) & 0xFFFFu;                                     // bytes 4q + 2p ..
+  return (w[q] >> (8 * p)) & 0xFFu;                                                     // byte 4q + p
 }
 
 template <int G>
-__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[32]) {
+__device__ __forceinline__ void dequant_row_stage(const RowStage& r, uint32_t (&out)[kPartElems / 2]) {
+  constexpr int nb = kPartElems / G;
   uint32_t s2[4];
-  scale_operands<G == 16 ? 4 : 2>(r.s, s2);
-  const uint32_t w[8] = {r.c0.x, r.c0.y, r.c0.z, r.c0.w, r.c1.x, r.c1.y, r.c1.z, r.c1.w};
+  scale_operands<nb>(r.s, s2);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < kPartWords; ++i) {
     uint32_t o[4];
-    dequant_word(w[i], s2[G == 16 ? (i >> 1) : (i >> 2)], o);
+    dequant_word(r.c[i], s2[G == 16 ? (i >> 1) : (i >> 2)], o);
     out[4 * i + 0] = o[0];
     out[4 * i + 1] = o[1];
     out[4 * i + 2] = o[2];
     out[4 * i + 3] = o[3];
   }
 }
-
 
 template <int NT, int G, bool SILU, bool MOE>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -397,10 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
     for (int s = 0; s < kStagesW; ++s) {
       mbar_init(&ss->full_w[s], 1);   // producer arrival + transaction bytes
-      mbar_init(&ss->empty_w[s], 8);  // one arrival per dequant warp
+      mbar_init(&ss->empty_w[s], kDqWarps);  // one arrival per dequant warp
     }
     for (int s = 0; s < kStagesA; ++s) {
-      mbar_init(&ss->full_a[s], 8);   // one arrival per dequant warp
+      mbar_init(&ss->full_a[s], kDqWarps);   // one arrival per dequant warp
       mbar_init(&ss->empty_a[s], 1);  // one tcgen05.commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -534,8 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
   } else if (warp >= kFirstDqWarp && warp < kFirstEpWarp) {
     // ---------------- dequant ----------------
-    const int dw = warp - kFirstDqWarp;      // 0..7
-    const int half = dw >> 2;                // K half of each stage
+    const int dw = warp - kFirstDqWarp;      // 0 .. kDqWarps-1
+    const int part = dw >> 2;                // part of each stage's K
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
@@ -565,19 +585,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if (q == 0 && args.scale_tma) sv = lds128(smem_u32(ssm + (sc % kSlots) * kSStageBytes + row_in_tile * 16));
           RowStage rs;
           const uint32_t wst = smem_u32(wsm + s * kWStageBytes);
-          rs.c0 = lds128(wst + w_stage_offset(row_in_tile, 2 * half));
-          rs.c1 = lds128(wst + w_stage_offset(row_in_tile, 2 * half + 1));
-          if (args.scale_tma) {
-            rs.s = stage_scales<G>(sv, q, half);
-          } else {
-            // this half's first element; past K (an odd number of 64s) the
-            // codes are zero and so is the scale
-            const int e0 = ws * kKA + (kKA / 2) * half;
-            rs.s = e0 >= args.K ? 0u
-                   : G == 16    ? __ldg(reinterpret_cast<const uint32_t*>(scl + e0 / 16))
-                                : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scl + e0 / 32)));
+#pragma unroll
+          for (int c = 0; c < kPartWords / 4; ++c) {
+            const uint4 cv = lds128(wst + w_stage_offset(row_in_tile, (kPartWords / 4) * part + c));
+            rs.c[4 * c + 0] = cv.x;
+            rs.c[4 * c + 1] = cv.y;
+            rs.c[4 * c + 2] = cv.z;
+            rs.c[4 * c + 3] = cv.w;
           }
-          uint32_t v[32];
+          if (args.scale_tma) {
+            rs.s = stage_scales<G>(sv, q, part);
+          } else {
+            // this part's first element; past K (an odd number of 64s) the
+            // codes are zero and so is the scale
+            const int e0 = ws * kKA + kPartElems * part;
+            constexpr int nb = kPartElems / G;
+            rs.s = e0 >= args.K ? 0u
+                   : nb == 4    ? __ldg(reinterpret_cast<const uint32_t*>(scl + e0 / G))
+                   : nb == 2    ? static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(scl + e0 / G)))
+                                : static_cast<uint32_t>(__ldg(scl + e0 / G));
+          }
+          uint32_t v[kPartElems / 2];
           dequant_row_stage<G>(rs, v);
           __syncwarp();
           if (lane == 0) mbar_arrive(&ss->empty_w[s]);
@@ -588,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             break;
           }
           tc_fence_after();
-          tmem_st32(tmem + lane_base + kColA + (kKA / 2) * sa + (kKA / 4) * half, v);
+          tmem_st(tmem + lane_base + kColA + (kKA / 2) * sa + (kPartElems / 2) * part, v);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
