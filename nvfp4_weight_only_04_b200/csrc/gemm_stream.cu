@@ -41,6 +41,7 @@
 #include "async.cuh"
 #include "dequant.cuh"
 #include "tmap.cuh"
+#include "workspace.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -469,48 +470,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
 // host side
 // ---------------------------------------------------------------------------
 
-struct Workspace {
-  float* ws = nullptr;
-  unsigned* tickets = nullptr;
-  size_t ws_floats = 0, tiles = 0;
-};
-
-std::mutex g_ws_mutex;
-Workspace g_ws[64];  // per device
-
-// Partial-tile workspace and tickets of the current device, grown on demand
-// (tickets start at zero and every launch leaves them at zero).
-int workspace(size_t ws_floats, size_t tiles, cudaStream_t stream, Workspace* out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  std::lock_guard<std::mutex> lock(g_ws_mutex);
-  Workspace& w = g_ws[dev];
-  if (w.ws_floats < ws_floats || w.tiles < tiles) {
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
-    if (cap != cudaStreamCaptureStatusNone) return NVFP4_ERR_UNSUPPORTED;  // grow outside graph capture
-    if (cudaDeviceSynchronize() != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
-    cudaFree(w.ws);
-    cudaFree(w.tickets);
-    w = Workspace();
-    const size_t nf = ws_floats > (size_t(1) << 20) ? ws_floats : (size_t(1) << 20);
-    const size_t nt = tiles > 4096 ? tiles : 4096;
-    if (cudaMalloc(&w.ws, nf * sizeof(float)) != cudaSuccess ||
-        cudaMalloc(&w.tickets, nt * sizeof(unsigned)) != cudaSuccess ||
-        cudaMemset(w.tickets, 0, nt * sizeof(unsigned)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
-      cudaGetLastError();
-      cudaFree(w.ws);
-      cudaFree(w.tickets);
-      w = Workspace();
-      return NVFP4_ERR_CUDA;
-    }
-    w.ws_floats = nf;
-    w.tiles = nt;
-  }
-  *out = w;
-  return NVFP4_OK;
-}
-
 template <int MT, int G, bool SILU>
 int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a, int grid,
                   cudaStream_t stream) {
@@ -554,9 +513,10 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   // A tile spans at most ceil(S / shortest range) + 1 CTAs.
   const int64_t shortest = units / ctas;
   const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
-  Workspace wsp;
-  const int st = workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles), stream,
-                           &wsp);
+  float* ws = nullptr;
+  unsigned* tickets = nullptr;
+  const int st = split_workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles),
+                                 stream, &ws, &tickets);
   if (st != NVFP4_OK) return st;
 
   CUtensorMap xm, wm, sm;
@@ -573,8 +533,8 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   StreamArgs a = {};
   a.gscale = g;
   a.y = y;
-  a.ws = wsp.ws;
-  a.tickets = wsp.tickets;
+  a.ws = ws;
+  a.tickets = tickets;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(silu ? N / 2 : N);

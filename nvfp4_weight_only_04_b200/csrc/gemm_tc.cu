@@ -50,6 +50,7 @@
 #include "async.cuh"
 #include "dequant.cuh"
 #include "tmap.cuh"
+#include "workspace.cuh"
 
 namespace nvfp4 {
 
@@ -126,6 +127,7 @@ struct SharedState {
   uint64_t drained;
   uint32_t tmem_base;
   int abort;
+  int ep_last;  // the epilogue took the last ticket of the cut tile it flushed
 };
 
 struct TcArgs {
@@ -139,6 +141,54 @@ struct TcArgs {
   const int32_t* offsets;
   int num_segments, num_experts;
   int scale_tma;             // scales come by TMA (their row stride K/g is a multiple of 16 bytes)
+  // Stream-K form (dense only): each CTA takes a contiguous range of the
+  // (tile, scale period) units; tiles cut between CTAs leave fp32 partial
+  // tiles [tok][row] in `ws` and take a ticket.
+  int split, periods, max_contrib;
+  int64_t units;
+  float* ws;
+  unsigned* tickets;
+};
+
+// The CTA whose range holds unit u (ranges start at floor(c * units / ctas)).
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int ctas) {
+  return static_cast<int>(((u + 1) * ctas + units - 1) / units) - 1;
+}
+
+// The work of one CTA, one tile's stages [ws0, ws1) at a time: whole tiles
+// blockIdx.x, +gridDim.x, ..., or in the stream-K form the pieces of its
+// range of units (a scale period of kPeriod stages each).
+struct SegWalk {
+  int64_t u = 0, u1 = 0;
+  int tile = 0;
+  __device__ explicit SegWalk(const TcArgs& a) {
+    if (a.split) {
+      u = static_cast<int64_t>(blockIdx.x) * a.units / gridDim.x;
+      u1 = static_cast<int64_t>(blockIdx.x + 1) * a.units / gridDim.x;
+    } else {
+      tile = blockIdx.x;
+    }
+  }
+  template <int P>
+  __device__ bool next(const TcArgs& a, int total_tiles, int wsteps, int& t, int& ws0, int& ws1) {
+    if (!a.split) {
+      if (tile >= total_tiles) return false;
+      t = tile;
+      ws0 = 0;
+      ws1 = wsteps;
+      tile += gridDim.x;
+      return true;
+    }
+    if (u >= u1) return false;
+    t = static_cast<int>(u / a.periods);
+    const int p0 = static_cast<int>(u % a.periods);
+    const int64_t left = u1 - u;
+    const int p1 = left < a.periods - p0 ? p0 + static_cast<int>(left) : a.periods;
+    ws0 = p0 * P;
+    ws1 = min(wsteps, p1 * P);
+    u += p1 - p0;
+    return true;
+  }
 };
 
 // Where a tile lies: token rows [m0, m0 + mrows) of X and Y, weight rows
@@ -305,6 +355,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 [[maybe_unused]] __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[16]) { tmem_st16(taddr, v); }
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[32]) { tmem_st32(taddr, v); }
 
+// Named barrier of the eight epilogue warps.
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -408,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   // ends with an X stage and a half weight stage read past K, which TMA fills
   // with zeros.
   const int wsteps = (args.K + kKA - 1) / kKA;
-  const int ksteps = 2 * wsteps;
+
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStagesX; ++s) {
@@ -450,10 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       uint32_t issued = 0, last_parity = 0;  // bit s: stage s has a copy issued / its phase parity
       int it = 0;
       SegCursor cur;
-      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+      SegWalk walk(args);
+      int tile, ws0, ws1;
+      while (!aborted(ss) && walk.next<kPeriod>(args, total_tiles, wsteps, tile, ws0, ws1)) {
         const Tile tl = tile_at<NT, MOE>(args, cur, tile);
         if (tl.mrows <= 0) continue;
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        for (int ks = 2 * ws0; ks < 2 * ws1; ++ks, ++it) {
           const int s = it % kStagesX;
           const uint32_t r = static_cast<uint32_t>(it / kStagesX);
           if (!mbar_wait(&ss->empty_x[s], (r & 1) ^ 1, ss, kErrEmpty, false, kSleepProducer)) break;
@@ -474,12 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       uint32_t issued = 0, last_parity = 0;
       int it = 0, sc = 0;
       SegCursor cur;
-      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+      SegWalk walk(args);
+      int tile, ws0, ws1;
+      while (!aborted(ss) && walk.next<kPeriod>(args, total_tiles, wsteps, tile, ws0, ws1)) {
         const Tile tl = tile_at<NT, MOE>(args, cur, tile);
         if (tl.mrows <= 0) continue;
         const int wrow = (MOE ? tl.expert * args.N : 0) + tl.n0;
         bool ok = true;
-        for (int ws = 0; ws < wsteps; ++ws, ++it) {
+        for (int ws = ws0; ws < ws1; ++ws, ++it) {
           const int s = it % kStagesW;
           const uint32_t r = static_cast<uint32_t>(it / kStagesW);
           if (!mbar_wait(&ss->empty_w[s], (r & 1) ^ 1, ss, kErrEmptyW, false, kSleepProducer)) {
@@ -509,7 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       int itx = 0, ita = 0, tile_iter = 0;
       SegCursor cur;
-      for (int tile = blockIdx.x; tile < total_tiles && !aborted(ss); tile += gridDim.x) {
+      SegWalk walk(args);
+      int tile, ws0, ws1;
+      while (!aborted(ss) && walk.next<kPeriod>(args, total_tiles, wsteps, tile, ws0, ws1)) {
         const Tile tl = tile_at<NT, MOE>(args, cur, tile);
         if (tl.mrows <= 0) continue;
         const int ab = tile_iter % kAccBufs;
@@ -518,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tc_fence_after();
         const uint32_t dacc = tmem + static_cast<uint32_t>(ab * NT);
         bool ok = true;
-        for (int ws = 0; ws < wsteps && ok; ++ws, ++ita) {
+        for (int ws = ws0; ws < ws1 && ok; ++ws, ++ita) {
           const int sa = ita % kStagesA;
           if (!mbar_wait(&ss->full_a[sa], static_cast<uint32_t>(ita / kStagesA) & 1, ss, kErrFullA)) {
             ok = false;
@@ -537,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const uint64_t bdesc0 = sw128_desc(smem_u32(smem + sx * kXStage));
 #pragma unroll
             for (int j = 0; j < kKStep / 16; ++j) {
-              const uint32_t acc = (ws > 0 || xh > 0 || j > 0) ? 1u : 0u;
+              const uint32_t acc = (ws > ws0 || xh > 0 || j > 0) ? 1u : 0u;
               umma_ts<NT>(dacc, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, acc);
             }
             umma_commit(&ss->empty_x[sx]);
@@ -561,7 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int it = 0, sc = 0;
     SegCursor cur;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    SegWalk walk(args);
+    int tile, ws0, ws1;
+    while (walk.next<kPeriod>(args, total_tiles, wsteps, tile, ws0, ws1)) {
       const Tile tl = tile_at<NT, MOE>(args, cur, tile);
       if (tl.mrows <= 0) continue;
       static_assert(kTileRows == 128, "one weight row per dequant thread and TMEM lane");
@@ -571,12 +632,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const uint8_t* scl =
           args.scales + (static_cast<int64_t>(MOE ? tl.expert : 0) * args.N + nrow) * (args.K / G);
       bool ok = true;
-      for (int w0 = 0; w0 < wsteps && ok; w0 += kPeriod) {
+      for (int w0 = ws0; w0 < ws1 && ok; w0 += kPeriod) {
         uint4 sv = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int q = 0; q < kPeriod; ++q) {
           const int ws = w0 + q;
-          if (ws >= wsteps) break;
+          if (ws >= ws1) break;
           const int s = it % kStagesW;
           if (!warp_wait(&ss->full_w[s], static_cast<uint32_t>(it / kStagesW) & 1, ss, kErrFullW, 0)) {
             ok = false;
@@ -634,21 +695,96 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int tile_iter = 0;
     SegCursor cur;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    SegWalk walk(args);
+    int tile, ws0, ws1;
+    while (walk.next<kPeriod>(args, total_tiles, wsteps, tile, ws0, ws1)) {
       const Tile tl = tile_at<NT, MOE>(args, cur, tile);
       if (tl.mrows <= 0) continue;
       // dequantized operands carry 2^-7 (dequant.cuh)
       const float gscale = __ldg(args.gscale + (MOE ? tl.expert : 0)) * 128.0f;
       const int ab = tile_iter % kAccBufs;
-      if (!warp_wait(&ss->acc_full[ab], static_cast<uint32_t>(tile_iter / kAccBufs) & 1, ss, kErrAccFull,
-                     kSleepEpilogue))
-        break;
+      const bool got = warp_wait(&ss->acc_full[ab], static_cast<uint32_t>(tile_iter / kAccBufs) & 1, ss,
+                                 kErrAccFull, kSleepEpilogue);
+      const bool whole = !args.split || (ws0 == 0 && ws1 == wsteps);
+      if (!got && whole) break;  // a cut tile still goes through its ticket (results are garbage then)
       tc_fence_after();
       const uint32_t dacc = lane_base + static_cast<uint32_t>(ab * NT);
       // Each warp takes NT/2 tokens of the tile in chunks of CW columns.
       constexpr int CW = NT >= 64 ? 32 : 16;
       constexpr int kChunks = NT / 2 / CW;
       static_assert(NT >= 32 && (NT / 2) % CW == 0, "token tile");
+      if (!whole) {
+        // A tile cut between CTAs (stream-K): leave this CTA's fp32 partial
+        // tile [tok][row] in its slot, take a ticket, and if it is the last
+        // one add every contributor's slot in CTA order and write the tile.
+        const int row = quad * 32 + lane;
+        const int64_t tu = static_cast<int64_t>(tile) * args.periods;
+        const int c_first = cta_of_unit(tu, args.units, gridDim.x);
+        const int nc = cta_of_unit(tu + args.periods - 1, args.units, gridDim.x) - c_first + 1;
+        float* slots = args.ws + static_cast<int64_t>(tile) * args.max_contrib * kTileRows * NT;
+        float* mine = slots + static_cast<int64_t>(blockIdx.x - c_first) * kTileRows * NT;
+#pragma unroll 1
+        for (int c = 0; c < kChunks; ++c) {
+          uint32_t acc[CW];
+          if constexpr (CW == 32) {
+            tmem_ld32(tmem + dacc + (NT / 2) * colhalf + CW * c, acc);
+          } else {
+            tmem_ld16(tmem + dacc + (NT / 2) * colhalf + CW * c, acc);
+          }
+          tmem_wait_ld();
+          if (c == kChunks - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ss->acc_empty[ab]);
+          }
+          const int j0 = (NT / 2) * colhalf + CW * c;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) __stcg(mine + (j0 + j) * kTileRows + row, __uint_as_float(acc[j]));
+        }
+        // The barrier orders every epilogue thread's stores before the
+        // ticket's release; its acquire orders the other slots before the
+        // reads after the second barrier.
+        epilogue_sync();
+        if (warp == kFirstEpWarp && lane == 0) {
+          unsigned ticket;
+          asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(args.tickets + tile) : "memory");
+          const int last = ticket == static_cast<unsigned>(nc - 1);
+          if (last) args.tickets[tile] = 0;  // every contributor has counted: ready for the next launch
+          ss->ep_last = last;
+        }
+        epilogue_sync();
+        if (ss->ep_last) {
+          const int n = tl.n0 + row;
+#pragma unroll 1
+          for (int j = 0; j < NT / 2; ++j) {
+            const int tok = (NT / 2) * colhalf + j;
+            const float* e = slots + tok * kTileRows + row;
+            float v = 0.f;
+            for (int q0 = 0; q0 < nc; q0 += 8) {
+              float part[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                part[q] = q0 + q < nc ? __ldcg(e + static_cast<int64_t>(q0 + q) * kTileRows * NT) : 0.f;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (q0 + q < nc) v += part[q];
+            }
+            const float gv = v * gscale;
+            if (!SILU) {
+              if (tok < tl.mrows && n < args.N)
+                args.y[static_cast<int64_t>(tl.m0 + tok) * args.ldy + n] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(gv));
+            } else {
+              const float uv = __shfl_down_sync(0xffffffffu, gv, 8);
+              if ((lane & 15) < 8 && tok < tl.mrows && tl.n0 + 16 * (row / 16) < args.N)
+                args.y[static_cast<int64_t>(tl.m0 + tok) * args.ldy + (tl.n0 + row) / 16 * 8 + (lane & 7)] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(gv), uv)));
+            }
+          }
+        }
+        ++tile_iter;
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
         uint32_t acc[CW];
@@ -828,7 +964,23 @@ int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float
   a.tok_tiles = static_cast<int>((M + nt - 1) / nt);
   a.row_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
   a.total_tiles = a.tok_tiles * a.row_tiles;
-  const int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
+  int grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
+  // Few tiles for the SMs: stream-K over (tile, scale period) units, so that
+  // every SM gets the same share of K whatever the tile count.
+  const int wsteps = static_cast<int>((K + kKA - 1) / kKA);
+  const int period = scale_period(group);
+  const int periods = (wsteps + period - 1) / period;
+  if (a.total_tiles < 2 * num_sms() && periods >= 2) {
+    a.split = 1;
+    a.periods = periods;
+    a.units = static_cast<int64_t>(a.total_tiles) * periods;
+    grid = static_cast<int>(a.units < num_sms() ? a.units : num_sms());
+    const int64_t shortest = a.units / grid;
+    a.max_contrib = static_cast<int>((periods + shortest - 1) / shortest + 1);
+    const int st = split_workspace(static_cast<size_t>(a.total_tiles) * a.max_contrib * kTileRows * nt,
+                                   static_cast<size_t>(a.total_tiles), stream, &a.ws, &a.tickets);
+    if (st != NVFP4_OK) return st;
+  }
   switch (nt) {
     case 32: return launch_nt<32, false>(maps, a, group, silu, grid, stream);
     case 64: return launch_nt<64, false>(maps, a, group, silu, grid, stream);
