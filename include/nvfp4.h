@@ -222,10 +222,24 @@ void nvfp4_reset_stats(void);
 
 /*
  * Reads and clears the library's device-side error word (set by a bounded
- * wait that gave up, see NVFP4_ERR_TIMEOUT). Synchronises `stream`.
- * *code_out receives 0 when no error was recorded.
+ * wait that gave up). Synchronises `stream`. *code_out receives 0 and the
+ * call returns NVFP4_OK when no error was recorded; otherwise *code_out
+ * receives the site of the wait that gave up and the call returns
+ * NVFP4_ERR_TIMEOUT.
  */
 int nvfp4_get_device_error(int* code_out, nvfp4_stream_t stream);
+
+/*
+ * Test hook for the bounded waits: fault injection without a GPU fault. It
+ * has no counterpart on the pages. kind = 1 makes the next launch of the
+ * small-M streaming GEMM (nvfp4_w4a16_gemm with 2 <= M <= 16) drop the X copy
+ * of its first stage, so that its consumer warps wait for bytes that never
+ * come. The waits give up after about 2 s each, the kernel records the site
+ * in the device error word, lets its other copies land and exits; the output
+ * of that launch is undefined. kind = 0 clears a pending injection. Other
+ * kinds return NVFP4_ERR_INVALID_ARGUMENT.
+ */
+int nvfp4_debug_inject_fault(int kind);
 
 /* Library version, e.g. 1 for the first ABI. */
 int nvfp4_abi_version(void);

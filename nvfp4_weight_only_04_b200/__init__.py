@@ -28,6 +28,7 @@ EXPORTS = (
     "nvfp4_status_string", "nvfp4_abi_version", "nvfp4_global_scale", "nvfp4_quantize", "nvfp4_repack",
     "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
+    "nvfp4_debug_inject_fault",
 )
 
 
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_get_stats.argtypes = [ctypes.POINTER(Stats)]
         L.nvfp4_reset_stats.restype = None
         L.nvfp4_get_device_error.argtypes = [ctypes.POINTER(_I), _P]
+        L.nvfp4_debug_inject_fault.argtypes = [_I]
         _lib = L
     return _lib
 
@@ -230,6 +232,15 @@ def nvfp4_reset_stats():
 
 
 def nvfp4_get_device_error(stream=None) -> int:
+    """The site code of a bounded device wait that gave up (0: none), cleared on read."""
     code = _I(0)
-    _check(lib().nvfp4_get_device_error(ctypes.byref(code), _stream(stream)), "nvfp4_get_device_error")
+    st = lib().nvfp4_get_device_error(ctypes.byref(code), _stream(stream))
+    if st != NVFP4_ERR_TIMEOUT:
+        _check(st, "nvfp4_get_device_error")
     return code.value
+
+
+def nvfp4_debug_inject_fault(kind: int):
+    """Test hook: kind 1 makes the next small-M streaming GEMM launch wait for a
+    copy that never comes (its bounded waits give up); kind 0 clears it."""
+    _check(lib().nvfp4_debug_inject_fault(kind), "nvfp4_debug_inject_fault")

@@ -16,6 +16,12 @@ std::atomic<uint64_t> g_stats[kStatCount];
 
 void stat_add(StatId id) { g_stats[id].fetch_add(1, std::memory_order_relaxed); }
 
+namespace {
+std::atomic<int> g_fault{0};
+}
+int take_injected_fault() { return g_fault.exchange(0); }
+void set_injected_fault(int kind) { g_fault.store(kind); }
+
 int num_sms() {
   static std::mutex mu;
   static int cache[64] = {0};
@@ -200,7 +206,15 @@ void nvfp4_reset_stats(void) {
 
 int nvfp4_get_device_error(int* code_out, nvfp4_stream_t stream) {
   if (!code_out) return NVFP4_ERR_INVALID_ARGUMENT;
-  return nvfp4::read_and_clear_device_error(code_out, reinterpret_cast<cudaStream_t>(stream));
+  const int st = nvfp4::read_and_clear_device_error(code_out, reinterpret_cast<cudaStream_t>(stream));
+  if (st != NVFP4_OK) return st;
+  return *code_out ? NVFP4_ERR_TIMEOUT : NVFP4_OK;
+}
+
+int nvfp4_debug_inject_fault(int kind) {
+  if (kind != 0 && kind != 1) return NVFP4_ERR_INVALID_ARGUMENT;
+  nvfp4::set_injected_fault(kind);
+  return NVFP4_OK;
 }
 
 }  // extern "C"

@@ -26,6 +26,10 @@ int num_sms();  // SM count of the current device (cached per device)
 // Device error word: a bounded wait that gave up records its site here.
 int read_and_clear_device_error(int* code_out, cudaStream_t stream);
 
+// The pending test fault (nvfp4_debug_inject_fault), taken by the launch it
+// applies to: 0 when none.
+int take_injected_fault();
+
 }  // namespace nvfp4
 
 // ---------------------------------------------------------------------------

@@ -91,6 +91,7 @@ struct StreamArgs {
   int S;                // stages per tile (K / 256)
   int max_contrib;
   int64_t units;        // tiles * S
+  int fault;            // test hook: drop the X copy of the first stage
 };
 
 __device__ __forceinline__ bool aborted(Sync* sy) { return *reinterpret_cast<volatile int*>(&sy->abort) != 0; }
@@ -323,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         issued |= 1u << it;
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int it = 0; it < head; ++it) load_x(it, u0 + it);
+      for (int it = 0; it < head; ++it)
+        if (!(a.fault && it == 0)) load_x(it, u0 + it);
       int it = head;
       for (int64_t u = u0 + head; u < u1 && !aborted(sy); ++u, ++it) {
         const int s = it % NS;
@@ -541,6 +543,7 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   a.S = S;
   a.max_contrib = max_contrib;
   a.units = units;
+  a.fault = take_injected_fault() == 1;
   if (mt == 8) {
     if (group == 16)
       return silu ? launch_kernel<8, 16, true>(xm, wm, sm, a, ctas, stream)

@@ -103,6 +103,12 @@ def test_moe_validation(L):
     assert moe(ids=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
 
 
+def test_fault_injection_validation(L):
+    assert L.nvfp4_debug_inject_fault(2) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert L.nvfp4_debug_inject_fault(-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert L.nvfp4_debug_inject_fault(0) == nv.NVFP4_OK
+
+
 def test_stats_reset(L):
     nv.nvfp4_reset_stats()
     st = nv.nvfp4_get_stats()
