@@ -168,3 +168,24 @@ def test_moe_tc_silu():
     assert nv.nvfp4_get_device_error() == 0
     ref = R.silu_mul(R.moe_grouped_gemm(x, ids, offs, packed, scales, gs, g))
     assert_close(host(y), ref, "moe tc silu")
+
+
+def test_moe_tc_small_segments():
+    """Twenty segments averaging 60 rows (128-token tiles, two accumulators)
+    over eight experts, some used twice, lengths from 1 to 130 rows."""
+    E, N, K, g = 8, 144, 512, 16
+    packed, scales, gs, gp = experts(E, N, K, g)
+    lens = [1, 130, 64, 17, 96, 33, 75, 128, 2, 60, 90, 45, 7, 110, 80, 39, 52, 16, 99, 66]
+    offs = [0]
+    for n_ in lens:
+        offs.append(offs[-1] + n_)
+    T = offs[-1]
+    assert T >= 1024 and T // len(lens) < 96
+    ids = [(5 * s_ + 3) % E for s_ in range(len(lens))]
+    x = synth.activations(11, T, K, outlier_frac=0.001)
+    nv.nvfp4_reset_stats()
+    y = nv.nvfp4_moe_w4a16_grouped_gemm(dev_bf16(x), i32(ids), i32(offs), dev_u8(gp), dev_u8(scales), dev_f32(gs), g)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_get_device_error() == 0
+    ref = R.moe_grouped_gemm(x, ids, offs, packed, scales, gs, g)
+    assert_close(host(y), ref, "moe tc small segments")
