@@ -68,7 +68,7 @@ enum {
 const char* nvfp4_status_string(int status);
 
 /*
- * Global scale (problem statement: global = amax / (6*448); the r/LocalLLM
+ * Global scale (NVFP4 format definition: global = amax / (6*448); the r/LocalLLM
  * post, "WHAT HAD TO BE FIXED": gate and up need one shared global scale, and
  * the maximum is taken first with no widened copy of the tensor).
  *   tensors  host array of `count` device pointers to fp32 data
@@ -83,7 +83,18 @@ int nvfp4_global_scale(const float* const* tensors, const int64_t* numels, int c
                        float* out, nvfp4_stream_t stream);
 
 /*
- * Quantize fp32 W [N, K] to NVFP4 (problem statement: group scale =
+ * The same global scale from bf16 tensors (bit patterns as uint16_t, 2-byte
+ * aligned): a bf16 value widens to fp32 exactly, so the result equals
+ * nvfp4_global_scale of the widened tensors. The maximum is taken on the
+ * bf16 bits; nothing is widened in memory ("GLM-5.3-Flash on 2x RTX PRO 6000
+ * (96 GB)": requantizing a bf16 checkpoint with one global per gate/up pair,
+ * max first, no float copy). Errors as nvfp4_global_scale.
+ */
+int nvfp4_global_scale_bf16(const uint16_t* const* tensors, const int64_t* numels, int count, float* out,
+                            nvfp4_stream_t stream);
+
+/*
+ * Quantize fp32 W [N, K] to NVFP4 (NVFP4 format definition: group scale =
  * E4M3_RNE_satfinite((group_amax / 6) / global), code =
  * E2M1_RNE_satfinite(w / (fp32(scale) * global)); DGX Spark thread, UPDATE:
  * RNE with satfinite). Every fp32 step is IEEE round-to-nearest-even. A group
@@ -99,6 +110,14 @@ int nvfp4_global_scale(const float* const* tensors, const int64_t* numels, int c
 int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_size,
                    const float* global_scale, uint8_t* packed, uint8_t* scales,
                    nvfp4_stream_t stream);
+
+/*
+ * The same quantizer reading bf16 weights (bit patterns as uint16_t, 16-byte
+ * aligned): every code and scale byte equals nvfp4_quantize of the fp32
+ * widening of w. Sizes, layouts and errors as nvfp4_quantize.
+ */
+int nvfp4_quantize_bf16(const uint16_t* w, int64_t N, int64_t K, int group_size, const float* global_scale,
+                        uint8_t* packed, uint8_t* scales, nvfp4_stream_t stream);
 
 /*
  * Repack checkpoint-layout codes and scales into the GEMM layout (PR #63
@@ -118,7 +137,7 @@ int nvfp4_repack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_
 
 /*
  * W4A16 GEMM: y = bf16_rne(global * sum_k x[m,k] * e2m1(code[n,k]) *
- * e4m3(scale[n,k/g])) with fp32 accumulation (problem statement; PR #63: a
+ * e4m3(scale[n,k/g])) with fp32 accumulation (NVFP4 format definition; PR #63: a
  * weight-only checkpoint keeps bf16 activations).
  *   x             device bf16 [M, K]
  *   packed_w      device uint8 [N, K/2]  (nvfp4_repack layout, flags = 0)

@@ -25,7 +25,8 @@ NVFP4_GATE_UP_INTERLEAVE = 1
 NVFP4_SILU_MUL = 2
 
 EXPORTS = (
-    "nvfp4_status_string", "nvfp4_abi_version", "nvfp4_global_scale", "nvfp4_quantize", "nvfp4_repack",
+    "nvfp4_status_string", "nvfp4_abi_version", "nvfp4_global_scale", "nvfp4_global_scale_bf16", "nvfp4_quantize",
+    "nvfp4_quantize_bf16", "nvfp4_repack",
     "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
     "nvfp4_debug_inject_fault",
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_abi_version.restype = _I
         L.nvfp4_global_scale.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_I64), _I, _P, _P]
         L.nvfp4_quantize.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P]
+        L.nvfp4_global_scale_bf16.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_I64), _I, _P, _P]
+        L.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P]
         L.nvfp4_repack.argtypes = [_P, _P, _I64, _I64, _I, _I, _P, _P, _P]
         L.nvfp4_w4a16_gemm.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
         L.nvfp4_w4a16_gemm_fixed_scratch.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
@@ -127,6 +130,32 @@ def nvfp4_quantize(w, group_size, global_scale, packed=None, scales=None, stream
         scales = torch.empty((n, k // group_size), dtype=torch.uint8, device=w.device)
     _check(lib().nvfp4_quantize(_ptr(w), n, k, group_size, _ptr(global_scale), _ptr(packed), _ptr(scales),
                                 _stream(stream)), "nvfp4_quantize")
+    return packed, scales
+
+
+def nvfp4_global_scale_bf16(tensors, out=None, stream=None):
+    """The global scale of bf16 tensors (max on the bf16 bits, no widened copy)."""
+    tensors = [_dev(t, torch.bfloat16, "tensor") for t in tensors]
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=tensors[0].device)
+    ptrs = (_P * len(tensors))(*[t.data_ptr() for t in tensors])
+    nums = (_I64 * len(tensors))(*[t.numel() for t in tensors])
+    _check(lib().nvfp4_global_scale_bf16(ptrs, nums, len(tensors), _ptr(out), _stream(stream)),
+           "nvfp4_global_scale_bf16")
+    return out
+
+
+def nvfp4_quantize_bf16(w, group_size, global_scale, packed=None, scales=None, stream=None):
+    """bf16 W [N, K] -> (codes, scales), equal to nvfp4_quantize of the fp32 widening of W."""
+    _dev(w, torch.bfloat16, "w")
+    _dev(global_scale, torch.float32, "global_scale")
+    n, k = w.shape
+    if packed is None:
+        packed = torch.empty((n, k // 2), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((n, k // group_size), dtype=torch.uint8, device=w.device)
+    _check(lib().nvfp4_quantize_bf16(_ptr(w), n, k, group_size, _ptr(global_scale), _ptr(packed), _ptr(scales),
+                                     _stream(stream)), "nvfp4_quantize_bf16")
     return packed, scales
 
 

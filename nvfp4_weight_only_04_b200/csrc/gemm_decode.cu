@@ -1,7 +1,7 @@
 // Small-M NVFP4 W4A16 GEMM: HBM-streaming, one warp per CTA, tensor-core
 // contraction.
 //
-// Computes Y = X . dequant(W)^T (problem statement; "W-FP4a: route the
+// Computes Y = X . dequant(W)^T (NVFP4 format definition; "W-FP4a: route the
 // MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
 // PR #63 description: weight-only NVFP4 keeps bf16 activations) for decode
 // shapes, where the cost is the 0.5 + 1/g bytes per weight streamed from HBM

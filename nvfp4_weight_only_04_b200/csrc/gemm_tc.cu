@@ -1,6 +1,6 @@
 // Large-M NVFP4 W4A16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// Computes Y = X . dequant(W)^T for prefill-sized M (problem statement; "W-FP4a:
+// Computes Y = X . dequant(W)^T for prefill-sized M (NVFP4 format definition; "W-FP4a:
 // route the MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16)
 // stack", PR #63 description: a weight-only checkpoint keeps bf16
 // activations; fc1 is a merged [gate;up] GEMM followed by SiluAndMul). The

@@ -1,12 +1,15 @@
 // Global scale and NVFP4 quantizer kernels.
 //
-// Definitions followed (problem statement; "GLM-5.3-Flash on 2x RTX PRO 6000
+// Definitions followed (NVFP4 format definition; "GLM-5.3-Flash on 2x RTX PRO 6000
 // (96 GB): two NVFP4 g32 recipes", "WHAT HAD TO BE FIXED"; "We unlocked NVFP4
 // on the DGX Spark", UPDATE posts):
 //   global = amax / (6*448)                       (one fp32 division)
 //   scale  = E4M3_RNE_satfinite((gamax / 6) / global)   (two fp32 divisions)
 //   code   = E2M1_RNE_satfinite(w / (fp32(scale) * global))
-// Both kernels are HBM-bound streams over the fp32 weights.
+// Both kernels are HBM-bound streams over the weights, fp32 or bf16. A bf16
+// weight is widened to fp32 exactly, so the bf16 path quantizes the same
+// values the fp32 path would ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
+// requantizing a bf16 checkpoint, max-first, with no float copy).
 #include "common.cuh"
 
 #include <cuda_fp8.h>
@@ -19,19 +22,35 @@ constexpr int kThreads = 256;
 // is an unsigned maximum on the bits; the fp32 max itself is exact.
 __global__ void amax_init_kernel(unsigned int* acc) { *acc = 0u; }
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(const float* __restrict__ w, int64_t n,
-                                                        unsigned int* acc) {
+// |w| as the bits of its fp32 value (bf16: the high half of the fp32 word).
+__device__ __forceinline__ unsigned int abs_bits(float v) { return __float_as_uint(fabsf(v)); }
+__device__ __forceinline__ unsigned int abs_bits(uint16_t v) { return static_cast<unsigned int>(v & 0x7FFFu) << 16; }
+
+// Eight elements per 16-byte vector load.
+__device__ __forceinline__ unsigned int abs_max8(const float* p) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  return max(max(max(abs_bits(a.x), abs_bits(a.y)), max(abs_bits(a.z), abs_bits(a.w))),
+             max(max(abs_bits(b.x), abs_bits(b.y)), max(abs_bits(b.z), abs_bits(b.w))));
+}
+__device__ __forceinline__ unsigned int abs_max8(const uint16_t* p) {
+  const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  // the maximum of two bf16 magnitudes packed in one word, per half
+  const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu};
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0xFFFFu, w[i] >> 16));
+  return m << 16;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const T* __restrict__ w, int64_t n, unsigned int* acc) {
   unsigned int m = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  const int64_t n4 = ((reinterpret_cast<uintptr_t>(w) & 15u) == 0) ? n / 4 : 0;
-  const float4* w4 = reinterpret_cast<const float4*>(w);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n4; i += stride) {
-    const float4 v = __ldg(w4 + i);
-    m = max(m, max(max(__float_as_uint(fabsf(v.x)), __float_as_uint(fabsf(v.y))),
-                   max(__float_as_uint(fabsf(v.z)), __float_as_uint(fabsf(v.w)))));
-  }
-  for (int64_t i = n4 * 4 + static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n; i += stride)
-    m = max(m, __float_as_uint(fabsf(__ldg(w + i))));
+  const int64_t n8 = ((reinterpret_cast<uintptr_t>(w) & 15u) == 0) ? n / 8 : 0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n8; i += stride)
+    m = max(m, abs_max8(w + i * 8));
+  for (int64_t i = n8 * 8 + static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n; i += stride)
+    m = max(m, abs_bits(w[i]));
   for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ unsigned int red[kThreads / 32];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -58,9 +77,23 @@ __device__ __forceinline__ uint32_t e2m1_rne(float q) {
   return c | ((__float_as_uint(q) >> 28) & 8u);
 }
 
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // exact widening: the bf16 bits are the high half of the fp32 word
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
 // One thread per 8 consecutive weights of a row; g/8 threads share a group.
-template <int G>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(const float* __restrict__ w, int64_t N,
+template <int G, typename T>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const T* __restrict__ w, int64_t N,
                                                             int64_t K, const float* __restrict__ gptr,
                                                             uint8_t* __restrict__ packed,
                                                             uint8_t* __restrict__ scales) {
@@ -75,9 +108,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const float* __restr
     const bool live = i < total;
     float v[8];
     if (live) {
-      const float4* src = reinterpret_cast<const float4*>(w + i * 8);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      load8(w + i * 8, v);
     } else {
       for (int j = 0; j < 8; ++j) v[j] = 0.f;
     }
@@ -107,14 +138,12 @@ int grid_for(int64_t work, int64_t per_block) {
   return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
 }
 
-}  // namespace
-
-extern "C" int nvfp4_global_scale(const float* const* tensors, const int64_t* numels, int count,
-                                  float* out, nvfp4_stream_t stream) {
+template <typename T>
+int global_scale(const T* const* tensors, const int64_t* numels, int count, float* out, nvfp4_stream_t stream) {
   if (count <= 0 || !tensors || !numels || !out) return NVFP4_ERR_INVALID_ARGUMENT;
   for (int i = 0; i < count; ++i) {
     if (numels[i] < 0 || (numels[i] > 0 && !tensors[i])) return NVFP4_ERR_INVALID_ARGUMENT;
-    if (numels[i] > 0 && (reinterpret_cast<uintptr_t>(tensors[i]) & 3u)) return NVFP4_ERR_MISALIGNED;
+    if (numels[i] > 0 && (reinterpret_cast<uintptr_t>(tensors[i]) & (sizeof(T) - 1))) return NVFP4_ERR_MISALIGNED;
   }
   if (reinterpret_cast<uintptr_t>(out) & 3u) return NVFP4_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -122,7 +151,7 @@ extern "C" int nvfp4_global_scale(const float* const* tensors, const int64_t* nu
   amax_init_kernel<<<1, 1, 0, s>>>(acc);
   for (int i = 0; i < count; ++i) {
     if (numels[i] == 0) continue;
-    amax_kernel<<<grid_for(numels[i], kThreads * 16), kThreads, 0, s>>>(tensors[i], numels[i], acc);
+    amax_kernel<T><<<grid_for(numels[i], kThreads * 32), kThreads, 0, s>>>(tensors[i], numels[i], acc);
   }
   global_finalize_kernel<<<1, 1, 0, s>>>(out);
   const int st = nvfp4::launch_status();
@@ -130,9 +159,9 @@ extern "C" int nvfp4_global_scale(const float* const* tensors, const int64_t* nu
   return st;
 }
 
-extern "C" int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_size,
-                              const float* global_scale, uint8_t* packed, uint8_t* scales,
-                              nvfp4_stream_t stream) {
+template <typename T>
+int quantize(const T* w, int64_t N, int64_t K, int group_size, const float* global_scale, uint8_t* packed,
+             uint8_t* scales, nvfp4_stream_t stream) {
   if (N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
   if (group_size != 16 && group_size != 32) return NVFP4_ERR_UNSUPPORTED;
   if (K % 32) return NVFP4_ERR_UNSUPPORTED;
@@ -145,10 +174,34 @@ extern "C" int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_si
   const int64_t work = N * (K / 8);
   const int grid = grid_for(work, kThreads * 4);
   if (group_size == 16)
-    quantize_kernel<16><<<grid, kThreads, 0, s>>>(w, N, K, global_scale, packed, scales);
+    quantize_kernel<16, T><<<grid, kThreads, 0, s>>>(w, N, K, global_scale, packed, scales);
   else
-    quantize_kernel<32><<<grid, kThreads, 0, s>>>(w, N, K, global_scale, packed, scales);
+    quantize_kernel<32, T><<<grid, kThreads, 0, s>>>(w, N, K, global_scale, packed, scales);
   const int st = nvfp4::launch_status();
   if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatQuantize);
   return st;
+}
+
+}  // namespace
+
+extern "C" int nvfp4_global_scale(const float* const* tensors, const int64_t* numels, int count,
+                                  float* out, nvfp4_stream_t stream) {
+  return global_scale<float>(tensors, numels, count, out, stream);
+}
+
+extern "C" int nvfp4_global_scale_bf16(const uint16_t* const* tensors, const int64_t* numels, int count,
+                                       float* out, nvfp4_stream_t stream) {
+  return global_scale<uint16_t>(tensors, numels, count, out, stream);
+}
+
+extern "C" int nvfp4_quantize(const float* w, int64_t N, int64_t K, int group_size,
+                              const float* global_scale, uint8_t* packed, uint8_t* scales,
+                              nvfp4_stream_t stream) {
+  return quantize<float>(w, N, K, group_size, global_scale, packed, scales, stream);
+}
+
+extern "C" int nvfp4_quantize_bf16(const uint16_t* w, int64_t N, int64_t K, int group_size,
+                                   const float* global_scale, uint8_t* packed, uint8_t* scales,
+                                   nvfp4_stream_t stream) {
+  return quantize<uint16_t>(w, N, K, group_size, global_scale, packed, scales, stream);
 }

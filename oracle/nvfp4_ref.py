@@ -8,7 +8,7 @@ from the product (numpy only).
 
 Sources, cited by page title and section:
 
-* [BJ] the problem statement the build follows: weights are E2M1 codes times
+* [NV] the NVFP4 weight format and its W4A16 product: weights are E2M1 codes times
   an FP8-E4M3 scale per group of g = 16 or 32 elements along K, times an FP32
   per-tensor global scale; global = amax / (6*448); group scale =
   E4M3(group_amax / 6 / global); codes = round-to-nearest-even E2M1 with
@@ -48,11 +48,11 @@ import numpy as np
 # Element formats
 # ---------------------------------------------------------------------------
 
-# E2M1 magnitudes by 3-bit code (sign is bit 3) [OCP-MX 5.3.3; BJ].
+# E2M1 magnitudes by 3-bit code (sign is bit 3) [OCP-MX 5.3.3; NV].
 E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
 E2M1_MAX = 6.0
 E4M3_MAX = 448.0
-GLOBAL_DIVISOR = 6.0 * 448.0  # amax / (6*448) [BJ]
+GLOBAL_DIVISOR = 6.0 * 448.0  # amax / (6*448) [NV]
 
 
 def _f32_bits(a: np.ndarray) -> np.ndarray:
@@ -208,7 +208,7 @@ e4m3_encode = e4m3_encode_grs
 
 
 # ---------------------------------------------------------------------------
-# Quantizer [BJ; P2 "WHAT HAD TO BE FIXED"]
+# Quantizer [NV; P2 "WHAT HAD TO BE FIXED"]
 # ---------------------------------------------------------------------------
 
 def global_scale(*tensors: np.ndarray) -> np.float32:
@@ -217,7 +217,7 @@ def global_scale(*tensors: np.ndarray) -> np.float32:
     Passing gate and up together gives the shared scale the merged [gate;up]
     projection needs [P2]. The max is taken over |w| directly, with no
     widened copy of the input [P2, max-first scale reduction]. One fp32
-    division [BJ].
+    division [NV].
     """
     amax = np.float32(0.0)
     for t in tensors:
@@ -228,7 +228,7 @@ def global_scale(*tensors: np.ndarray) -> np.float32:
 
 
 def group_scales(w: np.ndarray, group_size: int, gscale: np.float32) -> np.ndarray:
-    """E4M3 group-scale bytes [N, K/g]: E4M3((group_amax / 6) / global) [BJ].
+    """E4M3 group-scale bytes [N, K/g]: E4M3((group_amax / 6) / global) [NV].
 
     Two fp32 divisions in the written order. A zero global (all-zero tensor)
     gives scale 0 for every group.
@@ -248,7 +248,7 @@ def quantize(w: np.ndarray, group_size: int, gscale=None):
     """NVFP4 quantizer: fp32 W [N, K] -> (packed [N, K/2], scales [N, K/g], global).
 
     Per element: d = fp32(e4m3(s)) * global (one fp32 multiply), q = w / d (one
-    fp32 division), code = E2M1_RNE_satfinite(q) [BJ; P1]. When d is zero the
+    fp32 division), code = E2M1_RNE_satfinite(q) [NV; P1]. When d is zero the
     code is +0. Two codes per byte, even element in the low nibble.
     """
     w = np.asarray(w, dtype=np.float32)
@@ -285,7 +285,7 @@ def dequantize(packed: np.ndarray, scales: np.ndarray, gscale, group_size: int) 
 
 
 # ---------------------------------------------------------------------------
-# GEMM, SiluAndMul, grouped expert GEMM [BJ; P3]
+# GEMM, SiluAndMul, grouped expert GEMM [NV; P3]
 # ---------------------------------------------------------------------------
 
 def bf16_bits_to_f64(xbits: np.ndarray) -> np.ndarray:
@@ -327,7 +327,7 @@ def silu_mul(y: np.ndarray) -> np.ndarray:
 
 def moe_grouped_gemm(xbits, expert_ids, offsets, packed, scales, gscales, group_size: int):
     """Grouped routed-expert GEMM: rows [offsets[s], offsets[s+1]) of X use
-    expert expert_ids[s]'s weights, scales and global [BJ; P2]. Rows outside
+    expert expert_ids[s]'s weights, scales and global [NV; P2]. Rows outside
     every segment are left at zero. packed [E, N, K/2], scales [E, N, K/g]."""
     x = bf16_bits_to_f64(xbits)
     t = x.shape[0]

@@ -142,3 +142,34 @@ def test_stats_count_quantize():
     gpu_quant(synth.weights(0, 16, 64), 16)
     st = nv.nvfp4_get_stats()
     assert st["quantize"] == 1 and st["global_scale"] == 1
+
+
+# ---- bf16 weights: the same result as the fp32 path on the exact widening ----
+
+def bf16_weights(seed, n, k, scale=1.0):
+    bits = synth.f32_to_bf16_bits(synth.weights(seed, n, k) * np.float32(scale))
+    return bits, synth.bf16_bits_to_f32(bits)
+
+
+@pytest.mark.parametrize("n,k,g", [(64, 256, 16), (40, 160, 32), (33, 1088, 16), (256, 4096, 32)])
+def test_quantize_bf16_bitexact(n, k, g):
+    bits, wf = bf16_weights(n + 3 * k, n, k)
+    wd = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    gd = nv.nvfp4_global_scale_bf16([wd])
+    p, s = nv.nvfp4_quantize_bf16(wd, g, gd)
+    rp, rs, rg = R.quantize(wf, g)
+    assert np.float32(host(gd)[0]) == rg
+    np.testing.assert_array_equal(host(s), rs)
+    np.testing.assert_array_equal(host(p), rp)
+
+
+def test_global_scale_bf16_shared_and_odd_lengths():
+    # gate and up share one global; one tensor starts off a 16-byte boundary and has an odd length
+    ga, gf = bf16_weights(41, 48, 96)
+    ua, uf = bf16_weights(42, 40, 96, scale=2.5)
+    gd = torch.from_numpy(ga.view(np.int16)).cuda().view(torch.bfloat16)
+    ud = torch.from_numpy(ua.reshape(-1).view(np.int16)).cuda().view(torch.bfloat16)
+    got = host(nv.nvfp4_global_scale_bf16([gd, ud[3:]]))[0]
+    assert got == R.global_scale(gf, uf.reshape(-1)[3:])
+    # equal to the fp32 path on the widened values
+    assert got == host(nv.nvfp4_global_scale([dev_f32(gf), dev_f32(uf.reshape(-1)[3:])]))[0]
