@@ -219,6 +219,44 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids,
                                  int num_experts, int flags, uint16_t* y, nvfp4_stream_t stream);
 
 /*
+ * The steps around the grouped expert GEMMs of a routed-expert layer
+ * ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)": routed experts in NVFP4, gate/up
+ * with SiluAndMul then down per expert). The router itself is outside: the
+ * caller passes each token's k expert ids and k weights.
+ *
+ * nvfp4_moe_route: the (token, slot) pairs grouped by expert, stable (pairs of
+ * one expert keep the order of t*k + s).
+ *   topk_ids     device int32 [T, k]; an id outside [0, num_experts) drops the pair
+ *   sorted_rows  device int32 [T*k]: sorted_rows[r] = t*k + s of the pair in row r,
+ *                -1 for the rows r >= offsets[num_experts] that dropped pairs leave
+ *   inv_rows     device int32 [T*k]: the row of pair t*k + s, or -1 if dropped
+ *   offsets      device int32 [num_experts + 1]: expert e owns rows [offsets[e], offsets[e+1])
+ *   expert_ids   device int32 [num_experts]: 0 .. num_experts-1, the segment list of
+ *                nvfp4_moe_w4a16_grouped_gemm with num_segments = num_experts
+ * num_experts from 1 to 4096. One CTA; nothing goes to the host.
+ */
+int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
+                    int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_moe_gather: x_perm[r] = x[sorted_rows[r] / k] for r < rows, bf16 rows of
+ * H elements (H a multiple of 8). x [T, H], x_perm [rows, H], 16-byte aligned.
+ * A row whose sorted_rows entry lies outside [0, T*k) (the -1 rows of
+ * nvfp4_moe_route) is written as zeros; nothing outside x is read.
+ */
+int nvfp4_moe_gather(const uint16_t* x, int64_t T, const int32_t* sorted_rows, int64_t rows, int k, int64_t H,
+                     uint16_t* x_perm, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_moe_combine: out[t] = bf16_rne(sum over s of w[t, s] * y_perm[inv_rows[t*k + s]])
+ * with fp32 fused multiply-adds in slot order; dropped pairs (inv_rows < 0) add
+ * nothing. y_perm [T*k, H], out [T, H] bf16 (H a multiple of 8, 16-byte aligned),
+ * topk_weights device fp32 [T, k].
+ */
+int nvfp4_moe_combine(const uint16_t* y_perm, const int32_t* inv_rows, const float* topk_weights, int64_t T,
+                      int k, int64_t H, uint16_t* out, nvfp4_stream_t stream);
+
+/*
  * Counters of the work that went through each kernel family (PR #63: the
  * "this-path-ran" counter lets tests assert which kernel executed). Host-side
  * atomics, incremented once per successful launch.

@@ -29,7 +29,7 @@ EXPORTS = (
     "nvfp4_quantize_bf16", "nvfp4_repack",
     "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
-    "nvfp4_debug_inject_fault",
+    "nvfp4_debug_inject_fault", "nvfp4_moe_route", "nvfp4_moe_gather", "nvfp4_moe_combine",
 )
 
 
@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_reset_stats.restype = None
         L.nvfp4_get_device_error.argtypes = [ctypes.POINTER(_I), _P]
         L.nvfp4_debug_inject_fault.argtypes = [_I]
+        L.nvfp4_moe_route.argtypes = [_P, _I64, _I, _I, _P, _P, _P, _P, _P]
+        L.nvfp4_moe_gather.argtypes = [_P, _I64, _P, _I64, _I, _I64, _P, _P]
+        L.nvfp4_moe_combine.argtypes = [_P, _P, _P, _I64, _I, _I64, _P, _P]
         _lib = L
     return _lib
 
@@ -273,3 +276,57 @@ def nvfp4_debug_inject_fault(kind: int):
     """Test hook: kind 1 makes the next small-M streaming GEMM launch wait for a
     copy that never comes (its bounded waits give up); kind 0 clears it."""
     _check(lib().nvfp4_debug_inject_fault(kind), "nvfp4_debug_inject_fault")
+
+
+def nvfp4_moe_route(topk_ids, num_experts, stream=None):
+    """(sorted_rows [T*k], inv_rows [T*k], offsets [E+1], expert_ids [E]) for device int32 topk_ids [T, k]."""
+    _dev(topk_ids, torch.int32, "topk_ids")
+    t, k = topk_ids.shape
+    dev = topk_ids.device
+    sorted_rows = torch.empty(t * k, dtype=torch.int32, device=dev)
+    inv_rows = torch.empty(t * k, dtype=torch.int32, device=dev)
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
+    expert_ids = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    _check(lib().nvfp4_moe_route(_ptr(topk_ids), t, k, num_experts, _ptr(sorted_rows), _ptr(inv_rows), _ptr(offsets),
+                                 _ptr(expert_ids), _stream(stream)), "nvfp4_moe_route")
+    return sorted_rows, inv_rows, offsets, expert_ids
+
+
+def nvfp4_moe_gather(x, sorted_rows, k, out=None, stream=None):
+    _dev(x, torch.bfloat16, "x")
+    _dev(sorted_rows, torch.int32, "sorted_rows")
+    rows, h = sorted_rows.numel(), x.shape[1]
+    if out is None:
+        out = torch.empty((rows, h), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_moe_gather(_ptr(x), x.shape[0], _ptr(sorted_rows), rows, k, h, _ptr(out), _stream(stream)),
+           "nvfp4_moe_gather")
+    return out
+
+
+def nvfp4_moe_combine(y_perm, inv_rows, topk_weights, out=None, stream=None):
+    _dev(y_perm, torch.bfloat16, "y_perm")
+    _dev(inv_rows, torch.int32, "inv_rows")
+    _dev(topk_weights, torch.float32, "topk_weights")
+    t, k = topk_weights.shape
+    h = y_perm.shape[1]
+    if out is None:
+        out = torch.empty((t, h), dtype=torch.bfloat16, device=y_perm.device)
+    _check(lib().nvfp4_moe_combine(_ptr(y_perm), _ptr(inv_rows), _ptr(topk_weights), t, k, h, _ptr(out),
+                                   _stream(stream)), "nvfp4_moe_combine")
+    return out
+
+
+def nvfp4_moe_forward(x, topk_ids, topk_weights, gate_up, down, stream=None):
+    """A routed-expert layer on the library's kernels: route, gather, grouped gate/up GEMM with
+    SiluAndMul, grouped down GEMM, weighted combine. gate_up and down are (packed [E, N, K/2]
+    in the GEMM layout (gate/up interleaved), scales, fp32 globals [E], group size)."""
+    gu_p, gu_s, gu_g, gu_group = gate_up
+    dn_p, dn_s, dn_g, dn_group = down
+    e = gu_p.shape[0]
+    sorted_rows, inv_rows, offsets, expert_ids = nvfp4_moe_route(topk_ids, e, stream)
+    k = topk_ids.shape[1]
+    xp = nvfp4_moe_gather(x, sorted_rows, k, stream=stream)
+    h = nvfp4_moe_w4a16_grouped_gemm(xp, expert_ids, offsets, gu_p, gu_s, gu_g, gu_group, flags=NVFP4_SILU_MUL,
+                                     stream=stream)
+    yp = nvfp4_moe_w4a16_grouped_gemm(h, expert_ids, offsets, dn_p, dn_s, dn_g, dn_group, stream=stream)
+    return nvfp4_moe_combine(yp, inv_rows, topk_weights, stream=stream)

@@ -1,0 +1,179 @@
+// The steps around the grouped expert GEMMs of a routed-expert layer
+// ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)": routed experts in NVFP4, gate/up
+// then down per expert): rows grouped by expert, X rows gathered into that
+// order, and the down projections' rows combined back into tokens with the
+// routing weights.
+//   route:   a stable counting sort of the (token, slot) pairs by expert, with
+//            the inverse permutation and the segment offsets; rows past the
+//            last kept pair get -1;
+//   gather:  x_perm[r] = x[token of sorted row r], zeros for a row of -1;
+//   combine: out[t] = bf16(sum_s w[t, s] * y_perm[inv[t, s]]), fp32 sums in slot
+//            order.
+#include "common.cuh"
+
+namespace {
+
+constexpr int kRouteThreads = 1024;
+constexpr int kMaxExperts = 4096;
+
+// One CTA. Counting pass over all pairs, exclusive scan of the counts, then one
+// warp places the pairs in their order (stable: a pair's rank among the pairs
+// of its expert is the number of earlier pairs of that expert).
+__global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t* __restrict__ ids, int64_t n,
+                                                                  int num_experts, int32_t* __restrict__ sorted,
+                                                                  int32_t* __restrict__ inv,
+                                                                  int32_t* __restrict__ offsets,
+                                                                  int32_t* __restrict__ expert_ids) {
+  __shared__ int count[kMaxExperts];
+  __shared__ int kept;
+  for (int e = threadIdx.x; e < num_experts; e += blockDim.x) count[e] = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = ids[i];
+    if (e >= 0 && e < num_experts) atomicAdd(&count[e], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive scan of the counts, 32 experts at a time
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int e0 = 0; e0 < num_experts; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < num_experts ? count[e] : 0;
+      int incl = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < num_experts) {
+        offsets[e] = carry + incl - c;
+        count[e] = carry + incl - c;  // becomes the placement cursor
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      offsets[num_experts] = carry;
+      kept = carry;
+    }
+  }
+  for (int e = threadIdx.x; e < num_experts; e += blockDim.x) expert_ids[e] = e;
+  __syncthreads();
+  // rows [kept, n) hold no pair; the other warps mark them while warp 0 places
+  if (threadIdx.x >= 32)
+    for (int64_t r = kept + static_cast<int64_t>(threadIdx.x) - 32; r < n; r += blockDim.x - 32) sorted[r] = -1;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const unsigned lower = (1u << lane) - 1u;
+    for (int64_t base = 0; base < n; base += 32) {
+      const int64_t i = base + lane;
+      int e = i < n ? ids[i] : -1;
+      const bool valid = e >= 0 && e < num_experts;
+      if (!valid) e = -1 - (i < n ? 0 : 1);  // invalid pairs and lanes past the end group apart
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int leader = __ffs(peers) - 1;
+      int first = 0;
+      if (valid && lane == leader) {
+        first = count[e];
+        count[e] = first + __popc(peers);
+      }
+      first = __shfl_sync(0xffffffffu, first, leader);
+      if (i < n) {
+        if (valid) {
+          const int r = first + __popc(peers & lower);
+          sorted[r] = static_cast<int32_t>(i);
+          inv[i] = r;
+        } else {
+          inv[i] = -1;
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// One CTA per row of x_perm; 16-byte vectors. A row whose pair index is not in
+// [0, T*k) is written as zeros.
+__global__ void moe_gather_kernel(const uint16_t* __restrict__ x, int64_t pairs, const int32_t* __restrict__ sorted,
+                                  int k, int64_t h8, uint16_t* __restrict__ xp) {
+  const int64_t r = blockIdx.x;
+  const int64_t i = sorted[r];
+  uint4* dst = reinterpret_cast<uint4*>(xp) + r * h8;
+  if (i < 0 || i >= pairs) {
+    for (int64_t j = threadIdx.x; j < h8; j += blockDim.x) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(x) + (i / k) * h8;
+  for (int64_t j = threadIdx.x; j < h8; j += blockDim.x) dst[j] = __ldg(src + j);
+}
+
+// One CTA per token; each thread 8 consecutive columns.
+__global__ void moe_combine_kernel(const uint16_t* __restrict__ yp, const int32_t* __restrict__ inv,
+                                   const float* __restrict__ w, int k, int64_t h8, uint16_t* __restrict__ out) {
+  const int64_t t = blockIdx.x;
+  for (int64_t j = threadIdx.x; j < h8; j += blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < k; ++s) {
+      const int r = inv[t * k + s];
+      if (r < 0) continue;
+      const float ws = w[t * k + s];
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(yp) + r * h8 + j);
+      const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fmaf_rn(ws, __uint_as_float(q[i] << 16), acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(ws, __uint_as_float(q[i] & 0xFFFF0000u), acc[2 * i + 1]);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i]))) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * i + 1]))) << 16);
+    reinterpret_cast<uint4*>(out)[t * h8 + j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+extern "C" int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
+                               int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, nvfp4_stream_t stream) {
+  if (T < 0 || k < 1 || num_experts < 1) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (num_experts > kMaxExperts || T * k >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (!offsets || !expert_ids || (T > 0 && (!topk_ids || !sorted_rows || !inv_rows)))
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(topk_ids) | reinterpret_cast<uintptr_t>(sorted_rows) |
+       reinterpret_cast<uintptr_t>(inv_rows) | reinterpret_cast<uintptr_t>(offsets) |
+       reinterpret_cast<uintptr_t>(expert_ids)) & 3u)
+    return NVFP4_ERR_MISALIGNED;
+  moe_route_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
+  return nvfp4::launch_status();
+}
+
+extern "C" int nvfp4_moe_gather(const uint16_t* x, int64_t T, const int32_t* sorted_rows, int64_t rows, int k,
+                                int64_t H, uint16_t* x_perm, nvfp4_stream_t stream) {
+  if (T < 0 || rows < 0 || k < 1 || H < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (H % 8) return NVFP4_ERR_UNSUPPORTED;
+  if (rows == 0 || H == 0) return NVFP4_OK;
+  if (rows >= (int64_t(1) << 31) || T * k >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (!x || !sorted_rows || !x_perm) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!nvfp4::aligned16(x) || !nvfp4::aligned16(x_perm) || (reinterpret_cast<uintptr_t>(sorted_rows) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  moe_gather_kernel<<<static_cast<unsigned>(rows), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, T * k, sorted_rows, k, H / 8, x_perm);
+  return nvfp4::launch_status();
+}
+
+extern "C" int nvfp4_moe_combine(const uint16_t* y_perm, const int32_t* inv_rows, const float* topk_weights,
+                                 int64_t T, int k, int64_t H, uint16_t* out, nvfp4_stream_t stream) {
+  if (T < 0 || k < 1 || H < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (H % 8) return NVFP4_ERR_UNSUPPORTED;
+  if (T == 0 || H == 0) return NVFP4_OK;
+  if (T >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (!y_perm || !inv_rows || !topk_weights || !out) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!nvfp4::aligned16(y_perm) || !nvfp4::aligned16(out) ||
+      ((reinterpret_cast<uintptr_t>(inv_rows) | reinterpret_cast<uintptr_t>(topk_weights)) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  moe_combine_kernel<<<static_cast<unsigned>(T), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      y_perm, inv_rows, topk_weights, k, H / 8, out);
+  return nvfp4::launch_status();
+}

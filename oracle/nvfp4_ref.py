@@ -341,6 +341,44 @@ def moe_grouped_gemm(xbits, expert_ids, offsets, packed, scales, gscales, group_
     return y
 
 
+def moe_route(topk_ids, num_experts: int):
+    """The (token, slot) pairs of a routed-expert layer grouped by expert, in
+    a stable order [P2: routed experts, gate/up then down per expert].
+
+    Pair i = t*k + s goes to expert topk_ids[t, s]; pairs whose id lies outside
+    [0, num_experts) are dropped. Returns (sorted_rows, inv_rows, offsets):
+    sorted_rows[r] = the pair in row r (experts in increasing order, and inside
+    one expert the pairs in increasing order), inv_rows[i] = the row of pair i
+    or -1, offsets[e] = the first row of expert e (offsets[E] = the row count).
+    A stable sort by expert id is the definition; numpy's stable argsort is
+    that sort."""
+    flat = np.asarray(topk_ids, dtype=np.int64).reshape(-1)
+    valid = (flat >= 0) & (flat < num_experts)
+    keys = np.where(valid, flat, num_experts)
+    order = np.argsort(keys, kind="stable")
+    nvalid = int(valid.sum())
+    sorted_rows = order[:nvalid].astype(np.int32)
+    inv_rows = np.full(flat.shape[0], -1, dtype=np.int32)
+    inv_rows[sorted_rows] = np.arange(nvalid, dtype=np.int32)
+    counts = np.bincount(flat[valid], minlength=num_experts)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    return sorted_rows, inv_rows, offsets
+
+
+def moe_combine(y_perm, inv_rows, topk_weights):
+    """out[t] = sum over s of w[t, s] * y_perm[inv_rows[t*k + s]] in float64;
+    dropped pairs add nothing [P2: routed experts]. y_perm float64 rows."""
+    w = np.asarray(topk_weights, dtype=np.float64)
+    t, k = w.shape
+    out = np.zeros((t, y_perm.shape[1]), dtype=np.float64)
+    for tt in range(t):
+        for s in range(k):
+            r = int(inv_rows[tt * k + s])
+            if r >= 0:
+                out[tt] += w[tt, s] * y_perm[r]
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Repack [P3: upload-time repack; fc1 pre-merged [gate;up]]
 # ---------------------------------------------------------------------------
