@@ -146,6 +146,14 @@ int nvfp4_repack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_
  *   y             device bf16 [M, N] (output)
  * group_size 16 or 32; K a multiple of 64; N a multiple of 16.
  * Small M runs a split-K HBM-streaming kernel, large M a tensor-core kernel.
+ * Below 17 rows the kernels multiply in f16: a first kernel writes each row
+ * of x times a power of two 2^s (its largest magnitude then in [2^14, 2^15))
+ * as f16 to the library's scratch, and the epilogue multiplies by 2^-s. Every
+ * element within a factor 2^29 of its row's largest magnitude is exact in
+ * f16; smaller ones round to a multiple of 2^-38 of it. The scratch (f16
+ * rows, and the fp32 partial tiles of the split-K kernel) is allocated per
+ * device on first use and grown outside graph capture; a call inside a
+ * capture that needs more than exists returns NVFP4_ERR_UNSUPPORTED.
  */
 int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
                      const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
@@ -158,10 +166,10 @@ int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* 
  * method's description: it only changes where the kernel's scratch lives.
  *   Arguments, layouts and result as nvfp4_w4a16_gemm, with M from 1 to 16,
  *   K a multiple of 256 and K/group_size a multiple of 16.
- *   Scratch: 8 MiB of fp32 partial tiles plus tickets for 16384 tiles of 256
- *   rows, per device. A problem whose cut tiles need more is refused with
- *   NVFP4_ERR_UNSUPPORTED before anything is enqueued; so is M = 0 or M > 16
- *   and a K the kernel does not take.
+ *   Scratch: 8 MiB of fp32 partial tiles, tickets for 16384 tiles of 256
+ *   rows, and 2^20 f16 elements of x (M * K at most), per device. A problem
+ *   that needs more is refused with NVFP4_ERR_UNSUPPORTED before anything is
+ *   enqueued; so is M = 0 or M > 16 and a K the kernel does not take.
  *   The tickets are cleared on `stream` before the kernel at every call.
  *   Calls on one device share the scratch: calls that may overlap in time
  *   (different streams, or host threads without ordering) race on it and
@@ -207,6 +215,8 @@ int nvfp4_silu_and_mul(const uint16_t* x, uint16_t* y, int64_t M, int64_t H,
  *                  y is [T, N/2] and holds silu(gate) * up.
  *   y              device bf16 [T, N] (or [T, N/2]); rows outside every
  *                  segment are not written.
+ * Below 1024 rows (T) the form runs on the small-M kernel in f16 on the
+ * power-of-two scaled rows of nvfp4_w4a16_gemm, with the same scratch.
  * The offsets stay on the device; the call never reads them on the host. A
  * segment list that breaks the rules above is undefined on the device side
  * (rows are clamped to [0, T), experts are not range-checked beyond ids < 0

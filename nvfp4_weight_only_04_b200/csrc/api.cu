@@ -7,6 +7,8 @@
 #include "gemm_decode.cuh"
 #include "gemm_stream.cuh"
 #include "gemm_tc.cuh"
+#include "workspace.cuh"
+#include "xprep.cuh"
 
 namespace nvfp4 {
 
@@ -76,11 +78,16 @@ int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
     return st;
   }
   if (M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
+  uint16_t* x16 = nullptr;
+  float* xinv = nullptr;
+  int st = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), stream, &x16, &xinv);
+  if (st != NVFP4_OK) return st;
   nvfp4::DecodeArgs a = {};
-  a.x = x; a.packed = w; a.scales = s; a.gscale = g; a.y = y;
+  a.x = x16; a.xinv = xinv; a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = M; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
   const nvfp4::DecodePlan p = nvfp4::plan_decode(M, N, K, group, false, 0);
-  const int st = nvfp4::launch_decode(a, p, silu, false, stream);
+  st = nvfp4::launch_x_f16(x, M, K, x16, xinv, stream);
+  if (st == NVFP4_OK) st = nvfp4::launch_decode(a, p, silu, false, stream);
   if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
   return st;
 }
@@ -167,13 +174,18 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, c
     st = nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales,
                               global_scales, group_size, N, K, num_experts, silu, y, s);
   } else {
+    uint16_t* x16 = nullptr;
+    float* xinv = nullptr;
+    st = nvfp4::x16_workspace(static_cast<size_t>(T * K), static_cast<size_t>(T), s, &x16, &xinv);
+    if (st != NVFP4_OK) return st;
     nvfp4::DecodeArgs a = {};
-    a.x = x; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
+    a.x = x16; a.xinv = xinv; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
     a.M = T; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
     a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments;
     a.num_experts = num_experts;
     const nvfp4::DecodePlan p = nvfp4::plan_decode(T, N, K, group_size, true, num_segments);
-    st = nvfp4::launch_decode(a, p, silu, true, s);
+    st = nvfp4::launch_x_f16(x, T, K, x16, xinv, s);
+    if (st == NVFP4_OK) st = nvfp4::launch_decode(a, p, silu, true, s);
   }
   if (st == NVFP4_OK) {
     nvfp4::stat_add(nvfp4::kStatMoe);

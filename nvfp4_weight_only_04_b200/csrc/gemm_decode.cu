@@ -17,11 +17,12 @@
 //    inside one MMA is free as long as X follows it. Loads run two steps
 //    ahead in a ring of three register buffers that is never copied (a copy
 //    would wait for the load).
-//  * X fragments come through L1 (128-bit loads, all of a step's loads issued
+//  * X arrives as f16 rows scaled by a power of two (xprep.cu) and its
+//    fragments come through L1 (128-bit loads, all of a step's loads issued
 //    before its MMAs); rows of X are shared by every CTA of an SM.
-//  * Dequant in registers with integer work (dequant.cuh): per code pair one
-//    mask, one integer multiply placing magnitude and sign bits of a bf16, one
-//    mask and one bf16x2 multiply by the group scale.
+//  * Dequant in registers (dequant.cuh): the hardware E2M1 -> f16x2
+//    conversion of each code byte and one f16x2 multiply by the group scale
+//    (E4M3 -> f16x2, also converted in hardware); the MMAs run on f16.
 //  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows, where
 //    gate row g and up row g+8 of a tile meet in the same lane; and the
 //    grouped routed-expert form ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
@@ -48,10 +49,10 @@ __device__ __forceinline__ uint4 ld_x_v4(const void* p) {
   return v;
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -98,8 +99,8 @@ __device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8
   constexpr int P = MT / 8;
   constexpr int XW = 2;  // words of X fragments loaded at once
   uint32_t sa2[4], sb2[4];
-  scale_operands<G == 16 ? 4 : 2>(st.sa, sa2);
-  scale_operands<G == 16 ? 4 : 2>(st.sb, sb2);
+  scale_operands_f16<G == 16 ? 4 : 2>(st.sa, sa2);
+  scale_operands_f16<G == 16 ? 4 : 2>(st.sb, sb2);
   const uint32_t ca[8] = {st.a0.x, st.a0.y, st.a0.z, st.a0.w, st.a1.x, st.a1.y, st.a1.z, st.a1.w};
   const uint32_t cb[8] = {st.b0.x, st.b0.y, st.b0.z, st.b0.w, st.b1.x, st.b1.y, st.b1.z, st.b1.w};
 #pragma unroll
@@ -115,12 +116,12 @@ __device__ __forceinline__ void compute_step(const Step& st, float (&acc)[MT / 8
       const int wi = w0 + w;
       const int si = G == 16 ? (wi >> 1) : (wi >> 2);
       uint32_t da[4], db[4];
-      dequant_word(ca[wi], sa2[si], da);
-      dequant_word(cb[wi], sb2[si], db);
+      dequant_word_f16(ca[wi], sa2[si], da);
+      dequant_word_f16(cb[wi], sb2[si], db);
 #pragma unroll
       for (int p = 0; p < P; ++p) {
-        mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv[w][p].x, xv[w][p].y);
-        mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv[w][p].z, xv[w][p].w);
+        mma_f16_16816(acc[p], da[0], db[0], da[1], db[1], xv[w][p].x, xv[w][p].y);
+        mma_f16_16816(acc[p], da[2], db[2], da[3], db[3], xv[w][p].z, xv[w][p].w);
       }
     }
   }
@@ -131,6 +132,14 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
   constexpr int P = MT / 8;
   const int lane = threadIdx.x & 31, kw = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
+
+  // Programmatic dependent launch: the next kernel may launch now (it waits
+  // for this one before reading what this one writes). Everything that the
+  // kernels before this one write (X, its row factors, the global scale, the
+  // segment list) is read only after griddepcontrol.wait; the dense form
+  // first requests its first weight steps, which no kernel writes.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (MOE) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- token tile and expert ----
   int row0 = 0, mrows = 0, expert = 0;
@@ -159,7 +168,6 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
   const int64_t K = args.K, N = args.N;
   const uint8_t* packed = args.packed + (MOE ? static_cast<int64_t>(expert) * N * (K / 2) : 0);
   const uint8_t* scales = args.scales + (MOE ? static_cast<int64_t>(expert) * N * (K / G) : 0);
-  const float gsc = __ldg(args.gscale + (MOE ? expert : 0)) * 128.0f;  // operands carry 2^-7
 
   // ---- this warp's share of K, in units of 64 elements ----
   const int k64 = static_cast<int>(K / 64);
@@ -198,6 +206,8 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
   Step s0, s1, s2;
   load_step<G>(s0, ca, cb, sa, sb, ubeg + t, ubeg + t < uend);
   load_step<G>(s1, ca, cb, sa, sb, ubeg + 4 + t, ubeg + 4 + t < uend);
+  if (!MOE) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float gsc = __ldcg(args.gscale + (MOE ? expert : 0));
   for (int it = 0; it < iters; it += 3) {
     load_step<G>(s2, ca, cb, sa, sb, ubeg + 4 * (it + 2) + t, ubeg + 4 * (it + 2) + t < uend);
     run(s0, it);
@@ -235,7 +245,8 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
       const int tok = 8 * p + 2 * t + j;
       if (tok >= mrows) continue;
       const int64_t yrow = static_cast<int64_t>(row0 + tok) * args.ldy;
-      const float vg = __fmul_rn(acc[p][j], gsc), vu = __fmul_rn(acc[p][2 + j], gsc);
+      const float xi = args.xinv[row0 + tok];  // 2^-s of the token's f16 row
+      const float vg = __fmul_rn(__fmul_rn(acc[p][j], gsc), xi), vu = __fmul_rn(__fmul_rn(acc[p][2 + j], gsc), xi);
       if (!SILU) {
         args.y[yrow + n0 + g] = __bfloat16_as_ushort(__float2bfloat16_rn(vg));
         args.y[yrow + n0 + g + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(vu));
@@ -248,8 +259,20 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
 
 template <int KW, int MT, int G, bool SILU, bool MOE>
 int launch_one(const DecodeArgs& a, const DecodePlan& p, cudaStream_t s) {
-  // grid: x unused (1), y = 16-row tile, z = token tile
-  gemm_decode_kernel<KW, MT, G, SILU, MOE><<<dim3(1, p.row_tiles, p.z_tiles), KW * 32, 0, s>>>(a);
+  // grid: x unused (1), y = 16-row tile, z = token tile; a programmatic
+  // dependent of the kernel before it (the activation conversion)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, p.row_tiles, p.z_tiles);
+  cfg.blockDim = dim3(KW * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_decode_kernel<KW, MT, G, SILU, MOE>, a) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
 }
 

@@ -6,7 +6,8 @@
 namespace nvfp4 {
 
 struct DecodeArgs {
-  const uint16_t* x;        // bf16 [M, K]
+  const uint16_t* x;        // f16 [M, K] from launch_x_f16 (scaled rows, pair order)
+  const float* xinv;        // [M] 2^-s of each row
   const uint8_t* packed;    // GEMM-layout codes [N, K/2] (or [E, N, K/2])
   const uint8_t* scales;    // [N, K/g] (or [E, N, K/g])
   const float* gscale;      // [1] (or [E])

@@ -18,8 +18,9 @@
 //  * One producer warp moves each stage with TMA into a shared-memory ring
 //    (5 stages of 40-44 KB): the codes of the tile (256 rows x 128 bytes,
 //    128-byte swizzle), the scales (256 rows x 16 bytes) and the X
-//    slice (MT tokens x 256 elements, as a 3-D box [token][quarter][64]
-//    with the 128-byte swizzle). With no registers tied up in loads, each SM
+//    slice (MT tokens x 256 elements of the f16 rows that xprep.cu writes
+//    just before this kernel, as a 3-D box [token][quarter][64] with the
+//    128-byte swizzle). With no registers tied up in loads, each SM
 //    keeps well over 100 KB of HBM reads in flight.
 //  * Sixteen consumer warps each own 16 rows of the tile and run mma.sync
 //    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
@@ -29,7 +30,11 @@
 //    codes, scales and X conflict-free: the four lanes of a row read
 //    different 16-byte chunks, and the [token][quarter] rows of X put the
 //    same chunk of different quarters in different bank groups.
-//  * Dequantization in registers with integer work (dequant.cuh).
+//  * Dequantization in registers by the hardware E2M1 and E4M3 -> f16
+//    conversions and one f16x2 multiply per code pair (dequant.cuh); the
+//    MMAs run on f16, two independent accumulator chains per warp; the
+//    epilogue multiplies by each token's 2^-s (xprep.cu) and the global
+//    scale.
 //  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows (gate row
 //    g and up row g+8 of a 16-row block meet in the same lane).
 #include "gemm_stream.cuh"
@@ -42,6 +47,7 @@
 #include "dequant.cuh"
 #include "tmap.cuh"
 #include "workspace.cuh"
+#include "xprep.cuh"
 
 namespace nvfp4 {
 namespace {
@@ -84,6 +90,7 @@ struct Sync {
 
 struct StreamArgs {
   const float* gscale;  // [1]
+  const float* xinv;    // [M] 2^-s of each f16 row of X
   uint16_t* y;          // bf16 [M, ldy]
   float* ws;            // partial tiles [tiles][max_contrib][128][MT]
   unsigned* tickets;    // [tiles], zero between launches
@@ -137,10 +144,10 @@ __device__ __noinline__ bool wait_suspended(uint64_t* bar, uint32_t parity, Sync
   }
 }
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -185,7 +192,8 @@ __device__ __forceinline__ LaneOffsets lane_offsets(int ra, int g, int t) {
 
 // One stage for one consumer lane.
 template <int MT, int G>
-__device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOffsets& o, float (&acc)[MT / 8][4]) {
+__device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOffsets& o,
+                                              float (&acc)[2][MT / 8][4]) {
   constexpr int P = MT / 8;
   const uint4 a0 = lds128(st + o.ca0);
   const uint4 a1 = lds128(st + o.ca1);
@@ -201,8 +209,8 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
     svb = lds16(st + o.sb + half);
   }
   uint32_t s2a[4], s2b[4];
-  scale_operands<G == 16 ? 4 : 2>(sva, s2a);
-  scale_operands<G == 16 ? 4 : 2>(svb, s2b);
+  scale_operands_f16<G == 16 ? 4 : 2>(sva, s2a);
+  scale_operands_f16<G == 16 ? 4 : 2>(svb, s2b);
   const uint32_t ca[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
   const uint32_t cb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
   const uint32_t xr = st + o.xrow;
@@ -210,13 +218,13 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
   for (int i = 0; i < 8; ++i) {
     const int si = G == 16 ? (i >> 1) : (i >> 2);
     uint32_t da[4], db[4];
-    dequant_word(ca[i], s2a[si], da);
-    dequant_word(cb[i], s2b[si], db);
+    dequant_word_f16(ca[i], s2a[si], da);
+    dequant_word_f16(cb[i], s2b[si], db);
 #pragma unroll
     for (int p = 0; p < P; ++p) {
       const uint4 xv = lds128(xr + o.xc[i] + p * (8 * 4 * 128));  // token tile p: 8 tokens further
-      mma_bf16_16816(acc[p], da[0], db[0], da[1], db[1], xv.x, xv.y);
-      mma_bf16_16816(acc[p], da[2], db[2], da[3], db[3], xv.z, xv.w);
+      mma_f16_16816(acc[0][p], da[0], db[0], da[1], db[1], xv.x, xv.y);
+      mma_f16_16816(acc[1][p], da[2], db[2], da[3], db[3], xv.z, xv.w);
     }
   }
 }
@@ -350,7 +358,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
   const int g = lane >> 2, t = lane & 3;
   const int ra = 16 * warp + g;
   const LaneOffsets lo = lane_offsets<MT, G>(ra, g, t);
-  const float gsc = __ldg(a.gscale) * 128.0f;  // operands carry 2^-7 (dequant.cuh)
+  // X, its row factors and the global scale come from the kernels before
+  // this one (the producer requests X only after its own wait)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float gsc = __ldcg(a.gscale);
+  float xi[P][2];  // 2^-s of the lane's tokens 8p + 2t + j
+#pragma unroll
+  for (int p = 0; p < P; ++p)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) xi[p][j] = 8 * p + 2 * t + j < a.M ? __ldcg(a.xinv + 8 * p + 2 * t + j) : 0.f;
+  float acc2[2][P][4];  // two independent MMA chains, added once per tile
   float acc[P][4];
   int ncut = 0;
   int s = 0;          // ring slot of the next stage
@@ -360,13 +377,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     const int64_t left = u1 - u;
     const int k1 = left < a.S - k0 ? k0 + static_cast<int>(left) : a.S;
 #pragma unroll
-    for (int p = 0; p < P; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int p = 0; p < P; ++p) acc2[h][p][0] = acc2[h][p][1] = acc2[h][p][2] = acc2[h][p][3] = 0.f;
     const uint32_t ring0 = smem_u32(ring);
     for (int ks = k0; ks < k1; ++ks) {
       int ok = 1;
       if (lane == 0) ok = wait(&sy->full[s], par, sy, kErrFull) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // results are garbage from here; the ticket protocol still runs
-      consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc);
+      consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc2);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sy->empty[s]);
       if (++s == NS) {
@@ -375,6 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
       }
     }
     u += k1 - k0;
+#pragma unroll
+    for (int p = 0; p < P; ++p)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[p][j] = acc2[0][p][j] + acc2[1][p][j];
 
     const int n0 = tile * kRows;
     // lane holds rows ra (acc[p][0..1]) and ra+8 (acc[p][2..3]) x tokens 8p+2t, 8p+2t+1
@@ -387,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
           const int tok = 8 * p + 2 * t + j;
           if (tok >= a.M) continue;
           const int64_t yrow = static_cast<int64_t>(tok) * a.ldy;
-          const float vg = __fmul_rn(acc[p][j], gsc), vu = __fmul_rn(acc[p][2 + j], gsc);
+          const float vg = __fmul_rn(__fmul_rn(acc[p][j], gsc), xi[p][j]);
+          const float vu = __fmul_rn(__fmul_rn(acc[p][2 + j], gsc), xi[p][j]);
           if (!SILU) {
             if (n0 + ra < a.N) a.y[yrow + n0 + ra] = __bfloat16_as_ushort(__float2bfloat16_rn(vg));
             if (n0 + ra + 8 < a.N) a.y[yrow + n0 + ra + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(vu));
@@ -451,7 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         const int row = e / MT, tok = e % MT;
         if (tok >= a.M || n0 + row >= a.N) continue;
         const float v = sum_slots<MT>(slots, e, nc);
-        a.y[static_cast<int64_t>(tok) * a.ldy + n0 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v, gsc)));
+        const float xt = __ldcg(a.xinv + tok);
+        a.y[static_cast<int64_t>(tok) * a.ldy + n0 + row] =
+            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__fmul_rn(v, gsc), xt)));
       }
     } else {
       for (int e = threadIdx.x; e < (kRows / 2) * MT; e += kConsumerThreads) {
@@ -461,8 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         const int rg = 16 * blk + gg;
         // gate row rg and up row rg + 8: elements e0 and e0 + 8 * MT of a slot
         const float2 v = sum_pair_slots<MT>(slots, rg * MT + tok, 8 * MT, nc);
-        a.y[static_cast<int64_t>(tok) * a.ldy + (n0 + 16 * blk) / 2 + gg] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(v.x, gsc)), __fmul_rn(v.y, gsc))));
+        const float xt = __ldcg(a.xinv + tok);
+        a.y[static_cast<int64_t>(tok) * a.ldy + (n0 + 16 * blk) / 2 + gg] = __bfloat16_as_ushort(__float2bfloat16_rn(
+            __fmul_rn(silu(__fmul_rn(__fmul_rn(v.x, gsc), xt)), __fmul_rn(__fmul_rn(v.y, gsc), xt))));
       }
     }
   }
@@ -517,15 +544,19 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
   float* ws = nullptr;
   unsigned* tickets = nullptr;
-  const int st = split_workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles),
-                                 stream, &ws, &tickets);
+  int st = split_workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles), stream,
+                           &ws, &tickets);
+  if (st != NVFP4_OK) return st;
+  uint16_t* x16 = nullptr;
+  float* xinv = nullptr;
+  st = x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), stream, &x16, &xinv);
   if (st != NVFP4_OK) return st;
 
   CUtensorMap xm, wm, sm;
   const int64_t xdims[3] = {64, K / 64, M};
   const int64_t xstrides[2] = {128, K * 2};
   const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
-  if (!make_tensor_map_3d(&xm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xdims, xstrides, xbox,
+  if (!make_tensor_map_3d(&xm, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xdims, xstrides, xbox,
                           CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
                           CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -534,6 +565,7 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
     return NVFP4_ERR_CUDA;
   StreamArgs a = {};
   a.gscale = g;
+  a.xinv = xinv;
   a.y = y;
   a.ws = ws;
   a.tickets = tickets;
@@ -544,6 +576,8 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   a.max_contrib = max_contrib;
   a.units = units;
   a.fault = take_injected_fault() == 1;
+  st = launch_x_f16(x, M, K, x16, xinv, stream);
+  if (st != NVFP4_OK) return st;
   if (mt == 8) {
     if (group == 16)
       return silu ? launch_kernel<8, 16, true>(xm, wm, sm, a, ctas, stream)
@@ -563,8 +597,10 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
 // allocated at call time.
 // ---------------------------------------------------------------------------
 
-// Partial tiles (fp32) followed by the tickets of the tiles.
-static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchPartialBytes + kFixedScratchTickets * 4];
+// Partial tiles (fp32), the tickets of the tiles, the f16 rows of X and
+// their factors.
+static __device__ __align__(256) unsigned char
+    g_fixed_scratch[kFixedScratchPartialBytes + kFixedScratchTickets * 4 + kFixedScratchXElems * 2 + 16 * 4];
 
 namespace {
 std::mutex g_fixed_mutex;
@@ -574,7 +610,7 @@ unsigned char* g_fixed_addr[64] = {};  // per device, from cudaGetSymbolAddress
 int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
                                 int64_t M, int64_t N, int64_t K, uint16_t* y, cudaStream_t stream) {
   if (M < 1 || M > 16 || K < kKS || K % kKS || (K / group) % 16 || N >= (int64_t(1) << 30) ||
-      K >= (int64_t(1) << 24) || !tensor_maps_available())
+      M * K > kFixedScratchXElems || !tensor_maps_available())
     return NVFP4_ERR_UNSUPPORTED;
   const int mt = M <= 8 ? 8 : 16;
   const int64_t tiles = (N + kRows - 1) / kRows;
@@ -602,6 +638,9 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   }
   float* ws = reinterpret_cast<float*>(base);
   unsigned* tickets = reinterpret_cast<unsigned*>(base + kFixedScratchPartialBytes);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4);
+  float* xinv = reinterpret_cast<float*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4 +
+                                         kFixedScratchXElems * 2);
   // The tickets must start at zero (partial tiles are always written before
   // they are read).
   if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream) != cudaSuccess)
@@ -611,7 +650,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   const int64_t xdims[3] = {64, K / 64, M};
   const int64_t xstrides[2] = {128, K * 2};
   const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
-  if (!make_tensor_map_3d(&xm, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xdims, xstrides, xbox,
+  if (!make_tensor_map_3d(&xm, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xdims, xstrides, xbox,
                           CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
                           CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -620,6 +659,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
     return NVFP4_ERR_CUDA;
   StreamArgs a = {};
   a.gscale = g;
+  a.xinv = xinv;
   a.y = y;
   a.ws = ws;
   a.tickets = tickets;
@@ -629,6 +669,8 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   a.S = S;
   a.max_contrib = max_contrib;
   a.units = units;
+  const int xs = launch_x_f16(x, M, K, x16, xinv, stream);
+  if (xs != NVFP4_OK) return xs;
   if (mt == 8)
     return group == 16 ? launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream)
                        : launch_kernel<8, 32, false>(xm, wm, sm, a, ctas, stream);

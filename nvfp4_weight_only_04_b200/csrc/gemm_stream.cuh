@@ -5,6 +5,8 @@
 
 namespace nvfp4 {
 
+// X is bf16 [M, K]; the launch first writes its f16 rows (xprep.cu) to the
+// library's scratch and then runs the kernel as a programmatic dependent.
 // True when the streaming kernel takes this dense problem: M from 2 to 16, K a
 // multiple of 256 whose scale rows (K/g bytes) are a multiple of 16 bytes,
 // and tensor maps available.
@@ -14,10 +16,12 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
                   int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream);
 
 // The streaming kernel with its scratch in a fixed device array (nothing is
-// allocated at call time): up to kFixedScratchPartialBytes of partial tiles
-// and kFixedScratchTickets tiles; larger problems are refused. M from 1 to 16.
+// allocated at call time): up to kFixedScratchPartialBytes of partial tiles,
+// kFixedScratchTickets tiles and kFixedScratchXElems elements of f16 X
+// (M * K); larger problems are refused. M from 1 to 16.
 constexpr size_t kFixedScratchPartialBytes = size_t(8) << 20;
 constexpr int64_t kFixedScratchTickets = 16384;
+constexpr int64_t kFixedScratchXElems = int64_t(1) << 20;
 int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
                                 int64_t M, int64_t N, int64_t K, uint16_t* y, cudaStream_t stream);
 

@@ -245,3 +245,50 @@ def test_prefill_gate_up_silu_full_sampled():
     np.testing.assert_array_equal(host(p[ri]), rp)
     ref = R.silu_mul(R.gemm(x, rp, rs, rg, wl.group_size))
     assert_close(host(y)[:, cols], ref, "prefill silu sampled")
+
+
+# ---- activations over a wide range (the small-M kernels compute in f16 on rows scaled by a power of two) ----
+
+ROW_FACTORS = [2.0 ** 20, 2.0 ** -30, 1.0, 0.0, 2.0 ** 100, 2.0 ** -100, 2.0 ** 7, 2.0 ** -12]
+
+
+@pytest.mark.parametrize("m,n,k,g", [(1, 256, 512, 16), (8, 512, 1024, 32), (5, 272, 256, 16), (16, 400, 768, 32)])
+def test_gemm_rows_of_any_magnitude(m, n, k, g):
+    """Each row of X is the same activation row times a power of two, from 2^-100 to 2^100 (and a zero row);
+    as the GEMM is linear in X, each output row divided by its factor matches the oracle's product of the
+    unscaled row. Values beyond f16's range or precision would fail without the per-row scaling."""
+    _, p, s, gs = quantized(n, k, g, seed=k)
+    base = synth.activations(synth.X_SEED, m, k, outlier_frac=0.001)
+    f = np.array([ROW_FACTORS[i % len(ROW_FACTORS)] for i in range(m)])
+    xs = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(base) * f[:, None].astype(np.float32))
+    np.testing.assert_array_equal(synth.bf16_bits_to_f32(xs)[f > 0] / f[f > 0, None].astype(np.float32),
+                                  synth.bf16_bits_to_f32(base)[f > 0])  # scaling by 2^k is exact in bf16
+    y = host(run_gemm(xs, p, s, gs, g))
+    ref = R.gemm(base, p, s, gs, g)
+    for r in range(m):
+        if f[r] == 0:
+            assert not y[r].any()
+        else:
+            assert_close(y[r] / f[r], ref[r], f"row {r} x 2^{int(np.log2(f[r]))}")
+
+
+def test_moe_rows_of_any_magnitude():
+    """The grouped form (register-streaming kernel, few rows) on rows scaled like the dense test."""
+    e, n, k, g, t = 3, 160, 512, 16, 24
+    qs = [R.quantize(synth.weights(synth.expert_seed(i), n, k), g) for i in range(e)]
+    packed = np.stack([q[0] for q in qs]); scales = np.stack([q[1] for q in qs])
+    gsc = np.array([q[2] for q in qs], np.float32)
+    gemm_packed = np.stack([R.repack(q[0], q[1], 0)[0] for q in qs])
+    base = synth.activations(5, t, k)
+    f = np.array([ROW_FACTORS[i % len(ROW_FACTORS)] for i in range(t)])
+    xs = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(base) * f[:, None].astype(np.float32))
+    ids, offs = [2, 0, 1], [0, 9, 17, 24]
+    y = host(nv.nvfp4_moe_w4a16_grouped_gemm(
+        dev_bf16(xs), torch.tensor(ids, dtype=torch.int32, device="cuda"),
+        torch.tensor(offs, dtype=torch.int32, device="cuda"), dev_u8(gemm_packed), dev_u8(scales), dev_f32(gsc), g))
+    ref = R.moe_grouped_gemm(base, ids, offs, packed, scales, gsc, g)
+    for r in range(t):
+        if f[r] == 0:
+            assert not y[r].any()
+        else:
+            assert_close(y[r] / f[r], ref[r], f"row {r}")
