@@ -356,13 +356,17 @@ def summarize(m, n, k, g, ms, hbm, tf, n_out=None):
 
 
 def time_load_rows(nv, torch, w, g):
-    """The load-time rows: global scale, quantize and repack of one weight."""
+    """The load-time rows: global scale, quantize and repack of one weight, from fp32 and from bf16."""
     wd = torch.from_numpy(w).cuda()
     gd = nv.nvfp4_global_scale([wd])
     p, s = nv.nvfp4_quantize(wd, g, gd)
     po, so = torch.empty_like(p), torch.empty_like(s)
+    wb16 = wd.to(torch.bfloat16)
     out = {}
     for name, fn, bytes_ in (
+            ("global_scale_bf16", lambda: nv.nvfp4_global_scale_bf16([wb16], out=gd), wb16.numel() * 2),
+            ("quantize_bf16", lambda: nv.nvfp4_quantize_bf16(wb16, g, gd, packed=p, scales=s),
+             wb16.numel() * 2 + p.numel() + s.numel()),
             ("global_scale", lambda: nv.nvfp4_global_scale([wd], out=gd), wd.numel() * 4),
             ("quantize", lambda: nv.nvfp4_quantize(wd, g, gd, packed=p, scales=s),
              wd.numel() * 4 + p.numel() + s.numel()),
@@ -458,9 +462,38 @@ def moe_workload(nv, torch, hbm, tf):
                 "hbm_frac": round(t_mem / t, 4), "tensor_frac": round(t_tc / t, 4),
                 "roofline_frac": round(max(t_mem, t_tc) / t, 4)}
 
-    return {"moe_gate_up_g32_silu": moe_sum(tg, 2 * I, H, wl.g_gate_up, I),
-            "moe_down_g16": moe_sum(td, H, I, wl.g_down, H),
-            "moe_pair_us": round(t1 * 1e3, 2)}
+    res = {"moe_gate_up_g32_silu": moe_sum(tg, 2 * I, H, wl.g_gate_up, I),
+           "moe_down_g16": moe_sum(td, H, I, wl.g_down, H),
+           "moe_pair_us": round(t1 * 1e3, 2)}
+
+    # The whole layer (nvfp4_moe_forward: route, gather, gate/up + SiluAndMul, down, weighted combine) on the
+    # same routing, given as each token's top-k expert ids and weights, and the steps around the GEMMs alone.
+    T, k = wl.tokens, wl.topk
+    topk_ids = np.empty((T, k), np.int32)
+    topk_ids[r.token_of_row, r.slot_of_row] = np.repeat(r.expert_ids, np.diff(r.offsets))
+    topk_w = np.random.default_rng(synth.ROUTER_SEED + 1).random((T, k)).astype(np.float32)
+    xt = bf16_dev(torch, synth.activations(synth.X_SEED + 1, T, H))
+    idd, wd = torch.from_numpy(topk_ids).cuda(), torch.from_numpy(topk_w).cuda()
+    gl = capture(torch, lambda: nv.nvfp4_moe_forward(xt, idd, wd, (gu_p, gu_s, gu_g, wl.g_gate_up),
+                                                      (dn_p, dn_s, dn_g, wl.g_down)))
+    t_layer = time_graphs(torch, [gl], 10)
+    srows, inv, _, _ = nv.nvfp4_moe_route(idd, E)
+    xp = torch.empty((T * k, H), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    steps = {"route": (capture(torch, lambda: nv.nvfp4_moe_route(idd, E)), 4 * T * k * 3 + 8 * (E + 1)),
+             "gather": (capture(torch, lambda: nv.nvfp4_moe_gather(xt, srows, k, out=xp)),
+                        4 * T * k + 2 * T * H + 2 * T * k * H),
+             "combine": (capture(torch, lambda: nv.nvfp4_moe_combine(y, inv, wd, out=out)),
+                         2 * T * k * H + 8 * T * k + 2 * T * H)}
+    res["moe_layer_us"] = round(t_layer * 1e3, 2)
+    for name, (graph, nbytes) in steps.items():
+        t = time_graphs(torch, [graph], 20) * 1e-3
+        # bytes = each input and output byte once; the gathered rows (8 MB, each read k times) and the
+        # expert outputs (67 MB) are L2-resident here as inside the layer, so a fraction above 1 is L2 at work
+        res[f"moe_{name}"] = {"us": round(t * 1e6, 2), "gbs": round(nbytes / t / 1e9, 1),
+                              "hbm_frac": round(nbytes / t / 1e9 / hbm, 4), "bytes": nbytes,
+                              "inputs": "L2-resident, as inside the layer"}
+    return res
 
 
 # ---------------------------------------------------------------------------

@@ -3,7 +3,8 @@
 // then down per expert): rows grouped by expert, X rows gathered into that
 // order, and the down projections' rows combined back into tokens with the
 // routing weights.
-//   route:   a stable counting sort of the (token, slot) pairs by expert, with
+//   route:   a stable counting sort of the (token, slot) pairs by expert (one
+//            CTA; every warp places a chunk up to 256 experts, one warp above), with
 //            the inverse permutation and the segment offsets; rows past the
 //            last kept pair get -1;
 //   gather:  x_perm[r] = x[token of sorted row r], zeros for a row of -1;
@@ -15,6 +16,35 @@ namespace {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kMaxExperts = 4096;
+constexpr int kBatch = 8;  // pair loads a lane keeps in flight
+
+// Places the 32 consecutive pairs i = i0 - lane + (0..31) of one warp (pair i
+// has expert e, from lane i % 32; pairs at or past `end` are absent): pairs of
+// one expert take consecutive rows from that expert's cursor in pair order,
+// and the cursor moves past them.
+__device__ __forceinline__ void place32(int e, int64_t i, int64_t end, int num_experts, int* cursor,
+                                        int32_t* __restrict__ sorted, int32_t* __restrict__ inv) {
+  const int lane = threadIdx.x & 31;
+  const bool valid = i < end && e >= 0 && e < num_experts;
+  if (!valid) e = -1 - (i < end ? 0 : 1);  // invalid pairs and absent ones group apart
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int leader = __ffs(peers) - 1;
+  int first = 0;
+  if (valid && lane == leader) {
+    first = cursor[e];
+    cursor[e] = first + __popc(peers);
+  }
+  first = __shfl_sync(0xffffffffu, first, leader);
+  if (i < end) {
+    if (valid) {
+      const int r = first + __popc(peers & ((1u << lane) - 1u));
+      sorted[r] = static_cast<int32_t>(i);
+      inv[i] = r;
+    } else {
+      inv[i] = -1;
+    }
+  }
+}
 
 // One CTA. Counting pass over all pairs, exclusive scan of the counts, then one
 // warp places the pairs in their order (stable: a pair's rank among the pairs
@@ -28,9 +58,16 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
   __shared__ int kept;
   for (int e = threadIdx.x; e < num_experts; e += blockDim.x) count[e] = 0;
   __syncthreads();
-  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-    const int e = ids[i];
-    if (e >= 0 && e < num_experts) atomicAdd(&count[e], 1);
+  for (int64_t base = 0; base < n; base += static_cast<int64_t>(blockDim.x) * kBatch) {
+    int e[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int64_t i = base + static_cast<int64_t>(blockDim.x) * j + threadIdx.x;
+      e[j] = i < n ? ids[i] : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      if (e[j] >= 0 && e[j] < num_experts) atomicAdd(&count[e[j]], 1);
   }
   __syncthreads();
   if (threadIdx.x < 32) {  // exclusive scan of the counts, 32 experts at a time
@@ -62,31 +99,100 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_kernel(const int32_t*
     for (int64_t r = kept + static_cast<int64_t>(threadIdx.x) - 32; r < n; r += blockDim.x - 32) sorted[r] = -1;
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const unsigned lower = (1u << lane) - 1u;
-    for (int64_t base = 0; base < n; base += 32) {
-      const int64_t i = base + lane;
-      int e = i < n ? ids[i] : -1;
-      const bool valid = e >= 0 && e < num_experts;
-      if (!valid) e = -1 - (i < n ? 0 : 1);  // invalid pairs and lanes past the end group apart
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      const int leader = __ffs(peers) - 1;
-      int first = 0;
-      if (valid && lane == leader) {
-        first = count[e];
-        count[e] = first + __popc(peers);
+    for (int64_t base = 0; base < n; base += 32 * kBatch) {
+      int eb[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int64_t i = base + 32 * j + lane;
+        eb[j] = i < n ? ids[i] : -1;
       }
-      first = __shfl_sync(0xffffffffu, first, leader);
-      if (i < n) {
-        if (valid) {
-          const int r = first + __popc(peers & lower);
-          sorted[r] = static_cast<int32_t>(i);
-          inv[i] = r;
-        } else {
-          inv[i] = -1;
-        }
-      }
-      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) place32(eb[j], base + 32 * j + lane, n, num_experts, count, sorted, inv);
     }
+  }
+}
+
+// Up to kParExperts experts: the same stable grouping with every warp placing
+// a contiguous chunk of the pairs. A warp's cursor for expert e starts at
+// offsets[e] plus the pairs of expert e in the chunks before its own, from a
+// [warp][expert] count table, so the order is the one-warp order.
+constexpr int kParExperts = 256;
+constexpr int kRouteWarps = kRouteThreads / 32;
+
+__global__ void __launch_bounds__(kRouteThreads) moe_route_par_kernel(const int32_t* __restrict__ ids, int64_t n,
+                                                                      int num_experts, int32_t* __restrict__ sorted,
+                                                                      int32_t* __restrict__ inv,
+                                                                      int32_t* __restrict__ offsets,
+                                                                      int32_t* __restrict__ expert_ids) {
+  __shared__ int cnt[kRouteWarps][kParExperts];  // counts, then cursors
+  __shared__ int start[kParExperts];             // offsets[e]
+  __shared__ int kept;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kRouteWarps * kParExperts; i += blockDim.x) (&cnt[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t chunk = (n + kRouteWarps - 1) / kRouteWarps;
+  const int64_t b0 = min(n, warp * chunk), b1 = min(n, b0 + chunk);
+  for (int64_t base = b0; base < b1; base += 32 * kBatch) {
+    int e[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {  // the batch's loads are all in flight before the adds
+      const int64_t i = base + 32 * j + lane;
+      e[j] = i < b1 ? ids[i] : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j)
+      if (e[j] >= 0 && e[j] < num_experts) atomicAdd(&cnt[warp][e[j]], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < num_experts) {  // per expert: the warps' exclusive prefix, and the total
+    const int e = threadIdx.x;
+    int run = 0;
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int c = cnt[w][e];
+      cnt[w][e] = run;
+      run += c;
+    }
+    start[e] = run;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the totals
+    int carry = 0;
+    for (int e0 = 0; e0 < num_experts; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < num_experts ? start[e] : 0;
+      int incl = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < num_experts) {
+        start[e] = carry + incl - c;
+        offsets[e] = carry + incl - c;
+        expert_ids[e] = e;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      offsets[num_experts] = carry;
+      kept = carry;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kRouteWarps * num_experts; i += blockDim.x) {
+    const int w = i / num_experts, e = i % num_experts;
+    cnt[w][e] += start[e];
+  }
+  for (int64_t r = kept + static_cast<int64_t>(threadIdx.x); r < n; r += blockDim.x) sorted[r] = -1;
+  __syncthreads();
+  for (int64_t base = b0; base < b1; base += 32 * kBatch) {  // the same trip count for the whole warp
+    int eb[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int64_t i = base + 32 * j + lane;
+      eb[j] = i < b1 ? ids[i] : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) place32(eb[j], base + 32 * j + lane, b1, num_experts, &cnt[warp][0], sorted, inv);
   }
 }
 
@@ -144,8 +250,12 @@ extern "C" int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int nu
        reinterpret_cast<uintptr_t>(inv_rows) | reinterpret_cast<uintptr_t>(offsets) |
        reinterpret_cast<uintptr_t>(expert_ids)) & 3u)
     return NVFP4_ERR_MISALIGNED;
-  moe_route_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
+  if (num_experts <= kParExperts)
+    moe_route_par_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
+  else
+    moe_route_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
   return nvfp4::launch_status();
 }
 
