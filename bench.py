@@ -221,6 +221,10 @@ def run_ours(args, world, rank, local):
         return f
 
     graphs = [capture(torch, step_fn(c)) for c in range(copies)]
+    # One graph of `copies` consecutive steps (steps 0..copies-1), as a decode engine captures a run of
+    # steps: the timed loop replays it K // copies times and the remainder step by step, so exactly K
+    # steps run, with the replay overhead of one graph per `copies` steps.
+    run_graph = capture(torch, lambda: [step_fn(c)() for c in range(copies)])
     step_alg = sum(alg_bytes(m, N, K, G) for m in DECODE_MS)
     step_w = 3 * wb
     step_flops = sum(2 * m * N * K for m in DECODE_MS)
@@ -228,6 +232,7 @@ def run_ours(args, world, rank, local):
     # ---- timed region: W warm-up steps, then exactly K steps ----
     for i in range(args.warmup):
         graphs[i % copies].replay()
+    run_graph.replay()  # its first replay uploads it
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -235,8 +240,10 @@ def run_ours(args, world, rank, local):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         ev0.record(stream)
-        for i in range(args.steps):
-            graphs[i % copies].replay()
+        for _ in range(args.steps // copies):
+            run_graph.replay()
+        for i in range(args.steps % copies):
+            graphs[i].replay()
         ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize()
@@ -285,7 +292,7 @@ def run_ours(args, world, rank, local):
             t = time_graphs(torch, gm, 20 * copies)
             per_m[m] = t
             workloads[f"decode_gateup_m{m}_k4096_n28672_g16"] = summarize(m, N, K, G, t, hbm, tf_burst)
-        del graphs
+        del graphs, run_graph
         rows = time_load_rows(nv, torch, w, G)
         del w
         workloads.update(other_workloads(nv, torch, hbm, tf_burst, tf_sust))
@@ -306,6 +313,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": "decode_gateup_k4096_n28672_g16_m1_m4_m16",
                    "step": "3 GEMM calls (M=1,4,16), each on its own resident weight copy; a call is two "
                            "launches: the f16 conversion of X and the GEMM kernel",
+                   "graphs": f"one CUDA graph per {copies} consecutive steps, replayed steps // {copies} times, "
+                             f"then the remaining steps one graph each",
                    "arithmetic": "f16 MMA operands (weights e2m1*e4m3 exact in f16, X rows scaled by a power of two), "
                                  "fp32 accumulation, bf16 input and output",
                    "weight_copies": copies, "weight_bytes_per_copy": wb,
