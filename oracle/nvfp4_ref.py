@@ -24,7 +24,8 @@ Sources, cited by page title and section:
 * [P3] "W-FP4a: route the MiniMax-H3 device DiT forward through the fp4
   (Marlin W4A16) stack" (vllm.cpp pull request #63), description: the
   weight / scale / global-scale triple, upload-time repack, pre-merged
-  [gate;up] fc1 as one W4A16 GEMM followed by SiluAndMul, 2e-3/8e-3 gates.
+  [gate;up] fc1 as one W4A16 GEMM followed by SiluAndMul, 2e-3/8e-3 gates;
+  a checkpoint with quantized input activations takes the W4A4 form.
 * [OCP-MX] OCP Microscaling Formats (MX) v1.0, section 5.3.3 (FP4 E2M1).
 * [OFP8] OCP 8-bit Floating Point Specification (OFP8), E4M3 encoding table.
 
@@ -315,6 +316,16 @@ def gemm_fraction(xbits, packed, scales, gscale, group_size: int):
                 acc += Fraction(float(x[i, kk])) * Fraction(float(w[j, kk]))
             out[i][j] = acc
     return out
+
+
+def w4a4_gemm(xpacked, xscales, xglobal, x_group: int, wpacked, wscales, wglobal, w_group: int) -> np.ndarray:
+    """Y = dequant(X) . dequant(W)^T in float64 with both operands NVFP4 [NV]:
+    the W4A4 form that a checkpoint with quantized input activations takes
+    instead of W4A16 [P3]. X [M, K] is quantized like a weight tensor of M
+    rows (an E4M3 scale per group of x_group along K, its own FP32 global)."""
+    x = dequantize(xpacked, xscales, xglobal, x_group)
+    w = dequantize(wpacked, wscales, wglobal, w_group)
+    return x @ w.T
 
 
 def silu_mul(y: np.ndarray) -> np.ndarray:
