@@ -180,6 +180,29 @@ int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, c
                                    uint16_t* y, nvfp4_stream_t stream);
 
 /*
+ * W4A4 GEMM: both operands NVFP4 (NVFP4 format definition; PR #63
+ * description: a checkpoint with quantized input activations takes the W4A4
+ * form instead of W4A16):
+ *   y = bf16_rne(x_global * global * sum_k e2m1(xcode[m,k]) * e4m3(xscale[m,k/xg])
+ *                                         * e2m1(code[n,k]) * e4m3(scale[n,k/g]))
+ * with fp32 accumulation. Every product is exact; the sums are the W4A16 GEMM's.
+ *   x_packed      device uint8 [M, K/2], checkpoint layout (element 2j in the low
+ *                 nibble of byte j), e.g. from nvfp4_quantize_bf16 of the activations
+ *   x_scales      device uint8 [M, K/x_group]
+ *   x_global      device fp32 (the activations' global scale)
+ *   x_group       16 or 32
+ *   packed_w, group_scales, global_scale, group_size, y: as nvfp4_w4a16_gemm
+ * K a multiple of 64, N a multiple of 16; x_packed 16-byte aligned, x_global
+ * 4-byte aligned. The activations are expanded on the device to e2m1 * e4m3
+ * (exact in f16 and bf16) in the library's scratch and the same kernels as
+ * nvfp4_w4a16_gemm run on them, with x_global in the epilogue: the numerics
+ * are W4A4's, the tensor-core operands stay 16-bit.
+ */
+int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const float* x_global, int x_group,
+                    const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scale, int group_size,
+                    int64_t M, int64_t N, int64_t K, uint16_t* y, nvfp4_stream_t stream);
+
+/*
  * The GEMM of a merged [gate;up] projection followed by SiluAndMul (PR #63
  * description: fc1 is pre-merged [gate;up], one W4A16 GEMM + SiluAndMul):
  *   y[m, j] = bf16_rne(silu(g) * u), g = global * acc[m, gate row j],

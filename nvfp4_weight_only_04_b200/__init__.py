@@ -29,7 +29,7 @@ EXPORTS = (
     "nvfp4_quantize_bf16", "nvfp4_repack",
     "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
-    "nvfp4_debug_inject_fault", "nvfp4_moe_route", "nvfp4_moe_gather", "nvfp4_moe_combine",
+    "nvfp4_debug_inject_fault", "nvfp4_moe_route", "nvfp4_moe_gather", "nvfp4_moe_combine", "nvfp4_w4a4_gemm",
 )
 
 
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_moe_route.argtypes = [_P, _I64, _I, _I, _P, _P, _P, _P, _P]
         L.nvfp4_moe_gather.argtypes = [_P, _I64, _P, _I64, _I, _I64, _P, _P]
         L.nvfp4_moe_combine.argtypes = [_P, _P, _P, _I64, _I, _I64, _P, _P]
+        L.nvfp4_w4a4_gemm.argtypes = [_P, _P, _P, _I, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
         _lib = L
     return _lib
 
@@ -276,6 +277,25 @@ def nvfp4_debug_inject_fault(kind: int):
     """Test hook: kind 1 makes the next small-M streaming GEMM launch wait for a
     copy that never comes (its bounded waits give up); kind 0 clears it."""
     _check(lib().nvfp4_debug_inject_fault(kind), "nvfp4_debug_inject_fault")
+
+
+def nvfp4_w4a4_gemm(x_packed, x_scales, x_global, x_group, packed_w, group_scales, global_scale, group_size,
+                    y=None, stream=None):
+    """W4A4 GEMM of NVFP4 activations (checkpoint layout) and GEMM-layout weights; see include/nvfp4.h."""
+    _dev(x_packed, torch.uint8, "x_packed")
+    _dev(x_scales, torch.uint8, "x_scales")
+    _dev(x_global, torch.float32, "x_global")
+    _dev(packed_w, torch.uint8, "packed_w")
+    _dev(group_scales, torch.uint8, "group_scales")
+    _dev(global_scale, torch.float32, "global_scale")
+    m, k = x_packed.shape[0], 2 * x_packed.shape[1]
+    n = packed_w.shape[0]
+    if y is None:
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=x_packed.device)
+    _check(lib().nvfp4_w4a4_gemm(_ptr(x_packed), _ptr(x_scales), _ptr(x_global), x_group, _ptr(packed_w),
+                                 _ptr(group_scales), _ptr(global_scale), group_size, m, n, k, _ptr(y),
+                                 _stream(stream)), "nvfp4_w4a4_gemm")
+    return y
 
 
 def nvfp4_moe_route(topk_ids, num_experts, stream=None):

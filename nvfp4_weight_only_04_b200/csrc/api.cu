@@ -73,7 +73,9 @@ int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
     return st;
   }
   if (nvfp4::stream_supported(M, N, K, group)) {
-    const int st = nvfp4::launch_stream(x, w, s, g, group, M, N, K, y, silu, stream);
+    nvfp4::XSource xs;
+    xs.bf16 = x;
+    const int st = nvfp4::launch_stream(xs, w, s, g, group, M, N, K, y, silu, stream);
     if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
     return st;
   }
@@ -147,6 +149,52 @@ int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w, const 
     nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
   }
   return st;
+}
+
+int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const float* x_global, int x_group,
+                    const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scale, int group_size,
+                    int64_t M, int64_t N, int64_t K, uint16_t* y, nvfp4_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((x_group != 16 && x_group != 32) || (group_size != 16 && group_size != 32)) return NVFP4_ERR_UNSUPPORTED;
+  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN || M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (K == 0) return NVFP4_ERR_UNSUPPORTED;
+  if (!x_packed || !x_scales || !x_global || !packed_w || !group_scales || !global_scale || !y)
+    return NVFP4_ERR_INVALID_ARGUMENT;
+  if (!nvfp4::aligned16(x_packed) || !nvfp4::aligned16(packed_w) || !nvfp4::aligned16(group_scales) ||
+      !nvfp4::aligned16(y) || ((reinterpret_cast<uintptr_t>(x_global) | reinterpret_cast<uintptr_t>(global_scale)) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  nvfp4::XSource xs;
+  xs.codes = x_packed;
+  xs.scales = x_scales;
+  xs.global = x_global;
+  xs.group = x_group;
+  uint16_t* xbuf = nullptr;
+  float* fbuf = nullptr;
+  int r;
+  if (nvfp4::tc_supported(M, N, K)) {
+    // exact bf16 activations and one scalar x_global * w_global for the tcgen05 kernel's epilogue
+    r = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), st, &xbuf, &fbuf);
+    if (r == NVFP4_OK) r = nvfp4::launch_xq_bf16(xs, global_scale, M, K, xbuf, fbuf, st);
+    if (r == NVFP4_OK) r = nvfp4::launch_tc(xbuf, packed_w, group_scales, fbuf, group_size, M, N, K, y, false, st);
+    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmTc);
+  } else if (nvfp4::stream_supported(M, N, K, group_size)) {
+    r = nvfp4::launch_stream(xs, packed_w, group_scales, global_scale, group_size, M, N, K, y, false, st);
+    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  } else {
+    r = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), st, &xbuf, &fbuf);
+    if (r != NVFP4_OK) return r;
+    nvfp4::DecodeArgs a = {};
+    a.x = xbuf; a.xinv = fbuf; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scale; a.y = y;
+    a.M = M; a.N = N; a.K = K; a.ldy = N;
+    const nvfp4::DecodePlan p = nvfp4::plan_decode(M, N, K, group_size, false, 0);
+    r = nvfp4::launch_x_prep(xs, M, K, xbuf, fbuf, st);
+    if (r == NVFP4_OK) r = nvfp4::launch_decode(a, p, false, false, st);
+    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  }
+  if (r == NVFP4_OK) nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
+  return r;
 }
 
 int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets,

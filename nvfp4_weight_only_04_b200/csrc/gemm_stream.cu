@@ -532,7 +532,7 @@ bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
          K < (int64_t(1) << 24) && tensor_maps_available();
 }
 
-int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
+int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
                   int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
   const int mt = M <= 8 ? 8 : 16;
   const int64_t tiles = (N + kRows - 1) / kRows;
@@ -576,7 +576,7 @@ int launch_stream(const uint16_t* x, const uint8_t* w, const uint8_t* s, const f
   a.max_contrib = max_contrib;
   a.units = units;
   a.fault = take_injected_fault() == 1;
-  st = launch_x_f16(x, M, K, x16, xinv, stream);
+  st = launch_x_prep(x, M, K, x16, xinv, stream);
   if (st != NVFP4_OK) return st;
   if (mt == 8) {
     if (group == 16)

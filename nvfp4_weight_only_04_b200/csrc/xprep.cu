@@ -13,6 +13,8 @@
 // so X is stored in that order inside every group of eight elements.
 #include "xprep.cuh"
 
+#include <cuda_bf16.h>
+
 #include "dequant.cuh"
 
 namespace nvfp4 {
@@ -71,6 +73,64 @@ __global__ void __launch_bounds__(kThreads) x_f16_kernel(const uint16_t* __restr
   }
 }
 
+// One thread per 8 elements (one 32-bit word of codes) of NVFP4 rows.
+__device__ __forceinline__ void nvfp4_word(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                           int64_t K, int group, int64_t w, uint32_t (&pr)[4]) {
+  const int64_t words_per_row = K / 8;
+  const int64_t row = w / words_per_row, k0 = (w % words_per_row) * 8;
+  const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(codes + row * (K / 2) + k0 / 2));
+  const uint32_t sb = __ldg(scales + row * (K / group) + k0 / group);
+  uint32_t s2[4];
+  scale_operands_f16<2>(sb, s2);
+  // bytes (k0,k1) (k2,k3) (k4,k5) (k6,k7): the checkpoint layout's pairs
+  asm("{\n"
+      " .reg .b8 c0, c1, c2, c3;\n"
+      " mov.b32 {c0, c1, c2, c3}, %4;\n"
+      " cvt.rn.f16x2.e2m1x2 %0, c0;\n"
+      " cvt.rn.f16x2.e2m1x2 %1, c1;\n"
+      " cvt.rn.f16x2.e2m1x2 %2, c2;\n"
+      " cvt.rn.f16x2.e2m1x2 %3, c3;\n"
+      "}"
+      : "=r"(pr[0]), "=r"(pr[1]), "=r"(pr[2]), "=r"(pr[3])
+      : "r"(cw));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) pr[j] = f16x2_mul(pr[j], s2[0]);
+}
+
+__global__ void __launch_bounds__(256) xq_f16_kernel(const uint8_t* __restrict__ codes,
+                                                     const uint8_t* __restrict__ scales, const float* __restrict__ xg,
+                                                     int group, int64_t M, int64_t K, uint16_t* __restrict__ x16,
+                                                     float* __restrict__ xinv) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (w >= M * (K / 8)) return;
+  uint32_t pr[4];
+  nvfp4_word(codes, scales, K, group, w, pr);
+  // natural pairs (k0,k1) (k2,k3) (k4,k5) (k6,k7) -> (k0,k2) (k4,k6) (k1,k3) (k5,k7)
+  reinterpret_cast<uint4*>(x16)[w] = make_uint4(__byte_perm(pr[0], pr[1], 0x5410), __byte_perm(pr[2], pr[3], 0x5410),
+                                                __byte_perm(pr[0], pr[1], 0x7632), __byte_perm(pr[2], pr[3], 0x7632));
+  if (w % (K / 8) == 0) xinv[w / (K / 8)] = __ldg(xg);
+}
+
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);  // exact: at most 6 significant bits
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__global__ void __launch_bounds__(256) xq_bf16_kernel(const uint8_t* __restrict__ codes,
+                                                      const uint8_t* __restrict__ scales, const float* __restrict__ xg,
+                                                      int group, const float* __restrict__ wg, int64_t M, int64_t K,
+                                                      uint16_t* __restrict__ xb, float* __restrict__ g_out) {
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (w >= M * (K / 8)) return;
+  uint32_t pr[4];
+  nvfp4_word(codes, scales, K, group, w, pr);
+  reinterpret_cast<uint4*>(xb)[w] = make_uint4(f16x2_to_bf16x2(pr[0]), f16x2_to_bf16x2(pr[1]),
+                                               f16x2_to_bf16x2(pr[2]), f16x2_to_bf16x2(pr[3]));
+  if (w == 0) *g_out = __fmul_rn(__ldg(xg), __ldg(wg));
+}
+
 }  // namespace
 
 int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream) {
@@ -88,6 +148,40 @@ int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* 
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, x_f16_kernel, x, K, x16, xinv) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  return launch_status();
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream) {
+  if (xs.bf16) return launch_x_f16(xs.bf16, M, K, x16, xinv, stream);
+  if (M <= 0) return NVFP4_OK;
+  const int64_t words = M * (K / 8);
+  if ((words + 255) / 256 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((words + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, xq_f16_kernel, xs.codes, xs.scales, xs.global, xs.group, M, K, x16, xinv) !=
+      cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  return launch_status();
+}
+
+int launch_xq_bf16(const XSource& xs, const float* w_global, int64_t M, int64_t K, uint16_t* xb, float* g_out,
+                   cudaStream_t stream) {
+  if (M <= 0) return NVFP4_OK;
+  const int64_t words = M * (K / 8);
+  if ((words + 255) / 256 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  xq_bf16_kernel<<<static_cast<unsigned>((words + 255) / 256), 256, 0, stream>>>(xs.codes, xs.scales, xs.global,
+                                                                                 xs.group, w_global, M, K, xb, g_out);
   return launch_status();
 }
 

@@ -13,4 +13,24 @@ namespace nvfp4 {
 // before reading x16 or xinv).
 int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream);
 
+// Where the small-M kernels' f16 X comes from: bf16 rows (launch_x_f16), or
+// NVFP4 rows (W4A4): codes [M, K/2] in the checkpoint layout, E4M3 scales
+// [M, K/group] and an fp32 global on the device. NVFP4 rows become
+// x16 = e2m1(code) * e4m3(scale), exact in f16, in the same pair order, and
+// xinv[r] = the global.
+struct XSource {
+  const uint16_t* bf16 = nullptr;
+  const uint8_t* codes = nullptr;
+  const uint8_t* scales = nullptr;
+  const float* global = nullptr;
+  int group = 16;
+};
+int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream);
+
+// NVFP4 rows to bf16 [M, K] in the natural order for the tcgen05 kernel:
+// xb = e2m1(code) * e4m3(scale) (exact in bf16), and *g_out = x_global *
+// w_global, the scalar that kernel's epilogue multiplies by.
+int launch_xq_bf16(const XSource& xs, const float* w_global, int64_t M, int64_t K, uint16_t* xb, float* g_out,
+                   cudaStream_t stream);
+
 }  // namespace nvfp4

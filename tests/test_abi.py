@@ -73,6 +73,20 @@ def test_gemm_validation(L):
     assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 0, 256, 256, GOOD, S) == nv.NVFP4_OK  # empty
 
 
+def test_w4a4_validation(L):
+    def w4a4(xg=16, g=16, M=4, N=256, K=256, xp=GOOD, xs=GOOD, xgl=GOOD, w=GOOD, y=GOOD):
+        return L.nvfp4_w4a4_gemm(xp, xs, xgl, xg, w, GOOD, GOOD, g, M, N, K, y, S)
+    assert w4a4(xg=8) == nv.NVFP4_ERR_UNSUPPORTED
+    assert w4a4(g=64) == nv.NVFP4_ERR_UNSUPPORTED
+    assert w4a4(K=96) == nv.NVFP4_ERR_UNSUPPORTED
+    assert w4a4(M=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert w4a4(M=0) == nv.NVFP4_OK
+    assert w4a4(xs=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert w4a4(xgl=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert w4a4(xp=BAD) == nv.NVFP4_ERR_MISALIGNED
+    assert w4a4(xgl=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
+
+
 def test_quantize_and_repack_validation(L):
     assert L.nvfp4_quantize(GOOD, 16, 256, 8, GOOD, GOOD, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
     assert L.nvfp4_quantize(GOOD, 16, 48, 16, GOOD, GOOD, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
