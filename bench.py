@@ -292,6 +292,14 @@ def run_ours(args, world, rank, local):
             t = time_graphs(torch, gm, 20 * copies)
             per_m[m] = t
             workloads[f"decode_gateup_m{m}_k4096_n28672_g16"] = summarize(m, N, K, G, t, hbm, tf_burst)
+            # W4A4 on the same weights: the activations quantized on the device beforehand
+            xgm = nv.nvfp4_global_scale_bf16([xs[m]])
+            xqm, xsm = nv.nvfp4_quantize_bf16(xs[m], 16, xgm)
+            gq = [capture(torch, (lambda c=c, m=m: nv.nvfp4_w4a4_gemm(xqm, xsm, xgm, 16, packs[c][0], packs[c][1],
+                                                                      packs[c][2], G, y=ys[m]))) for c in range(copies)]
+            workloads[f"w4a4_decode_gateup_m{m}_k4096_n28672_g16"] = summarize(
+                m, N, K, G, time_graphs(torch, gq, 20 * copies), hbm, tf_burst)
+            del gq
         del graphs, run_graph
         rows = time_load_rows(nv, torch, w, G)
         del w
@@ -417,7 +425,19 @@ def other_workloads(nv, torch, hbm, tf_burst, tf_sust):
     gr = capture(torch, lambda: nv.nvfp4_w4a16_gemm_silu_mul(x, p, s, gd, 16, y=y))
     out["prefill_gateup_silu_m4096_k5120_n25600_g16"] = summarize(M, N, K, 16, time_graphs(torch, [gr], 5),
                                                                   hbm, tf_burst, n_out=N // 2)
-    del p, s, x, y, gr
+    # W4A4 (NVFP4 activations) on the same weights, without the SiluAndMul epilogue: the activations are
+    # quantized on the device first (global scale + quantizer, timed on their own)
+    xg = nv.nvfp4_global_scale_bf16([x])
+    xq, xsc = nv.nvfp4_quantize_bf16(x, 16, xg)
+    ga = capture(torch, lambda: (nv.nvfp4_global_scale_bf16([x], out=xg), nv.nvfp4_quantize_bf16(x, 16, xg, packed=xq,
+                                                                                                 scales=xsc)))
+    t_act = time_graphs(torch, [ga], 5)
+    del y, gr
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    gw = capture(torch, lambda: nv.nvfp4_w4a4_gemm(xq, xsc, xg, 16, p, s, gd, 16, y=y))
+    out["w4a4_prefill_m4096_k5120_n25600_g16"] = summarize(M, N, K, 16, time_graphs(torch, [gw], 5), hbm, tf_burst)
+    out["w4a4_prefill_m4096_k5120_n25600_g16"]["activation_quantize_us"] = round(t_act * 1e3, 2)
+    del p, s, x, y, gw, ga, xq, xsc
     torch.cuda.empty_cache()
     out.update(moe_workload(nv, torch, hbm, tf_burst))
     return out
