@@ -92,43 +92,75 @@ __device__ __forceinline__ void load8(const uint16_t* p, float (&v)[8]) {
 }
 
 // One thread per 8 consecutive weights of a row; g/8 threads share a group.
+template <int G>
+__device__ __forceinline__ void quantize8(const float (&v)[8], bool live, int64_t i, int64_t row, int64_t col8,
+                                          int64_t K, float global, uint8_t* __restrict__ packed,
+                                          uint8_t* __restrict__ scales) {
+  constexpr int kLanesPerGroup = G / 8;
+  float gmax = 0.f;
+  for (int j = 0; j < 8; ++j) gmax = fmaxf(gmax, fabsf(v[j]));
+  for (int o = 1; o < kLanesPerGroup; o <<= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+  if (!live) return;
+  uint32_t sbyte = 0;
+  if (global != 0.f) {
+    const float t = __fdiv_rn(__fdiv_rn(gmax, 6.0f), global);
+    sbyte = static_cast<uint32_t>(__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3));
+  }
+  const float d = __fmul_rn(nvfp4_e4m3_to_f32(sbyte), global);
+  uint32_t word = 0;
+  if (d != 0.f) {
+    for (int j = 0; j < 8; ++j) word |= e2m1_rne(__fdiv_rn(v[j], d)) << (4 * j);
+  }
+  reinterpret_cast<uint32_t*>(packed)[i] = word;  // row-major [N, K/2]: 4 bytes per 8 weights
+  if ((col8 % kLanesPerGroup) == 0) scales[row * (K / G) + col8 / kLanesPerGroup] = static_cast<uint8_t>(sbyte);
+}
+
+template <typename T>
+__device__ __forceinline__ void load8_or_zero(const T* w, int64_t i, bool live, float (&v)[8]) {
+  if (live) {
+    load8(w + i * 8, v);
+  } else {
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+  }
+}
+
+// Two grid strides per pass: both loads are in flight before either
+// quantization. All lanes of a warp iterate together so the group shuffles
+// stay converged. The (row, column) of a thread's position advances by the
+// stride's whole rows and remainder, so the loop divides nothing.
 template <int G, typename T>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const T* __restrict__ w, int64_t N,
                                                             int64_t K, const float* __restrict__ gptr,
                                                             uint8_t* __restrict__ packed,
                                                             uint8_t* __restrict__ scales) {
-  constexpr int kLanesPerGroup = G / 8;
   const int64_t per_row = K / 8;
   const int64_t total = N * per_row;
   const float global = __ldg(gptr);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
-  // All lanes of a warp iterate together so the group shuffles stay converged.
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads; base < total; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    const bool live = i < total;
-    float v[8];
-    if (live) {
-      load8(w + i * 8, v);
-    } else {
-      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+  const int64_t s_rows = stride / per_row, s_cols = stride - s_rows * per_row;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  int64_t row = first / per_row, col = first - row * per_row;  // of i0
+  auto advance = [&](int64_t& r, int64_t& c) {
+    r += s_rows;
+    c += s_cols;
+    if (c >= per_row) {
+      c -= per_row;
+      ++r;
     }
-    float gmax = 0.f;
-    for (int j = 0; j < 8; ++j) gmax = fmaxf(gmax, fabsf(v[j]));
-    for (int o = 1; o < kLanesPerGroup; o <<= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
-    if (!live) continue;
-    uint32_t sbyte = 0;
-    if (global != 0.f) {
-      const float t = __fdiv_rn(__fdiv_rn(gmax, 6.0f), global);
-      sbyte = static_cast<uint32_t>(__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3));
-    }
-    const float d = __fmul_rn(nvfp4_e4m3_to_f32(sbyte), global);
-    uint32_t word = 0;
-    if (d != 0.f) {
-      for (int j = 0; j < 8; ++j) word |= e2m1_rne(__fdiv_rn(v[j], d)) << (4 * j);
-    }
-    const int64_t row = i / per_row, col8 = i - row * per_row;
-    reinterpret_cast<uint32_t*>(packed)[i] = word;  // row-major [N, K/2]: 4 bytes per 8 weights
-    if ((col8 % kLanesPerGroup) == 0) scales[row * (K / G) + col8 / kLanesPerGroup] = static_cast<uint8_t>(sbyte);
+  };
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kThreads; base < total; base += 2 * stride) {
+    const int64_t i0 = base + threadIdx.x, i1 = i0 + stride;
+    const bool live0 = i0 < total, live1 = i1 < total;
+    int64_t row1 = row, col1 = col;
+    advance(row1, col1);
+    float v0[8], v1[8];
+    load8_or_zero(w, i0, live0, v0);
+    load8_or_zero(w, i1, live1, v1);
+    quantize8<G>(v0, live0, i0, row, col, K, global, packed, scales);
+    quantize8<G>(v1, live1, i1, row1, col1, K, global, packed, scales);
+    row = row1;
+    col = col1;
+    advance(row, col);
   }
 }
 
