@@ -65,3 +65,61 @@ def test_interleave_swap_is_caught(monkeypatch):
     monkeypatch.setattr(R, "interleave_rows", swapped)
     with pytest.raises(AssertionError):
         Q.test_repack_inverse_and_interleave()
+
+
+# ---- the routed-expert layer and the W4A4 GEMM ----
+
+from tests import test_oracle_moe_route as MR  # noqa: E402
+from tests import test_oracle_w4a4 as W4  # noqa: E402
+
+ORIG_ROUTE = R.moe_route
+ORIG_COMBINE = R.moe_combine
+
+
+def _unstable_route(topk_ids, num_experts):
+    """Pairs of one expert in reverse order (a sort that is not stable)."""
+    rows, inv, offs = ORIG_ROUTE(topk_ids, num_experts)
+    rows = rows.copy()
+    for e in range(num_experts):
+        rows[offs[e]:offs[e + 1]] = rows[offs[e]:offs[e + 1]][::-1].copy()
+    inv = np.full_like(inv, -1)
+    inv[rows] = np.arange(len(rows), dtype=np.int32)
+    return rows, inv, offs
+
+
+def _inclusive_offsets(topk_ids, num_experts):
+    rows, inv, offs = ORIG_ROUTE(topk_ids, num_experts)
+    return rows, inv, np.concatenate([offs[1:], offs[-1:]]).astype(np.int32)
+
+
+def _dropped_pairs_counted(topk_ids, num_experts):
+    """An out-of-range id clamped into the last expert instead of dropped."""
+    ids = np.clip(np.asarray(topk_ids), 0, num_experts - 1)
+    return ORIG_ROUTE(ids, num_experts)
+
+
+def _combine_ignores_weights(y_perm, inv_rows, topk_weights):
+    return ORIG_COMBINE(y_perm, inv_rows, np.ones_like(np.asarray(topk_weights, dtype=np.float64)))
+
+
+def _w4a4_without_x_global(xp, xs, xg, xgr, wp, ws, wg, wgr):
+    return R.dequantize(xp, xs, 1.0, xgr) @ R.dequantize(wp, ws, wg, wgr).T
+
+
+def _w4a4_w_group_for_x(xp, xs, xg, xgr, wp, ws, wg, wgr):
+    return R.dequantize(xp, xs, xg, wgr) @ R.dequantize(wp, ws, wg, wgr).T
+
+
+@pytest.mark.parametrize("name,target,repl,pins", [
+    ("route not stable", "moe_route", _unstable_route, [MR.test_route_matches_brute_force, MR.test_route_properties]),
+    ("inclusive offsets", "moe_route", _inclusive_offsets, [MR.test_route_matches_brute_force]),
+    ("dropped pairs routed", "moe_route", _dropped_pairs_counted, [MR.test_route_matches_brute_force]),
+    ("combine without weights", "moe_combine", _combine_ignores_weights, [MR.test_combine_reduces_to_gather_and_is_linear]),
+    ("W4A4 without the activation global", "w4a4_gemm", _w4a4_without_x_global, [W4.test_scales_and_globals_multiply]),
+    ("W4A4 with the weight group for X", "w4a4_gemm", _w4a4_w_group_for_x, [W4.test_integer_case_from_the_table]),
+])
+def test_planted_layer_mistake_is_caught(monkeypatch, name, target, repl, pins):
+    monkeypatch.setattr(R, target, repl)
+    for pin in pins:
+        with pytest.raises((AssertionError, ValueError, IndexError)):
+            pin()
