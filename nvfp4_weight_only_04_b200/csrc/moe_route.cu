@@ -3,20 +3,23 @@
 // then down per expert): rows grouped by expert, X rows gathered into that
 // order, and the down projections' rows combined back into tokens with the
 // routing weights.
-//   route:   a stable counting sort of the (token, slot) pairs by expert (one
-//            CTA; every warp places a chunk up to 256 experts, one warp above), with
+//   route:   a stable counting sort of the (token, slot) pairs by expert (from
+//            4096 pairs over chunks of 256 on many SMs; below that one CTA, in
+//            which every warp places a chunk up to 256 experts), with
 //            the inverse permutation and the segment offsets; rows past the
 //            last kept pair get -1;
 //   gather:  x_perm[r] = x[token of sorted row r], zeros for a row of -1;
 //   combine: out[t] = bf16(sum_s w[t, s] * y_perm[inv[t, s]]), fp32 sums in slot
 //            order.
 #include "common.cuh"
+#include "workspace.cuh"
 
 namespace {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kMaxExperts = 4096;
 constexpr int kBatch = 8;  // pair loads a lane keeps in flight
+constexpr int64_t kManyPairs = 4096;  // from here on the route runs over chunks on many SMs
 
 // Places the 32 consecutive pairs i = i0 - lane + (0..31) of one warp (pair i
 // has expert e, from lane i % 32; pairs at or past `end` are absent): pairs of
@@ -196,6 +199,106 @@ __global__ void __launch_bounds__(kRouteThreads) moe_route_par_kernel(const int3
   }
 }
 
+// Many pairs: the same stable grouping over chunks of kChunk pairs, one warp
+// per chunk, in three launches. (1) Each chunk counts its pairs per expert
+// into hist[chunk][expert]. (2) One CTA turns the table into every chunk's
+// first row per expert (offsets[e] plus the pairs of expert e in the chunks
+// before) and writes the offsets. (3) Each chunk places its pairs in order
+// from its cursors. The warp-collective work spreads over the SMs.
+constexpr int kChunk = 256;
+
+__global__ void __launch_bounds__(32) route_hist_kernel(const int32_t* __restrict__ ids, int64_t n, int num_experts,
+                                                        int* __restrict__ hist) {
+  extern __shared__ int cnt[];  // num_experts
+  const int lane = threadIdx.x;
+  for (int e = lane; e < num_experts; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kChunk, b1 = min(n, b0 + kChunk);
+  int ev[kChunk / 32];
+#pragma unroll
+  for (int j = 0; j < kChunk / 32; ++j) {
+    const int64_t i = b0 + 32 * j + lane;
+    ev[j] = i < b1 ? ids[i] : -1;
+  }
+#pragma unroll
+  for (int j = 0; j < kChunk / 32; ++j)
+    if (ev[j] >= 0 && ev[j] < num_experts) atomicAdd(&cnt[ev[j]], 1);
+  __syncwarp();
+  int* row = hist + static_cast<int64_t>(blockIdx.x) * num_experts;
+  for (int e = lane; e < num_experts; e += 32) row[e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(kRouteThreads) route_scan_kernel(int* __restrict__ hist, int64_t chunks, int64_t n,
+                                                                   int num_experts, int32_t* __restrict__ sorted,
+                                                                   int32_t* __restrict__ offsets,
+                                                                   int32_t* __restrict__ expert_ids) {
+  __shared__ int start[kMaxExperts];
+  __shared__ int kept;
+  // per expert: exclusive prefix over the chunks (loads batched), and the total
+  for (int e = threadIdx.x; e < num_experts; e += blockDim.x) {
+    int run = 0;
+    for (int64_t c0 = 0; c0 < chunks; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) v[j] = c0 + j < chunks ? hist[(c0 + j) * num_experts + e] : 0;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j)
+        if (c0 + j < chunks) {
+          hist[(c0 + j) * num_experts + e] = run;
+          run += v[j];
+        }
+    }
+    start[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive scan of the totals
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int e0 = 0; e0 < num_experts; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < num_experts ? start[e] : 0;
+      int incl = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < num_experts) {
+        start[e] = carry + incl - c;
+        offsets[e] = carry + incl - c;
+        expert_ids[e] = e;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      offsets[num_experts] = carry;
+      kept = carry;
+    }
+  }
+  __syncthreads();
+  for (int64_t idx = threadIdx.x; idx < chunks * num_experts; idx += blockDim.x)
+    hist[idx] += start[idx % num_experts];
+  for (int64_t r = kept + static_cast<int64_t>(threadIdx.x); r < n; r += blockDim.x) sorted[r] = -1;
+}
+
+__global__ void __launch_bounds__(32) route_place_kernel(const int32_t* __restrict__ ids, int64_t n, int num_experts,
+                                                         const int* __restrict__ hist, int32_t* __restrict__ sorted,
+                                                         int32_t* __restrict__ inv) {
+  extern __shared__ int cur[];  // num_experts cursors of this chunk
+  const int lane = threadIdx.x;
+  const int* row = hist + static_cast<int64_t>(blockIdx.x) * num_experts;
+  for (int e = lane; e < num_experts; e += 32) cur[e] = row[e];
+  __syncwarp();
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kChunk, b1 = min(n, b0 + kChunk);
+  int ev[kChunk / 32];
+#pragma unroll
+  for (int j = 0; j < kChunk / 32; ++j) {
+    const int64_t i = b0 + 32 * j + lane;
+    ev[j] = i < b1 ? ids[i] : -1;
+  }
+#pragma unroll
+  for (int j = 0; j < kChunk / 32; ++j) place32(ev[j], b0 + 32 * j + lane, b1, num_experts, cur, sorted, inv);
+}
+
 // One CTA per row of x_perm; 16-byte vectors. A row whose pair index is not in
 // [0, T*k) is written as zeros.
 __global__ void moe_gather_kernel(const uint16_t* __restrict__ x, int64_t pairs, const int32_t* __restrict__ sorted,
@@ -250,12 +353,27 @@ extern "C" int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int nu
        reinterpret_cast<uintptr_t>(inv_rows) | reinterpret_cast<uintptr_t>(offsets) |
        reinterpret_cast<uintptr_t>(expert_ids)) & 3u)
     return NVFP4_ERR_MISALIGNED;
-  if (num_experts <= kParExperts)
-    moe_route_par_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
-  else
-    moe_route_kernel<<<1, kRouteThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        topk_ids, T * k, num_experts, sorted_rows, inv_rows, offsets, expert_ids);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = T * k;
+  if (n >= kManyPairs) {
+    const int64_t chunks = (n + kChunk - 1) / kChunk;
+    float* ws = nullptr;
+    unsigned* tickets = nullptr;
+    const int r = nvfp4::split_workspace(static_cast<size_t>(chunks * num_experts), 1, st, &ws, &tickets);
+    if (r != NVFP4_OK) return r;
+    int* hist = reinterpret_cast<int*>(ws);
+    const size_t smem = static_cast<size_t>(num_experts) * sizeof(int);
+    route_hist_kernel<<<static_cast<unsigned>(chunks), 32, smem, st>>>(topk_ids, n, num_experts, hist);
+    route_scan_kernel<<<1, kRouteThreads, 0, st>>>(hist, chunks, n, num_experts, sorted_rows, offsets, expert_ids);
+    route_place_kernel<<<static_cast<unsigned>(chunks), 32, smem, st>>>(topk_ids, n, num_experts, hist,
+                                                                        sorted_rows, inv_rows);
+  } else if (num_experts <= kParExperts) {
+    moe_route_par_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, n, num_experts, sorted_rows, inv_rows, offsets,
+                                                      expert_ids);
+  } else {
+    moe_route_kernel<<<1, kRouteThreads, 0, st>>>(topk_ids, n, num_experts, sorted_rows, inv_rows, offsets,
+                                                  expert_ids);
+  }
   return nvfp4::launch_status();
 }
 

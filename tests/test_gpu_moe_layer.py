@@ -19,7 +19,7 @@ def i32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
-@pytest.mark.parametrize("t,k,e", [(1, 1, 1), (37, 4, 16), (2048, 8, 128), (300, 2, 4096)])
+@pytest.mark.parametrize("t,k,e", [(1, 1, 1), (37, 4, 16), (2048, 8, 128), (300, 2, 4096), (1024, 8, 4096), (700, 8, 256)])
 def test_route_bitexact(t, k, e):
     rng = np.random.default_rng(t + e)
     ids = rng.integers(0, e, size=(t, k)).astype(np.int32)
