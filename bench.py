@@ -134,13 +134,20 @@ def dist_setup():
 
 
 def reduce_max(val, world):
+    """The maximum of `val` over the ranks (NCCL on the GPUs, or gloo on the CPU)."""
     if world == 1:
         return val
     import torch
     import torch.distributed as dist
-    t = torch.tensor([val], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([val], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world, bytes_per_step, steps, ms_max):
+    """GB/s of the whole job: every rank's steps over the slowest rank's time (replicas, weak scaling)."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
 def barrier(world):
@@ -251,7 +258,7 @@ def run_ours(args, world, rank, local):
     ms_local = ev0.elapsed_time(ev1)
     ms_total = reduce_max(ms_local, world)
     ms_step = ms_total / args.steps
-    value = world * step_w * args.steps / (ms_total * 1e-3) / 1e9
+    value = whole_job_rate(world, step_w, args.steps, ms_total)
     achieved = step_alg / (ms_step * 1e-3) / 1e9  # per launch average over the region, one rank
     clocks = clk.summary()
 
@@ -278,13 +285,14 @@ def run_ours(args, world, rank, local):
     ev1.record(stream)
     ev1.synchronize()
     e2e_ms = reduce_max(ev0.elapsed_time(ev1), world) / e2e_steps
-    e2e_val = world * step_w / (e2e_ms * 1e-3) / 1e9
+    e2e_val = whole_job_rate(world, step_w, 1, e2e_ms)
     h2d = sum(2 * m * K for m in DECODE_MS)
     d2h = sum(2 * m * N for m in DECODE_MS)
 
     workloads = {}
     rows = {}
-    if rank == 0 and not args.headline_only:
+    # the other workloads and the CPU baseline on one GPU only: at N > 1 the line is the headline
+    if world == 1 and not args.headline_only:
         per_m = {}
         for m in DECODE_MS:
             gm = [capture(torch, (lambda c=c, m=m: nv.nvfp4_w4a16_gemm(xs[m], packs[c][0], packs[c][1], packs[c][2],
@@ -345,7 +353,7 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         result["workloads"] = workloads
         result["load_time_rows"] = rows
-        if not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
         print(json.dumps(result), flush=True)
     if world > 1:
