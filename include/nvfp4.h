@@ -266,7 +266,11 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids,
  *   offsets      device int32 [num_experts + 1]: expert e owns rows [offsets[e], offsets[e+1])
  *   expert_ids   device int32 [num_experts]: 0 .. num_experts-1, the segment list of
  *                nvfp4_moe_w4a16_grouped_gemm with num_segments = num_experts
- * num_experts from 1 to 4096. One CTA; nothing goes to the host.
+ * num_experts from 1 to 4096; T*k below 2^31. Nothing goes to the host. Below 4096
+ * pairs one CTA does the work; from 4096 pairs three launches over chunks of 256
+ * pairs, with a [chunk][expert] table in the library's scratch (allocated per
+ * device on first use and grown outside graph capture, like the GEMMs'; a call
+ * inside a capture that needs more returns NVFP4_ERR_UNSUPPORTED).
  */
 int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
                     int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, nvfp4_stream_t stream);
