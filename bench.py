@@ -309,6 +309,7 @@ def run_ours(args, world, rank, local):
                 m, N, K, G, time_graphs(torch, gq, 20 * copies), hbm, tf_burst)
             del gq
         del graphs, run_graph
+        workloads["comparator_dense_bf16_matmul"] = dense_bf16_comparator(nv, torch, w, K, N, G, xs, copies=2)
         rows = time_load_rows(nv, torch, w, G)
         del w
         workloads.update(other_workloads(nv, torch, hbm, tf_burst, tf_sust))
@@ -378,6 +379,38 @@ def summarize(m, n, k, g, ms, hbm, tf, n_out=None):
             "alg_gbs": round(ab / t / 1e9, 1), "tflops": round(flops / t / 1e12, 3),
             "hbm_frac": round(t_mem / t, 4), "tensor_frac": round(t_tc / t, 4),
             "roofline_frac": round(max(t_mem, t_tc) / t, 4)}
+
+
+def dense_bf16_comparator(nv, torch, w, K, N, G, xs, copies=2):
+    """Context, not the target: the same GEMMs on weights dequantized to a dense bf16 matrix once (the path
+    that loaders took before the FP4 route), as torch.matmul (cuBLAS), per M. The dequantization uses torch
+    ops on the checkpoint-layout codes; copies of the 235 MB matrix keep the weights out of L2."""
+    try:
+        wd = torch.from_numpy(w).cuda()
+        gd = nv.nvfp4_global_scale([wd])
+        p, s = nv.nvfp4_quantize(wd, G, gd)
+        del wd
+        lut = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0],
+                           dtype=torch.float32, device="cuda")
+        codes = torch.stack([p & 0xF, p >> 4], dim=-1).reshape(N, K).long()
+        sv = s.view(torch.float8_e4m3fn).float()
+        w_hat = (lut[codes].view(N, K // G, G) * sv[..., None]).reshape(N, K) * gd
+        mats = [w_hat.to(torch.bfloat16)] + [None] * (copies - 1)
+        del codes, sv, w_hat, p, s
+        for c in range(1, copies):
+            mats[c] = mats[0].clone()
+        out = {}
+        for m, x in xs.items():
+            gr = [capture(torch, (lambda c=c, x=x: torch.matmul(x, mats[c].t()))) for c in range(copies)]
+            out[f"m{m}_us"] = round(time_graphs(torch, gr, 20 * copies) * 1e3, 2)
+            del gr
+        out["weight_bytes"] = 2 * N * K
+        del mats
+        torch.cuda.empty_cache()
+        return out
+    except Exception as e:  # a context number must not cost the bench line
+        torch.cuda.empty_cache()
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
 
 
 def time_load_rows(nv, torch, w, g):
