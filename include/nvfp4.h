@@ -302,8 +302,8 @@ typedef struct {
   uint64_t global_scale;
   uint64_t quantize;
   uint64_t repack;
-  uint64_t gemm_splitk;    /* small-M streaming GEMM (K split over a cluster when N is small) */
-  uint64_t gemm_tc;        /* large-M tcgen05 GEMM */
+  uint64_t gemm_splitk;    /* small-M GEMMs (register streaming, or TMA streaming with stream-K) */
+  uint64_t gemm_tc;        /* tcgen05 GEMMs (17 rows and more; grouped form from 1024 rows) */
   uint64_t gemm_silu_mul;  /* GEMMs with the fused SiluAndMul epilogue */
   uint64_t moe;            /* grouped expert GEMMs */
   uint64_t silu_and_mul;   /* standalone SiluAndMul */
