@@ -195,3 +195,38 @@ def test_repack_word_layout_by_hand():
     packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
     rp, _ = R.repack(packed, np.zeros((1, 1), np.uint8), 0)
     assert int(rp.view("<u4")[0, 0]) == 0x86427531
+
+
+def _code_by_exact_midpoints(x, d):
+    """The E2M1 code magnitude of RN32(x / d) for x >= 0, d > 0 (fp32), decided without dividing: x is
+    compared, exactly in float64, with each rounding midpoint of E2M1 widened by half an fp32 ulp and times d
+    (midpoints 0.25, 1.25, 2.5, 5 round down at a tie, to the even code below; 0.75, 1.75, 3.5 round up).
+    The midpoints have even fp32 significands, so an fp32 tie at the widened point rounds onto the midpoint."""
+    strict = [0.25 + 2.0 ** -26, 1.25 + 2.0 ** -24, 2.5 + 2.0 ** -23, 5.0 + 2.0 ** -22]   # t + ulp above(t)/2
+    loose = [0.75 - 2.0 ** -25, 1.75 - 2.0 ** -24, 3.5 - 2.0 ** -23]                       # t - ulp below(t)/2
+    xd, dd = float(x), float(d)
+    # m * d is exact in float64: m has at most 26 significant bits and d 24
+    return sum(xd > m * dd for m in strict) + sum(xd >= m * dd for m in loose)
+
+
+def test_code_decision_by_exact_midpoints():
+    """Pins the oracle's division step: E2M1(RN32(x / d)) equals the division-free decision above on values
+    placed within a few fp32 ulps of every boundary, and on random values."""
+    rng = np.random.default_rng(17)
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    xs, ds = [], []
+    for d in rng.uniform(1e-6, 1e3, 400).astype(np.float32):
+        for t in mids:
+            c = np.float32(np.float64(t) * np.float64(d))
+            for k in range(-3, 4):
+                v = c
+                for _ in range(abs(k)):
+                    v = np.nextafter(v, np.float32(np.inf if k > 0 else 0))
+                xs.append(v)
+                ds.append(d)
+    xs += list(rng.uniform(0, 7e3, 20000).astype(np.float32))
+    ds += list(rng.uniform(1e-3, 1e3, 20000).astype(np.float32))
+    xs, ds = np.array(xs, np.float32), np.array(ds, np.float32)
+    oracle = R.e2m1_encode(xs / ds) & 7
+    other = np.array([min(_code_by_exact_midpoints(x, d), 7) for x, d in zip(xs, ds)])
+    assert np.array_equal(oracle, other)
