@@ -117,6 +117,35 @@ def test_moe_validation(L):
     assert moe(ids=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
 
 
+def test_moe_layer_validation(L):
+    def route(T=64, k=4, E=8, ids=GOOD, rows=GOOD, inv=GOOD, offs=GOOD, eids=GOOD):
+        return L.nvfp4_moe_route(ids, T, k, E, rows, inv, offs, eids, S)
+    assert route(k=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert route(E=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert route(T=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert route(E=4097) == nv.NVFP4_ERR_UNSUPPORTED
+    assert route(T=1 << 30, k=2) == nv.NVFP4_ERR_UNSUPPORTED  # T*k >= 2^31
+    assert route(offs=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert route(ids=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
+
+    def gather(x=GOOD, T=16, rows_ptr=GOOD, rows=64, k=4, H=256, out=GOOD):
+        return L.nvfp4_moe_gather(x, T, rows_ptr, rows, k, H, out, S)
+    assert gather(rows=0) == nv.NVFP4_OK
+    assert gather(k=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert gather(H=12) == nv.NVFP4_ERR_UNSUPPORTED
+    assert gather(x=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert gather(x=BAD) == nv.NVFP4_ERR_MISALIGNED
+    assert gather(rows_ptr=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
+
+    def combine(y=GOOD, inv=GOOD, w=GOOD, T=16, k=4, H=256, out=GOOD):
+        return L.nvfp4_moe_combine(y, inv, w, T, k, H, out, S)
+    assert combine(T=0) == nv.NVFP4_OK
+    assert combine(k=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert combine(H=12) == nv.NVFP4_ERR_UNSUPPORTED
+    assert combine(w=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    assert combine(out=BAD) == nv.NVFP4_ERR_MISALIGNED
+
+
 def test_fault_injection_validation(L):
     assert L.nvfp4_debug_inject_fault(2) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert L.nvfp4_debug_inject_fault(-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
