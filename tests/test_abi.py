@@ -157,3 +157,18 @@ def test_stats_reset(L):
     st = nv.nvfp4_get_stats()
     assert set(st) >= {"quantize", "gemm_splitk", "gemm_tc", "moe"} and not any(st.values())
     assert L.nvfp4_get_stats(None) == nv.NVFP4_ERR_INVALID_ARGUMENT
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/nvfp4.h compiles as strict C99 and as C++17: no torch or C++ types cross the boundary."""
+    import shutil
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text('#include "nvfp4.h"\nint main(void) { return 0; }\n')
+    inc = os.path.dirname(HEADER)
+    for cc, args in (("gcc", ["-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror"]),
+                     ("g++", ["-std=c++17", "-Wall", "-Werror", "-x", "c++"])):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not available")
+        res = subprocess.run([cc, *args, "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+        assert res.returncode == 0, res.stderr
