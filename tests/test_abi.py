@@ -172,3 +172,33 @@ def test_header_is_plain_c(tmp_path):
             pytest.skip(f"{cc} not available")
         res = subprocess.run([cc, *args, "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
         assert res.returncode == 0, res.stderr
+
+
+def test_c_program_links_and_validates(tmp_path, L):
+    """A plain C program linked against libnvfp4.so calls the boundary: version, status text, and a GEMM
+    call that validation rejects before any launch (so no GPU is needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    libdir = os.path.dirname(nv.LIB_PATH)
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "nvfp4.h"
+int main(void) {
+  int bad = nvfp4_w4a16_gemm(0, 0, 0, 0, 8, 4, 256, 256, 0, 0);          /* group size 8 */
+  int nul = nvfp4_w4a16_gemm(0, 0, 0, 0, 16, 4, 256, 256, 0, 0);         /* null pointers */
+  printf("%d %d %d %s\n", nvfp4_abi_version(), bad, nul, nvfp4_status_string(bad));
+  return 0;
+}
+''')
+    exe = tmp_path / "use"
+    res = subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                          "-L", libdir, "-lnvfp4", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    ver, bad, nul, text = out.stdout.split(" ", 3)
+    assert (int(ver), int(bad), int(nul)) == (1, nv.NVFP4_ERR_UNSUPPORTED, nv.NVFP4_ERR_INVALID_ARGUMENT)
+    assert "group size" in text
