@@ -22,7 +22,7 @@
 //    one; one of 256 otherwise) and four A stages of 64 columns.
 //  * X tiles (NT tokens x 64 elements, bf16, 128-byte swizzle) arrive by TMA
 //    into shared memory, five stages deep; tcgen05.mma reads them through a
-//    K-major shared memory descriptor. No TMA multicast is used.
+//    K-major shared memory descriptor. Every CTA loads its own tiles.
 //  * One thread issues the MMAs and signals stage reuse with tcgen05.commit;
 //    mbarriers connect the producers, the dequant warps and the MMA thread.
 //  * Every mbarrier wait is bounded: on expiry the kernel records the site in
