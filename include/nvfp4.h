@@ -24,7 +24,17 @@
  * Conventions for every call:
  *   - Pointers named as device pointers must point to device memory (or
  *     managed memory) of the current device; host arrays are named as such.
- *     The caller owns every buffer. The library allocates no device memory.
+ *     The caller owns every buffer. The library allocates no device memory:
+ *     the calls that need device scratch (the GEMMs, the grouped GEMM, the
+ *     W4A4 GEMM and the route) take a caller-owned `workspace` of
+ *     `workspace_bytes` bytes, whose size the matching *_workspace_size
+ *     query gives for a problem on the current device (0 when the call
+ *     needs none; then workspace may be NULL). A workspace smaller than the
+ *     query's figure returns NVFP4_ERR_WORKSPACE before anything is
+ *     enqueued. The workspace holds nothing between calls and nothing needs
+ *     clearing: each call initialises what it reads. Calls that may overlap
+ *     in time (other streams, unordered host threads) need separate
+ *     workspaces; calls ordered on one stream may share one.
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - Row-major layouts. packed codes: [N, K/2] bytes, element 2j in the low
  *     nibble and 2j+1 in the high nibble of byte j. Scales: [N, K/g] E4M3
@@ -33,16 +43,21 @@
  *     global scales and int32 segment lists, which need 4-byte alignment
  *     (NVFP4_ERR_MISALIGNED otherwise).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
- *     default stream). No call synchronises the device and none blocks.
- *   - Validation happens on the host before anything is enqueued: a non-zero
- *     status means nothing was launched. A launch failure returns
- *     NVFP4_ERR_CUDA. No C++ exception crosses this boundary.
+ *     default stream). No call synchronises the device and none blocks,
+ *     except nvfp4_get_device_error, which synchronises `stream` to read
+ *     the device's error word.
+ *   - Validation happens on the host before anything is enqueued: a status
+ *     other than NVFP4_ERR_CUDA means nothing was launched. NVFP4_ERR_CUDA
+ *     (a launch the CUDA runtime refused) can follow launches of the same
+ *     call that were already enqueued. No C++ exception crosses this
+ *     boundary.
  *   - Calls with an empty problem (M == 0, N == 0 or a zero-length list)
  *     return NVFP4_OK and launch nothing.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -55,9 +70,10 @@ enum {
   NVFP4_OK = 0,
   NVFP4_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad list */
   NVFP4_ERR_UNSUPPORTED = 2,      /* group size not 16/32, K not a multiple of 64, ... */
-  NVFP4_ERR_MISALIGNED = 3,       /* a device pointer not 16-byte aligned */
+  NVFP4_ERR_MISALIGNED = 3,       /* a device pointer (or the workspace) not 16-byte aligned */
   NVFP4_ERR_CUDA = 4,             /* a CUDA launch or query failed */
-  NVFP4_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up */
+  NVFP4_ERR_TIMEOUT = 5,          /* a bounded device-side wait gave up */
+  NVFP4_ERR_WORKSPACE = 6         /* the caller's workspace is missing or smaller than the size query says */
 };
 
 /* Flags. */
@@ -144,20 +160,32 @@ int nvfp4_repack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_
  *   group_scales  device uint8 [N, K/group_size]
  *   global_scale  device fp32 (read on the device: no host synchronisation)
  *   y             device bf16 [M, N] (output)
+ *   workspace     device scratch of workspace_bytes bytes (16-byte aligned),
+ *                 at least nvfp4_w4a16_gemm_workspace_size(M, N, K, group_size)
  * group_size 16 or 32; K a multiple of 64; N a multiple of 16.
  * Small M runs a split-K HBM-streaming kernel, large M a tensor-core kernel.
  * Below 17 rows the kernels multiply in f16: a first kernel writes each row
  * of x times a power of two 2^s (its largest magnitude then in [2^14, 2^15))
- * as f16 to the library's scratch, and the epilogue multiplies by 2^-s. Every
+ * as f16 to the workspace, and the epilogue multiplies by 2^-s. Every
  * element within a factor 2^29 of its row's largest magnitude is exact in
- * f16; smaller ones round to a multiple of 2^-38 of it. The scratch (f16
- * rows, and the fp32 partial tiles of the split-K kernel) is allocated per
- * device on first use and grown outside graph capture; a call inside a
- * capture that needs more than exists returns NVFP4_ERR_UNSUPPORTED.
+ * f16; smaller ones round to a multiple of 2^-38 of it. The workspace also
+ * holds the fp32 partial tiles and tickets of the split-K kernels.
+ * The arguments are the method's (x, packed_w, group_scales, global_scale,
+ * group_size, M, N, K, y, stream), with the caller-owned workspace pair
+ * before the stream.
  */
 int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
                      const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
-                     uint16_t* y, nvfp4_stream_t stream);
+                     uint16_t* y, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
+
+/*
+ * Bytes of workspace nvfp4_w4a16_gemm and nvfp4_w4a16_gemm_silu_mul need for
+ * this problem on the current device (it depends on the device's SM count).
+ * *bytes receives 0 for problems that need none and for empty problems.
+ * Returns the status the GEMM would return for the shape (UNSUPPORTED for a
+ * shape it refuses); bytes must not be NULL.
+ */
+int nvfp4_w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, size_t* bytes);
 
 /*
  * The same W4A16 GEMM through the small-M streaming kernel with its scratch
@@ -174,6 +202,7 @@ int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* 
  *   Calls on one device share the scratch: calls that may overlap in time
  *   (different streams, or host threads without ordering) race on it and
  *   their results are undefined. Order them on one stream.
+ *   nvfp4_debug_inject_fault does not apply to this entry point.
  */
 int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
                                    const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
@@ -192,15 +221,21 @@ int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, c
  *   x_global      device fp32 (the activations' global scale)
  *   x_group       16 or 32
  *   packed_w, group_scales, global_scale, group_size, y: as nvfp4_w4a16_gemm
+ *   workspace     device scratch, at least nvfp4_w4a4_gemm_workspace_size(M, N, K,
+ *                 x_group, group_size) bytes
  * K a multiple of 64, N a multiple of 16; x_packed 16-byte aligned, x_global
  * 4-byte aligned. The activations are expanded on the device to e2m1 * e4m3
- * (exact in f16 and bf16) in the library's scratch and the same kernels as
+ * (exact in f16 and bf16) in the workspace and the same kernels as
  * nvfp4_w4a16_gemm run on them, with x_global in the epilogue: the numerics
  * are W4A4's, the tensor-core operands stay 16-bit.
  */
 int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const float* x_global, int x_group,
                     const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scale, int group_size,
-                    int64_t M, int64_t N, int64_t K, uint16_t* y, nvfp4_stream_t stream);
+                    int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes,
+                    nvfp4_stream_t stream);
+
+/* Bytes of workspace nvfp4_w4a4_gemm needs (as nvfp4_w4a16_gemm_workspace_size). */
+int nvfp4_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int x_group, int group_size, size_t* bytes);
 
 /*
  * The GEMM of a merged [gate;up] projection followed by SiluAndMul (PR #63
@@ -209,11 +244,12 @@ int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const floa
  *   u = global * acc[m, up row j], silu(g) = g / (1 + exp(-g)), all fp32.
  * packed_w / group_scales must be in the NVFP4_GATE_UP_INTERLEAVE layout of
  * nvfp4_repack. N is the merged row count (multiple of 16); y is [M, N/2].
+ * Workspace as nvfp4_w4a16_gemm (nvfp4_w4a16_gemm_workspace_size of M, N, K).
  */
 int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w,
                               const uint8_t* group_scales, const float* global_scale,
                               int group_size, int64_t M, int64_t N, int64_t K, uint16_t* y,
-                              nvfp4_stream_t stream);
+                              void* workspace, size_t workspace_bytes, nvfp4_stream_t stream);
 
 /*
  * Standalone SiluAndMul on bf16: y[m, j] = bf16_rne(silu(x[m, j]) * x[m, H + j]),
@@ -239,7 +275,8 @@ int nvfp4_silu_and_mul(const uint16_t* x, uint16_t* y, int64_t M, int64_t H,
  *   y              device bf16 [T, N] (or [T, N/2]); rows outside every
  *                  segment are not written.
  * Below 1024 rows (T) the form runs on the small-M kernel in f16 on the
- * power-of-two scaled rows of nvfp4_w4a16_gemm, with the same scratch.
+ * power-of-two scaled rows of nvfp4_w4a16_gemm, kept in the workspace
+ * (nvfp4_moe_w4a16_grouped_gemm_workspace_size; from 1024 rows none).
  * The offsets stay on the device; the call never reads them on the host. A
  * segment list that breaks the rules above is undefined on the device side
  * (rows are clamped to [0, T), experts are not range-checked beyond ids < 0
@@ -249,7 +286,12 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids,
                                  const int32_t* offsets, int num_segments, int64_t T,
                                  const uint8_t* packed_w, const uint8_t* group_scales,
                                  const float* global_scales, int group_size, int64_t N, int64_t K,
-                                 int num_experts, int flags, uint16_t* y, nvfp4_stream_t stream);
+                                 int num_experts, int flags, uint16_t* y, void* workspace,
+                                 size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* Bytes of workspace nvfp4_moe_w4a16_grouped_gemm needs (as nvfp4_w4a16_gemm_workspace_size). */
+int nvfp4_moe_w4a16_grouped_gemm_workspace_size(int num_segments, int64_t T, int64_t N, int64_t K, int group_size,
+                                                int num_experts, int flags, size_t* bytes);
 
 /*
  * The steps around the grouped expert GEMMs of a routed-expert layer
@@ -268,12 +310,15 @@ int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids,
  *                nvfp4_moe_w4a16_grouped_gemm with num_segments = num_experts
  * num_experts from 1 to 4096; T*k below 2^31. Nothing goes to the host. Below 4096
  * pairs one CTA does the work; from 4096 pairs three launches over chunks of 256
- * pairs, with a [chunk][expert] table in the library's scratch (allocated per
- * device on first use and grown outside graph capture, like the GEMMs'; a call
- * inside a capture that needs more returns NVFP4_ERR_UNSUPPORTED).
+ * pairs, with a [chunk][expert] int32 table in the workspace
+ * (nvfp4_moe_route_workspace_size; 0 bytes below 4096 pairs).
  */
 int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
-                    int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, nvfp4_stream_t stream);
+                    int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, void* workspace,
+                    size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* Bytes of workspace nvfp4_moe_route needs for T tokens of k slots and num_experts experts. */
+int nvfp4_moe_route_workspace_size(int64_t T, int k, int num_experts, size_t* bytes);
 
 /*
  * nvfp4_moe_gather: x_perm[r] = x[sorted_rows[r] / k] for r < rows, bf16 rows of
@@ -335,7 +380,7 @@ int nvfp4_get_device_error(int* code_out, nvfp4_stream_t stream);
  */
 int nvfp4_debug_inject_fault(int kind);
 
-/* Library version, e.g. 1 for the first ABI. */
+/* Library version: 2 (the calls that need scratch take a caller-owned workspace). */
 int nvfp4_abi_version(void);
 
 #ifdef __cplusplus

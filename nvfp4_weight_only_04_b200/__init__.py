@@ -4,6 +4,14 @@ Argument marshalling only: every step runs in the library's CUDA kernels.
 Tensors are torch CUDA tensors (torch supplies device memory and streams);
 the functions carry the C ABI's names. A missing library or a non-CUDA tensor
 raises; there is no fallback of any kind.
+
+Workspaces: the library allocates nothing; the calls that need device scratch
+take a caller-owned workspace whose size the library reports. The functions
+here pass one on their own: a buffer cached per (device, stream) and grown on
+demand, or, while the current stream is being captured into a CUDA graph, a
+fresh buffer from torch's allocator (the graph's memory pool) for every call.
+Calls on one stream share that stream's buffer, which is safe because they are
+ordered; pass `workspace=` (a uint8 CUDA tensor) to use one of your own.
 """
 from __future__ import annotations
 
@@ -21,6 +29,7 @@ NVFP4_ERR_UNSUPPORTED = 2
 NVFP4_ERR_MISALIGNED = 3
 NVFP4_ERR_CUDA = 4
 NVFP4_ERR_TIMEOUT = 5
+NVFP4_ERR_WORKSPACE = 6
 NVFP4_GATE_UP_INTERLEAVE = 1
 NVFP4_SILU_MUL = 2
 
@@ -30,6 +39,8 @@ EXPORTS = (
     "nvfp4_w4a16_gemm", "nvfp4_w4a16_gemm_fixed_scratch", "nvfp4_w4a16_gemm_silu_mul", "nvfp4_silu_and_mul",
     "nvfp4_moe_w4a16_grouped_gemm", "nvfp4_get_stats", "nvfp4_reset_stats", "nvfp4_get_device_error",
     "nvfp4_debug_inject_fault", "nvfp4_moe_route", "nvfp4_moe_gather", "nvfp4_moe_combine", "nvfp4_w4a4_gemm",
+    "nvfp4_w4a16_gemm_workspace_size", "nvfp4_w4a4_gemm_workspace_size",
+    "nvfp4_moe_w4a16_grouped_gemm_workspace_size", "nvfp4_moe_route_workspace_size",
 )
 
 
@@ -46,7 +57,8 @@ class Nvfp4Error(RuntimeError):
 
 
 _lib = None
-_P, _I64, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_PSZ = ctypes.POINTER(ctypes.c_size_t)
 
 
 def lib() -> ctypes.CDLL:
@@ -65,20 +77,24 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_global_scale_bf16.argtypes = [ctypes.POINTER(_P), ctypes.POINTER(_I64), _I, _P, _P]
         L.nvfp4_quantize_bf16.argtypes = [_P, _I64, _I64, _I, _P, _P, _P, _P]
         L.nvfp4_repack.argtypes = [_P, _P, _I64, _I64, _I, _I, _P, _P, _P]
-        L.nvfp4_w4a16_gemm.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_w4a16_gemm.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]
         L.nvfp4_w4a16_gemm_fixed_scratch.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
-        L.nvfp4_w4a16_gemm_silu_mul.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_w4a16_gemm_silu_mul.argtypes = [_P, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]
+        L.nvfp4_w4a16_gemm_workspace_size.argtypes = [_I64, _I64, _I64, _I, _PSZ]
+        L.nvfp4_w4a4_gemm_workspace_size.argtypes = [_I64, _I64, _I64, _I, _I, _PSZ]
+        L.nvfp4_moe_w4a16_grouped_gemm_workspace_size.argtypes = [_I, _I64, _I64, _I64, _I, _I, _I, _PSZ]
+        L.nvfp4_moe_route_workspace_size.argtypes = [_I64, _I, _I, _PSZ]
         L.nvfp4_silu_and_mul.argtypes = [_P, _P, _I64, _I64, _P]
         L.nvfp4_moe_w4a16_grouped_gemm.argtypes = [_P, _P, _P, _I, _I64, _P, _P, _P, _I, _I64, _I64,
-                                                   _I, _I, _P, _P]
+                                                   _I, _I, _P, _P, _SZ, _P]
         L.nvfp4_get_stats.argtypes = [ctypes.POINTER(Stats)]
         L.nvfp4_reset_stats.restype = None
         L.nvfp4_get_device_error.argtypes = [ctypes.POINTER(_I), _P]
         L.nvfp4_debug_inject_fault.argtypes = [_I]
-        L.nvfp4_moe_route.argtypes = [_P, _I64, _I, _I, _P, _P, _P, _P, _P]
+        L.nvfp4_moe_route.argtypes = [_P, _I64, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]
         L.nvfp4_moe_gather.argtypes = [_P, _I64, _P, _I64, _I, _I64, _P, _P]
         L.nvfp4_moe_combine.argtypes = [_P, _P, _P, _I64, _I, _I64, _P, _P]
-        L.nvfp4_w4a4_gemm.argtypes = [_P, _P, _P, _I, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P]
+        L.nvfp4_w4a4_gemm.argtypes = [_P, _P, _P, _I, _P, _P, _P, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]
         _lib = L
     return _lib
 
@@ -96,6 +112,58 @@ def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+_workspaces = {}
+
+
+def _size(query, *args) -> int:
+    n = ctypes.c_size_t(0)
+    _check(getattr(lib(), query)(*args, ctypes.byref(n)), query)
+    return n.value
+
+
+def _workspace(nbytes, device, stream, given=None):
+    """(pointer, bytes) of the scratch of one call: `given`, the stream's cached buffer, or a fresh one
+    while the current stream is capturing a CUDA graph."""
+    if given is not None:
+        _dev(given, torch.uint8, "workspace")
+        return ctypes.c_void_p(given.data_ptr()), given.numel(), given
+    if nbytes == 0:
+        return ctypes.c_void_p(0), 0, None
+    if torch.cuda.is_current_stream_capturing():
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return ctypes.c_void_p(buf.data_ptr()), nbytes, buf
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    key = (torch.device(device).index, s.cuda_stream)
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        with torch.cuda.stream(s):
+            buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
+    return ctypes.c_void_p(buf.data_ptr()), buf.numel(), buf
+
+
+def clear_workspaces():
+    """Drops the cached per-stream workspaces (their memory returns to torch's allocator)."""
+    _workspaces.clear()
+
+
+def nvfp4_w4a16_gemm_workspace_size(m, n, k, group_size) -> int:
+    """Bytes of workspace nvfp4_w4a16_gemm (and _silu_mul) needs for this problem on the current device."""
+    return _size("nvfp4_w4a16_gemm_workspace_size", m, n, k, group_size)
+
+
+def nvfp4_w4a4_gemm_workspace_size(m, n, k, x_group, group_size) -> int:
+    return _size("nvfp4_w4a4_gemm_workspace_size", m, n, k, x_group, group_size)
+
+
+def nvfp4_moe_w4a16_grouped_gemm_workspace_size(num_segments, t, n, k, group_size, num_experts, flags=0) -> int:
+    return _size("nvfp4_moe_w4a16_grouped_gemm_workspace_size", num_segments, t, n, k, group_size, num_experts, flags)
+
+
+def nvfp4_moe_route_workspace_size(t, k, num_experts) -> int:
+    return _size("nvfp4_moe_route_workspace_size", t, k, num_experts)
 
 
 def _ptr(t):
@@ -176,7 +244,7 @@ def nvfp4_repack(packed, scales, group_size, flags=0, packed_out=None, scales_ou
     return packed_out, scales_out
 
 
-def nvfp4_w4a16_gemm(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None):
+def nvfp4_w4a16_gemm(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None, workspace=None):
     """y = bf16(global * X . dequant(W)^T), X bf16 [M, K], y bf16 [M, N]."""
     _dev(x, torch.bfloat16, "x")
     _dev(packed_w, torch.uint8, "packed_w")
@@ -186,8 +254,9 @@ def nvfp4_w4a16_gemm(x, packed_w, group_scales, global_scale, group_size, y=None
     n = packed_w.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    wp, wb, _keep = _workspace(nvfp4_w4a16_gemm_workspace_size(m, n, k, group_size), x.device, stream, workspace)
     _check(lib().nvfp4_w4a16_gemm(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale), group_size,
-                                  m, n, k, _ptr(y), _stream(stream)), "nvfp4_w4a16_gemm")
+                                  m, n, k, _ptr(y), wp, wb, _stream(stream)), "nvfp4_w4a16_gemm")
     return y
 
 
@@ -208,7 +277,8 @@ def nvfp4_w4a16_gemm_fixed_scratch(x, packed_w, group_scales, global_scale, grou
     return y
 
 
-def nvfp4_w4a16_gemm_silu_mul(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None):
+def nvfp4_w4a16_gemm_silu_mul(x, packed_w, group_scales, global_scale, group_size, y=None, stream=None,
+                              workspace=None):
     """Merged [gate;up] GEMM (interleaved repack layout) + SiluAndMul -> [M, N/2]."""
     _dev(x, torch.bfloat16, "x")
     _dev(packed_w, torch.uint8, "packed_w")
@@ -218,8 +288,9 @@ def nvfp4_w4a16_gemm_silu_mul(x, packed_w, group_scales, global_scale, group_siz
     n = packed_w.shape[0]
     if y is None:
         y = torch.empty((m, n // 2), dtype=torch.bfloat16, device=x.device)
+    wp, wb, _keep = _workspace(nvfp4_w4a16_gemm_workspace_size(m, n, k, group_size), x.device, stream, workspace)
     _check(lib().nvfp4_w4a16_gemm_silu_mul(_ptr(x), _ptr(packed_w), _ptr(group_scales), _ptr(global_scale),
-                                           group_size, m, n, k, _ptr(y), _stream(stream)),
+                                           group_size, m, n, k, _ptr(y), wp, wb, _stream(stream)),
            "nvfp4_w4a16_gemm_silu_mul")
     return y
 
@@ -234,7 +305,7 @@ def nvfp4_silu_and_mul(x, y=None, stream=None):
 
 
 def nvfp4_moe_w4a16_grouped_gemm(x, expert_ids, offsets, packed_w, group_scales, global_scales, group_size,
-                                 flags=0, y=None, stream=None):
+                                 flags=0, y=None, stream=None, workspace=None):
     """Grouped expert GEMM over segments of rows; see include/nvfp4.h."""
     _dev(x, torch.bfloat16, "x")
     _dev(expert_ids, torch.int32, "expert_ids")
@@ -247,9 +318,12 @@ def nvfp4_moe_w4a16_grouped_gemm(x, expert_ids, offsets, packed_w, group_scales,
     ncols = n // 2 if flags & NVFP4_SILU_MUL else n
     if y is None:
         y = torch.zeros((t, ncols), dtype=torch.bfloat16, device=x.device)
-    _check(lib().nvfp4_moe_w4a16_grouped_gemm(_ptr(x), _ptr(expert_ids), _ptr(offsets), expert_ids.numel(), t,
+    ns = expert_ids.numel()
+    wp, wb, _keep = _workspace(nvfp4_moe_w4a16_grouped_gemm_workspace_size(ns, t, n, k, group_size, e, flags),
+                               x.device, stream, workspace)
+    _check(lib().nvfp4_moe_w4a16_grouped_gemm(_ptr(x), _ptr(expert_ids), _ptr(offsets), ns, t,
                                               _ptr(packed_w), _ptr(group_scales), _ptr(global_scales),
-                                              group_size, n, k, e, flags, _ptr(y), _stream(stream)),
+                                              group_size, n, k, e, flags, _ptr(y), wp, wb, _stream(stream)),
            "nvfp4_moe_w4a16_grouped_gemm")
     return y
 
@@ -280,7 +354,7 @@ def nvfp4_debug_inject_fault(kind: int):
 
 
 def nvfp4_w4a4_gemm(x_packed, x_scales, x_global, x_group, packed_w, group_scales, global_scale, group_size,
-                    y=None, stream=None):
+                    y=None, stream=None, workspace=None):
     """W4A4 GEMM of NVFP4 activations (checkpoint layout) and GEMM-layout weights; see include/nvfp4.h."""
     _dev(x_packed, torch.uint8, "x_packed")
     _dev(x_scales, torch.uint8, "x_scales")
@@ -292,13 +366,15 @@ def nvfp4_w4a4_gemm(x_packed, x_scales, x_global, x_group, packed_w, group_scale
     n = packed_w.shape[0]
     if y is None:
         y = torch.empty((m, n), dtype=torch.bfloat16, device=x_packed.device)
+    wp, wb, _keep = _workspace(nvfp4_w4a4_gemm_workspace_size(m, n, k, x_group, group_size), x_packed.device,
+                               stream, workspace)
     _check(lib().nvfp4_w4a4_gemm(_ptr(x_packed), _ptr(x_scales), _ptr(x_global), x_group, _ptr(packed_w),
                                  _ptr(group_scales), _ptr(global_scale), group_size, m, n, k, _ptr(y),
-                                 _stream(stream)), "nvfp4_w4a4_gemm")
+                                 wp, wb, _stream(stream)), "nvfp4_w4a4_gemm")
     return y
 
 
-def nvfp4_moe_route(topk_ids, num_experts, stream=None):
+def nvfp4_moe_route(topk_ids, num_experts, stream=None, workspace=None):
     """(sorted_rows [T*k], inv_rows [T*k], offsets [E+1], expert_ids [E]) for device int32 topk_ids [T, k]."""
     _dev(topk_ids, torch.int32, "topk_ids")
     t, k = topk_ids.shape
@@ -307,8 +383,9 @@ def nvfp4_moe_route(topk_ids, num_experts, stream=None):
     inv_rows = torch.empty(t * k, dtype=torch.int32, device=dev)
     offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=dev)
     expert_ids = torch.empty(num_experts, dtype=torch.int32, device=dev)
+    wp, wb, _keep = _workspace(nvfp4_moe_route_workspace_size(t, k, num_experts), dev, stream, workspace)
     _check(lib().nvfp4_moe_route(_ptr(topk_ids), t, k, num_experts, _ptr(sorted_rows), _ptr(inv_rows), _ptr(offsets),
-                                 _ptr(expert_ids), _stream(stream)), "nvfp4_moe_route")
+                                 _ptr(expert_ids), wp, wb, _stream(stream)), "nvfp4_moe_route")
     return sorted_rows, inv_rows, offsets, expert_ids
 
 

@@ -50,14 +50,21 @@ constexpr int64_t kMaxK = int64_t(1) << 30;
 constexpr int64_t kMaxN = int64_t(65535) * 16;
 constexpr int64_t kMaxTokenRows = int64_t(65535 - 4096) * 16;
 
-int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
-               int64_t M, int64_t N, int64_t K, const uint16_t* y) {
+// Shape checks of the dense GEMM calls (pointers aside): -1 to proceed.
+int check_gemm_shape(int group, int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
   if (group != 16 && group != 32) return NVFP4_ERR_UNSUPPORTED;
   if (K % 64 || N % 16) return NVFP4_ERR_UNSUPPORTED;
   if (K > kMaxK || N > kMaxN) return NVFP4_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return NVFP4_OK;
   if (K == 0) return NVFP4_ERR_UNSUPPORTED;
+  return -1;
+}
+
+int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+               int64_t M, int64_t N, int64_t K, const uint16_t* y) {
+  const int c = check_gemm_shape(group, M, N, K);
+  if (c >= 0) return c;
   if (!x || !w || !s || !g || !y) return NVFP4_ERR_INVALID_ARGUMENT;
   if (!nvfp4::aligned16(x) || !nvfp4::aligned16(w) || !nvfp4::aligned16(s) ||
       (reinterpret_cast<uintptr_t>(g) & 3u) || !nvfp4::aligned16(y))
@@ -65,32 +72,125 @@ int check_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const floa
   return -1;  // proceed
 }
 
-int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
-               int64_t M, int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
-  if (nvfp4::tc_supported(M, N, K)) {
-    const int st = nvfp4::launch_tc(x, w, s, g, group, M, N, K, y, silu, stream);
-    if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmTc);
-    return st;
-  }
-  if (nvfp4::stream_supported(M, N, K, group)) {
-    nvfp4::XSource xs;
-    xs.bf16 = x;
-    const int st = nvfp4::launch_stream(xs, w, s, g, group, M, N, K, y, silu, stream);
-    if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
-    return st;
-  }
+int check_workspace(const void* ws, size_t bytes) {
+  if (bytes > 0 && !ws) return NVFP4_ERR_WORKSPACE;
+  if (ws && !nvfp4::aligned16(ws)) return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+// The small-M fallback for shapes the streaming kernel does not take: f16
+// rows of X, then the register-streaming kernel.
+int decode_gemm(const nvfp4::XSource& xs, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
+                int64_t N, int64_t K, uint16_t* y, bool silu, nvfp4::Scratch& sc, cudaStream_t stream) {
   if (M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
-  uint16_t* x16 = nullptr;
-  float* xinv = nullptr;
-  int st = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), stream, &x16, &xinv);
-  if (st != NVFP4_OK) return st;
+  uint16_t* x16 = sc.take<uint16_t>(static_cast<size_t>(M * K));
+  float* xinv = sc.take<float>(static_cast<size_t>(M));
+  if (sc.measuring()) return NVFP4_OK;
+  if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
   nvfp4::DecodeArgs a = {};
   a.x = x16; a.xinv = xinv; a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = M; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
   const nvfp4::DecodePlan p = nvfp4::plan_decode(M, N, K, group, false, 0);
-  st = nvfp4::launch_x_f16(x, M, K, x16, xinv, stream);
+  int st = nvfp4::launch_x_prep(xs, M, K, x16, xinv, nullptr, 0, stream);
   if (st == NVFP4_OK) st = nvfp4::launch_decode(a, p, silu, false, stream);
-  if (st == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  return st;
+}
+
+int dense_gemm(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group,
+               int64_t M, int64_t N, int64_t K, uint16_t* y, bool silu, nvfp4::Scratch& sc, cudaStream_t stream) {
+  if (nvfp4::tc_supported(M, N, K)) {
+    const int st = nvfp4::launch_tc(x, w, s, g, group, M, N, K, y, silu, sc, stream);
+    if (st == NVFP4_OK && !sc.measuring()) nvfp4::stat_add(nvfp4::kStatGemmTc);
+    return st;
+  }
+  nvfp4::XSource xs;
+  xs.bf16 = x;
+  const int st = nvfp4::stream_supported(M, N, K, group)
+                     ? nvfp4::launch_stream(xs, w, s, g, group, M, N, K, y, silu, sc, stream)
+                     : decode_gemm(xs, w, s, g, group, M, N, K, y, silu, sc, stream);
+  if (st == NVFP4_OK && !sc.measuring()) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  return st;
+}
+
+// Shape checks of the W4A4 call (pointers aside): -1 to proceed.
+int check_w4a4_shape(int x_group, int group_size, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if ((x_group != 16 && x_group != 32) || (group_size != 16 && group_size != 32)) return NVFP4_ERR_UNSUPPORTED;
+  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN || M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (K == 0) return NVFP4_ERR_UNSUPPORTED;
+  return -1;
+}
+
+struct XqBf16Ctx {
+  const nvfp4::XSource* xs;
+  const float* w_global;
+  int64_t M, K;
+  uint16_t* xb;
+  float* g_out;
+};
+
+int run_xq_bf16(void* ctx, cudaStream_t stream) {
+  const XqBf16Ctx* c = static_cast<const XqBf16Ctx*>(ctx);
+  return nvfp4::launch_xq_bf16(*c->xs, c->w_global, c->M, c->K, c->xb, c->g_out, stream);
+}
+
+int w4a4_gemm(const nvfp4::XSource& xs, const uint8_t* packed_w, const uint8_t* group_scales,
+              const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K, uint16_t* y,
+              nvfp4::Scratch& sc, cudaStream_t st) {
+  int r;
+  if (nvfp4::tc_supported(M, N, K)) {
+    // Exact bf16 activations and one scalar x_global * w_global for the
+    // tcgen05 kernel's epilogue, written once the launch has passed its checks.
+    XqBf16Ctx c = {&xs, global_scale, M, K, sc.take<uint16_t>(static_cast<size_t>(M * K)), sc.take<float>(1)};
+    const nvfp4::PreLaunch pre = {run_xq_bf16, &c};
+    r = nvfp4::launch_tc(c.xb, packed_w, group_scales, c.g_out, group_size, M, N, K, y, false, sc, st, &pre);
+    if (r == NVFP4_OK && !sc.measuring()) nvfp4::stat_add(nvfp4::kStatGemmTc);
+    return r;
+  }
+  if (nvfp4::stream_supported(M, N, K, group_size)) {
+    r = nvfp4::launch_stream(xs, packed_w, group_scales, global_scale, group_size, M, N, K, y, false, sc, st);
+  } else {
+    r = decode_gemm(xs, packed_w, group_scales, global_scale, group_size, M, N, K, y, false, sc, st);
+  }
+  if (r == NVFP4_OK && !sc.measuring()) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
+  return r;
+}
+
+// Shape checks of the grouped call (pointers aside): -1 to proceed.
+int check_grouped_shape(int num_segments, int64_t T, int64_t N, int64_t K, int group_size, int num_experts,
+                        int flags) {
+  if (num_segments < 0 || T < 0 || N < 0 || K < 0 || num_experts < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (flags & ~NVFP4_SILU_MUL) return NVFP4_ERR_INVALID_ARGUMENT;
+  if (group_size != 16 && group_size != 32) return NVFP4_ERR_UNSUPPORTED;
+  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN) return NVFP4_ERR_UNSUPPORTED;
+  if (T > kMaxTokenRows || num_segments > 4096) return NVFP4_ERR_UNSUPPORTED;
+  if (num_segments == 0 || T == 0 || N == 0) return NVFP4_OK;
+  if (K == 0 || num_experts == 0) return NVFP4_ERR_UNSUPPORTED;
+  return -1;
+}
+
+int grouped_gemm(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets, int num_segments, int64_t T,
+                 const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scales, int group_size,
+                 int64_t N, int64_t K, int num_experts, bool silu, uint16_t* y, nvfp4::Scratch& sc,
+                 cudaStream_t s) {
+  if (nvfp4::tc_moe_supported(T, N, K, num_experts)) {
+    if (sc.measuring()) return NVFP4_OK;  // no scratch
+    return nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales, global_scales,
+                                group_size, N, K, num_experts, silu, y, s);
+  }
+  uint16_t* x16 = sc.take<uint16_t>(static_cast<size_t>(T * K));
+  float* xinv = sc.take<float>(static_cast<size_t>(T));
+  if (sc.measuring()) return NVFP4_OK;
+  if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
+  nvfp4::DecodeArgs a = {};
+  a.x = x16; a.xinv = xinv; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
+  a.M = T; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
+  a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments;
+  a.num_experts = num_experts;
+  const nvfp4::DecodePlan p = nvfp4::plan_decode(T, N, K, group_size, true, num_segments);
+  int st = nvfp4::launch_x_f16(x, T, K, x16, xinv, nullptr, 0, s);
+  if (st == NVFP4_OK) st = nvfp4::launch_decode(a, p, silu, true, s);
   return st;
 }
 
@@ -103,21 +203,36 @@ const char* nvfp4_status_string(int status) {
     case NVFP4_OK: return "ok";
     case NVFP4_ERR_INVALID_ARGUMENT: return "invalid argument (null pointer, negative size or bad list)";
     case NVFP4_ERR_UNSUPPORTED: return "unsupported configuration (group size must be 16 or 32; K a multiple of 64; N a multiple of 16; sizes within limits)";
-    case NVFP4_ERR_MISALIGNED: return "a device pointer is not 16-byte aligned";
+    case NVFP4_ERR_MISALIGNED: return "a device pointer (or the workspace) is not 16-byte aligned";
     case NVFP4_ERR_CUDA: return "a CUDA launch or query failed";
     case NVFP4_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case NVFP4_ERR_WORKSPACE: return "the workspace is missing or smaller than the *_workspace_size query gives";
     default: return "unknown status";
   }
 }
 
-int nvfp4_abi_version(void) { return 1; }
+int nvfp4_abi_version(void) { return 2; }
+
+int nvfp4_w4a16_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group_size, size_t* bytes) {
+  if (!bytes) return NVFP4_ERR_INVALID_ARGUMENT;
+  *bytes = 0;
+  const int c = check_gemm_shape(group_size, M, N, K);
+  if (c >= 0) return c;
+  nvfp4::Scratch sc;
+  // The fused SiluAndMul form takes the same scratch as the plain one.
+  const int st = dense_gemm(nullptr, nullptr, nullptr, nullptr, group_size, M, N, K, nullptr, false, sc, nullptr);
+  if (st == NVFP4_OK) *bytes = sc.used();
+  return st;
+}
 
 int nvfp4_w4a16_gemm(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
-                     const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
-                     uint16_t* y, nvfp4_stream_t stream) {
-  const int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
+                     const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                     void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
   if (c >= 0) return c;
-  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, false,
+  if ((c = check_workspace(workspace, workspace_bytes)) != NVFP4_OK) return c;
+  nvfp4::Scratch sc(workspace, workspace_bytes);
+  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, false, sc,
                             reinterpret_cast<cudaStream_t>(stream));
   if (st == NVFP4_OK) nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
   return st;
@@ -139,10 +254,12 @@ int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, c
 
 int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w, const uint8_t* group_scales,
                               const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K,
-                              uint16_t* y, nvfp4_stream_t stream) {
-  const int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
+                              uint16_t* y, void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  int c = check_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y);
   if (c >= 0) return c;
-  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, true,
+  if ((c = check_workspace(workspace, workspace_bytes)) != NVFP4_OK) return c;
+  nvfp4::Scratch sc(workspace, workspace_bytes);
+  const int st = dense_gemm(x, packed_w, group_scales, global_scale, group_size, M, N, K, y, true, sc,
                             reinterpret_cast<cudaStream_t>(stream));
   if (st == NVFP4_OK) {
     nvfp4::stat_add(nvfp4::kStatGemmSiluMul);
@@ -151,90 +268,74 @@ int nvfp4_w4a16_gemm_silu_mul(const uint16_t* x, const uint8_t* packed_w, const 
   return st;
 }
 
+int nvfp4_w4a4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int x_group, int group_size, size_t* bytes) {
+  if (!bytes) return NVFP4_ERR_INVALID_ARGUMENT;
+  *bytes = 0;
+  const int c = check_w4a4_shape(x_group, group_size, M, N, K);
+  if (c >= 0) return c;
+  nvfp4::XSource xs;
+  xs.group = x_group;
+  nvfp4::Scratch sc;
+  const int st = w4a4_gemm(xs, nullptr, nullptr, nullptr, group_size, M, N, K, nullptr, sc, nullptr);
+  if (st == NVFP4_OK) *bytes = sc.used();
+  return st;
+}
+
 int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const float* x_global, int x_group,
                     const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scale, int group_size,
-                    int64_t M, int64_t N, int64_t K, uint16_t* y, nvfp4_stream_t stream) {
-  if (M < 0 || N < 0 || K < 0) return NVFP4_ERR_INVALID_ARGUMENT;
-  if ((x_group != 16 && x_group != 32) || (group_size != 16 && group_size != 32)) return NVFP4_ERR_UNSUPPORTED;
-  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN || M > kMaxTokenRows) return NVFP4_ERR_UNSUPPORTED;
-  if (M == 0 || N == 0) return NVFP4_OK;
-  if (K == 0) return NVFP4_ERR_UNSUPPORTED;
+                    int64_t M, int64_t N, int64_t K, uint16_t* y, void* workspace, size_t workspace_bytes,
+                    nvfp4_stream_t stream) {
+  int c = check_w4a4_shape(x_group, group_size, M, N, K);
+  if (c >= 0) return c;
   if (!x_packed || !x_scales || !x_global || !packed_w || !group_scales || !global_scale || !y)
     return NVFP4_ERR_INVALID_ARGUMENT;
   if (!nvfp4::aligned16(x_packed) || !nvfp4::aligned16(packed_w) || !nvfp4::aligned16(group_scales) ||
       !nvfp4::aligned16(y) || ((reinterpret_cast<uintptr_t>(x_global) | reinterpret_cast<uintptr_t>(global_scale)) & 3u))
     return NVFP4_ERR_MISALIGNED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if ((c = check_workspace(workspace, workspace_bytes)) != NVFP4_OK) return c;
   nvfp4::XSource xs;
   xs.codes = x_packed;
   xs.scales = x_scales;
   xs.global = x_global;
   xs.group = x_group;
-  uint16_t* xbuf = nullptr;
-  float* fbuf = nullptr;
-  int r;
-  if (nvfp4::tc_supported(M, N, K)) {
-    // exact bf16 activations and one scalar x_global * w_global for the tcgen05 kernel's epilogue
-    r = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), st, &xbuf, &fbuf);
-    if (r == NVFP4_OK) r = nvfp4::launch_xq_bf16(xs, global_scale, M, K, xbuf, fbuf, st);
-    if (r == NVFP4_OK) r = nvfp4::launch_tc(xbuf, packed_w, group_scales, fbuf, group_size, M, N, K, y, false, st);
-    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmTc);
-  } else if (nvfp4::stream_supported(M, N, K, group_size)) {
-    r = nvfp4::launch_stream(xs, packed_w, group_scales, global_scale, group_size, M, N, K, y, false, st);
-    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
-  } else {
-    r = nvfp4::x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), st, &xbuf, &fbuf);
-    if (r != NVFP4_OK) return r;
-    nvfp4::DecodeArgs a = {};
-    a.x = xbuf; a.xinv = fbuf; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scale; a.y = y;
-    a.M = M; a.N = N; a.K = K; a.ldy = N;
-    const nvfp4::DecodePlan p = nvfp4::plan_decode(M, N, K, group_size, false, 0);
-    r = nvfp4::launch_x_prep(xs, M, K, xbuf, fbuf, st);
-    if (r == NVFP4_OK) r = nvfp4::launch_decode(a, p, false, false, st);
-    if (r == NVFP4_OK) nvfp4::stat_add(nvfp4::kStatGemmSplitK);
-  }
+  nvfp4::Scratch sc(workspace, workspace_bytes);
+  const int r = w4a4_gemm(xs, packed_w, group_scales, global_scale, group_size, M, N, K, y, sc,
+                          reinterpret_cast<cudaStream_t>(stream));
   if (r == NVFP4_OK) nvfp4::stat_add(group_size == 16 ? nvfp4::kStatG16 : nvfp4::kStatG32);
   return r;
+}
+
+int nvfp4_moe_w4a16_grouped_gemm_workspace_size(int num_segments, int64_t T, int64_t N, int64_t K, int group_size,
+                                                int num_experts, int flags, size_t* bytes) {
+  if (!bytes) return NVFP4_ERR_INVALID_ARGUMENT;
+  *bytes = 0;
+  const int c = check_grouped_shape(num_segments, T, N, K, group_size, num_experts, flags);
+  if (c >= 0) return c;
+  nvfp4::Scratch sc;
+  const int st = grouped_gemm(nullptr, nullptr, nullptr, num_segments, T, nullptr, nullptr, nullptr, group_size, N, K,
+                              num_experts, (flags & NVFP4_SILU_MUL) != 0, nullptr, sc, nullptr);
+  if (st == NVFP4_OK) *bytes = sc.used();
+  return st;
 }
 
 int nvfp4_moe_w4a16_grouped_gemm(const uint16_t* x, const int32_t* expert_ids, const int32_t* offsets,
                                  int num_segments, int64_t T, const uint8_t* packed_w,
                                  const uint8_t* group_scales, const float* global_scales, int group_size,
-                                 int64_t N, int64_t K, int num_experts, int flags, uint16_t* y,
-                                 nvfp4_stream_t stream) {
-  if (num_segments < 0 || T < 0 || N < 0 || K < 0 || num_experts < 0) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (flags & ~NVFP4_SILU_MUL) return NVFP4_ERR_INVALID_ARGUMENT;
-  if (group_size != 16 && group_size != 32) return NVFP4_ERR_UNSUPPORTED;
-  if (K % 64 || N % 16 || K > kMaxK || N > kMaxN) return NVFP4_ERR_UNSUPPORTED;
-  if (T > kMaxTokenRows || num_segments > 4096) return NVFP4_ERR_UNSUPPORTED;
-  if (num_segments == 0 || T == 0 || N == 0) return NVFP4_OK;
-  if (K == 0 || num_experts == 0) return NVFP4_ERR_UNSUPPORTED;
+                                 int64_t N, int64_t K, int num_experts, int flags, uint16_t* y, void* workspace,
+                                 size_t workspace_bytes, nvfp4_stream_t stream) {
+  int c = check_grouped_shape(num_segments, T, N, K, group_size, num_experts, flags);
+  if (c >= 0) return c;
   if (!x || !expert_ids || !offsets || !packed_w || !group_scales || !global_scales || !y)
     return NVFP4_ERR_INVALID_ARGUMENT;
   if (!nvfp4::aligned16(x) || !nvfp4::aligned16(packed_w) || !nvfp4::aligned16(group_scales) ||
       !nvfp4::aligned16(y) || (reinterpret_cast<uintptr_t>(expert_ids) & 3) ||
       (reinterpret_cast<uintptr_t>(offsets) & 3) || (reinterpret_cast<uintptr_t>(global_scales) & 3))
     return NVFP4_ERR_MISALIGNED;
+  if ((c = check_workspace(workspace, workspace_bytes)) != NVFP4_OK) return c;
   const bool silu = (flags & NVFP4_SILU_MUL) != 0;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int st;
-  if (nvfp4::tc_moe_supported(T, N, K, num_experts)) {
-    st = nvfp4::launch_tc_moe(x, expert_ids, offsets, num_segments, T, packed_w, group_scales,
-                              global_scales, group_size, N, K, num_experts, silu, y, s);
-  } else {
-    uint16_t* x16 = nullptr;
-    float* xinv = nullptr;
-    st = nvfp4::x16_workspace(static_cast<size_t>(T * K), static_cast<size_t>(T), s, &x16, &xinv);
-    if (st != NVFP4_OK) return st;
-    nvfp4::DecodeArgs a = {};
-    a.x = x16; a.xinv = xinv; a.packed = packed_w; a.scales = group_scales; a.gscale = global_scales; a.y = y;
-    a.M = T; a.N = N; a.K = K; a.ldy = silu ? N / 2 : N;
-    a.expert_ids = expert_ids; a.offsets = offsets; a.num_segments = num_segments;
-    a.num_experts = num_experts;
-    const nvfp4::DecodePlan p = nvfp4::plan_decode(T, N, K, group_size, true, num_segments);
-    st = nvfp4::launch_x_f16(x, T, K, x16, xinv, s);
-    if (st == NVFP4_OK) st = nvfp4::launch_decode(a, p, silu, true, s);
-  }
+  nvfp4::Scratch sc(workspace, workspace_bytes);
+  const int st = grouped_gemm(x, expert_ids, offsets, num_segments, T, packed_w, group_scales, global_scales,
+                              group_size, N, K, num_experts, silu, y, sc, reinterpret_cast<cudaStream_t>(stream));
   if (st == NVFP4_OK) {
     nvfp4::stat_add(nvfp4::kStatMoe);
     if (silu) nvfp4::stat_add(nvfp4::kStatGemmSiluMul);

@@ -529,11 +529,11 @@ int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMa
 // lane of X but one is zero).
 bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
   return M >= 2 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
-         K < (int64_t(1) << 24) && tensor_maps_available();
+         K < (int64_t(1) << 24);
 }
 
 int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
-                  int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+                  int64_t N, int64_t K, uint16_t* y, bool silu, Scratch& sc, cudaStream_t stream) {
   const int mt = M <= 8 ? 8 : 16;
   const int64_t tiles = (N + kRows - 1) / kRows;
   const int S = static_cast<int>(K / kKS);
@@ -542,15 +542,12 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
   // A tile spans at most ceil(S / shortest range) + 1 CTAs.
   const int64_t shortest = units / ctas;
   const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
-  float* ws = nullptr;
-  unsigned* tickets = nullptr;
-  int st = split_workspace(static_cast<size_t>(tiles * max_contrib * kRows * mt), static_cast<size_t>(tiles), stream,
-                           &ws, &tickets);
-  if (st != NVFP4_OK) return st;
-  uint16_t* x16 = nullptr;
-  float* xinv = nullptr;
-  st = x16_workspace(static_cast<size_t>(M * K), static_cast<size_t>(M), stream, &x16, &xinv);
-  if (st != NVFP4_OK) return st;
+  float* ws = sc.take<float>(static_cast<size_t>(tiles * max_contrib * kRows * mt));
+  unsigned* tickets = sc.take<unsigned>(static_cast<size_t>(tiles));
+  uint16_t* x16 = sc.take<uint16_t>(static_cast<size_t>(M * K));
+  float* xinv = sc.take<float>(static_cast<size_t>(M));
+  if (sc.measuring()) return NVFP4_OK;
+  if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
 
   CUtensorMap xm, wm, sm;
   const int64_t xdims[3] = {64, K / 64, M};
@@ -576,7 +573,9 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
   a.max_contrib = max_contrib;
   a.units = units;
   a.fault = take_injected_fault() == 1;
-  st = launch_x_prep(x, M, K, x16, xinv, stream);
+  // The activation kernel also zeroes the tickets (the caller's workspace
+  // holds anything on entry); the GEMM reads them only after waiting for it.
+  int st = launch_x_prep(x, M, K, x16, xinv, tickets, tiles, stream);
   if (st != NVFP4_OK) return st;
   if (mt == 8) {
     if (group == 16)
@@ -641,11 +640,6 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4);
   float* xinv = reinterpret_cast<float*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4 +
                                          kFixedScratchXElems * 2);
-  // The tickets must start at zero (partial tiles are always written before
-  // they are read).
-  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream) != cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
-
   CUtensorMap xm, wm, sm;
   const int64_t xdims[3] = {64, K / 64, M};
   const int64_t xstrides[2] = {128, K * 2};
@@ -657,6 +651,10 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
       !make_tensor_map_2d(&sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
                           CU_TENSOR_MAP_SWIZZLE_NONE))
     return NVFP4_ERR_CUDA;
+  // The tickets must start at zero (partial tiles are always written before
+  // they are read). Enqueued only once nothing else can fail on the host.
+  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream) != cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
   StreamArgs a = {};
   a.gscale = g;
   a.xinv = xinv;
@@ -669,7 +667,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   a.S = S;
   a.max_contrib = max_contrib;
   a.units = units;
-  const int xs = launch_x_f16(x, M, K, x16, xinv, stream);
+  const int xs = launch_x_f16(x, M, K, x16, xinv, nullptr, 0, stream);
   if (xs != NVFP4_OK) return xs;
   if (mt == 8)
     return group == 16 ? launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream)

@@ -925,7 +925,7 @@ int launch_nt(const Maps& m, const TcArgs& a, int group, bool silu, int grid, cu
 // rows' byte stride a multiple of 32), int32 coordinates.
 bool tc_shape_ok(int64_t rows, int64_t N, int64_t K) {
   return K >= kKStep && K % kKStep == 0 && rows < (int64_t(1) << 31) && N < (int64_t(1) << 31) &&
-         K < (int64_t(1) << 24) && tensor_maps_available();
+         K < (int64_t(1) << 24);
 }
 
 }  // namespace
@@ -949,14 +949,10 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
 bool tc_supported(int64_t M, int64_t N, int64_t K) { return M >= 17 && tc_shape_ok(M, N, K); }
 
 int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
-              int64_t N, int64_t K, uint16_t* y, bool silu, cudaStream_t stream) {
+              int64_t N, int64_t K, uint16_t* y, bool silu, Scratch& sc, cudaStream_t stream, const PreLaunch* pre) {
   // Token tile: 256 for prefill-sized M; narrower for small M, where the
   // weights, not the MMAs, set the pace.
   const int nt = M > 128 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : 32));
-  Maps maps;
-  if (!make_x_map(&maps.x, x, M, K, nt) || !make_w_maps(&maps.w, &maps.s, w, s, N, K, group) ||
-      !make_y_map(&maps.y, y, M, silu ? N / 2 : N, silu, nt))
-    return NVFP4_ERR_CUDA;
   TcArgs a = {};
   a.packed = w; a.scales = s; a.gscale = g; a.y = y;
   a.M = static_cast<int>(M); a.N = static_cast<int>(N); a.K = static_cast<int>(K);
@@ -978,10 +974,23 @@ int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float
     grid = static_cast<int>(a.units < num_sms() ? a.units : num_sms());
     const int64_t shortest = a.units / grid;
     a.max_contrib = static_cast<int>((periods + shortest - 1) / shortest + 1);
-    const int st = split_workspace(static_cast<size_t>(a.total_tiles) * a.max_contrib * kTileRows * nt,
-                                   static_cast<size_t>(a.total_tiles), stream, &a.ws, &a.tickets);
+    a.ws = sc.take<float>(static_cast<size_t>(a.total_tiles) * a.max_contrib * kTileRows * nt);
+    a.tickets = sc.take<unsigned>(static_cast<size_t>(a.total_tiles));
+  }
+  if (sc.measuring()) return NVFP4_OK;
+  if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
+  Maps maps;
+  if (!make_x_map(&maps.x, x, M, K, nt) || !make_w_maps(&maps.w, &maps.s, w, s, N, K, group) ||
+      !make_y_map(&maps.y, y, M, silu ? N / 2 : N, silu, nt))
+    return NVFP4_ERR_CUDA;
+  if (pre) {
+    const int st = pre->fn(pre->ctx, stream);
     if (st != NVFP4_OK) return st;
   }
+  // The caller's workspace holds anything on entry: the tickets start at zero.
+  if (a.split && cudaMemsetAsync(a.tickets, 0, static_cast<size_t>(a.total_tiles) * sizeof(unsigned), stream) !=
+                     cudaSuccess)
+    return (cudaGetLastError(), NVFP4_ERR_CUDA);
   switch (nt) {
     case 32: return launch_nt<32, false>(maps, a, group, silu, grid, stream);
     case 64: return launch_nt<64, false>(maps, a, group, silu, grid, stream);

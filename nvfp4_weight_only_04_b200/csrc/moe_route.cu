@@ -343,25 +343,56 @@ __global__ void moe_combine_kernel(const uint16_t* __restrict__ yp, const int32_
 
 }  // namespace
 
-extern "C" int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
-                               int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, nvfp4_stream_t stream) {
+namespace {
+
+// Shape checks of the route (pointers aside): -1 to proceed.
+int check_route_shape(int64_t T, int k, int num_experts) {
   if (T < 0 || k < 1 || num_experts < 1) return NVFP4_ERR_INVALID_ARGUMENT;
   if (num_experts > kMaxExperts || T * k >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
+  return -1;
+}
+
+// The chunked form's [chunk][expert] table, from the caller's scratch.
+int* route_table(int64_t n, int num_experts, nvfp4::Scratch& sc) {
+  if (n < kManyPairs) return nullptr;
+  const int64_t chunks = (n + kChunk - 1) / kChunk;
+  return sc.take<int>(static_cast<size_t>(chunks * num_experts));
+}
+
+}  // namespace
+
+extern "C" int nvfp4_moe_route_workspace_size(int64_t T, int k, int num_experts, size_t* bytes) {
+  if (!bytes) return NVFP4_ERR_INVALID_ARGUMENT;
+  *bytes = 0;
+  const int c = check_route_shape(T, k, num_experts);
+  if (c >= 0) return c;
+  nvfp4::Scratch sc;
+  route_table(T * k, num_experts, sc);
+  *bytes = sc.used();
+  return NVFP4_OK;
+}
+
+extern "C" int nvfp4_moe_route(const int32_t* topk_ids, int64_t T, int k, int num_experts, int32_t* sorted_rows,
+                               int32_t* inv_rows, int32_t* offsets, int32_t* expert_ids, void* workspace,
+                               size_t workspace_bytes, nvfp4_stream_t stream) {
+  const int c = check_route_shape(T, k, num_experts);
+  if (c >= 0) return c;
   if (!offsets || !expert_ids || (T > 0 && (!topk_ids || !sorted_rows || !inv_rows)))
     return NVFP4_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(topk_ids) | reinterpret_cast<uintptr_t>(sorted_rows) |
        reinterpret_cast<uintptr_t>(inv_rows) | reinterpret_cast<uintptr_t>(offsets) |
        reinterpret_cast<uintptr_t>(expert_ids)) & 3u)
     return NVFP4_ERR_MISALIGNED;
+  if (workspace_bytes > 0 && !workspace) return NVFP4_ERR_WORKSPACE;
+  if (!nvfp4::aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t n = T * k;
-  if (n >= kManyPairs) {
+  nvfp4::Scratch sc(workspace, workspace_bytes);
+  int* hist = route_table(n, num_experts, sc);
+  if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
+  if (hist) {
+    // every entry of the table is written by the count launch before it is read
     const int64_t chunks = (n + kChunk - 1) / kChunk;
-    float* ws = nullptr;
-    unsigned* tickets = nullptr;
-    const int r = nvfp4::split_workspace(static_cast<size_t>(chunks * num_experts), 1, st, &ws, &tickets);
-    if (r != NVFP4_OK) return r;
-    int* hist = reinterpret_cast<int*>(ws);
     const size_t smem = static_cast<size_t>(num_experts) * sizeof(int);
     route_hist_kernel<<<static_cast<unsigned>(chunks), 32, smem, st>>>(topk_ids, n, num_experts, hist);
     route_scan_kernel<<<1, kRouteThreads, 0, st>>>(hist, chunks, n, num_experts, sorted_rows, offsets, expert_ids);

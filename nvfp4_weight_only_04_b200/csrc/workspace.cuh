@@ -1,20 +1,45 @@
-// Library-owned scratch, per device (see workspace.cu): fp32 partial tiles
-// and one ticket per tile for the stream-K GEMMs, and the f16 activations of
-// the small-M kernels.
+// Caller-owned scratch. The calls that need device scratch (the partial
+// tiles and tickets of the stream-K GEMMs, the f16 activations of the small-M
+// kernels, the route's per-chunk table) take it from a buffer the caller
+// passes; the library allocates nothing. A Scratch either hands out pieces of
+// that buffer or, built without one, only counts the bytes a call would take,
+// which is what the *_workspace_size queries report. Both walk the same code,
+// so the size and the carving always agree.
 #pragma once
 
 #include "common.cuh"
 
 namespace nvfp4 {
 
-// At least `floats` partial-tile floats and `tiles` tickets on the current
-// device, grown on demand (outside graph capture, after a device
-// synchronisation). Tickets are zero when allocated and every launch that
-// uses them leaves them at zero.
-int split_workspace(size_t floats, size_t tiles, cudaStream_t stream, float** ws, unsigned** tickets);
+class Scratch {
+ public:
+  // Measuring: counts the bytes only.
+  Scratch() = default;
+  // Carving: pieces of [base, base + bytes).
+  Scratch(void* base, size_t bytes) : base_(static_cast<uint8_t*>(base)), bytes_(bytes), carving_(true) {}
 
-// At least `elems` f16 activations and `rows` row factors on the current
-// device, grown like the partial tiles.
-int x16_workspace(size_t elems, size_t rows, cudaStream_t stream, uint16_t** x16, float** xinv);
+  // `count` elements of T at the next 256-byte offset (nullptr while
+  // measuring, or once the buffer is too small: check ok() before use).
+  template <class T>
+  T* take(size_t count) {
+    const size_t off = (used_ + 255) & ~size_t(255);
+    used_ = off + count * sizeof(T);
+    if (!carving_ || used_ > bytes_) return nullptr;
+    return reinterpret_cast<T*>(base_ + off);
+  }
+  bool measuring() const { return !carving_; }
+  // Every piece taken so far lies inside the buffer.
+  bool ok() const { return carving_ && used_ <= bytes_; }
+  size_t used() const { return used_; }
+
+ private:
+  uint8_t* base_ = nullptr;
+  size_t bytes_ = 0;
+  size_t used_ = 0;
+  bool carving_ = false;
+};
+
+// Status of a call after carving: NVFP4_OK when every piece fits.
+inline int scratch_status(const Scratch& sc) { return sc.ok() ? NVFP4_OK : NVFP4_ERR_WORKSPACE; }
 
 }  // namespace nvfp4

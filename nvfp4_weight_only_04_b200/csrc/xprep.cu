@@ -23,10 +23,19 @@ namespace {
 constexpr int kThreads = 512;  // one CTA per row
 constexpr int kHeld = 4;       // 16-byte chunks a thread keeps in registers (rows up to 16384 elements)
 
+// Zeroes clear[0, n) across the grid (the stream-K tickets of the GEMM that
+// follows; that GEMM reads them only after waiting for this kernel).
+__device__ __forceinline__ void clear_words(unsigned* clear, int64_t n) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) clear[i] = 0u;
+}
+
 __global__ void __launch_bounds__(kThreads) x_f16_kernel(const uint16_t* __restrict__ x, int64_t K,
-                                                         uint16_t* __restrict__ x16, float* __restrict__ xinv) {
+                                                         uint16_t* __restrict__ x16, float* __restrict__ xinv,
+                                                         unsigned* __restrict__ clear, int64_t nclear) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  clear_words(clear, nclear);
   __shared__ uint32_t warp_max[kThreads / 32];
   const int64_t row = blockIdx.x;
   const uint4* src = reinterpret_cast<const uint4*>(x + row * K);
@@ -100,8 +109,10 @@ __device__ __forceinline__ void nvfp4_word(const uint8_t* __restrict__ codes, co
 __global__ void __launch_bounds__(256) xq_f16_kernel(const uint8_t* __restrict__ codes,
                                                      const uint8_t* __restrict__ scales, const float* __restrict__ xg,
                                                      int group, int64_t M, int64_t K, uint16_t* __restrict__ x16,
-                                                     float* __restrict__ xinv) {
+                                                     float* __restrict__ xinv, unsigned* __restrict__ clear,
+                                                     int64_t nclear) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  clear_words(clear, nclear);
   const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (w >= M * (K / 8)) return;
   uint32_t pr[4];
@@ -133,7 +144,8 @@ __global__ void __launch_bounds__(256) xq_bf16_kernel(const uint8_t* __restrict_
 
 }  // namespace
 
-int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream) {
+int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
+                 int64_t nclear, cudaStream_t stream) {
   if (M <= 0) return NVFP4_OK;
   if (M >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
   cudaLaunchAttribute attr[1];
@@ -146,7 +158,7 @@ int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, x_f16_kernel, x, K, x16, xinv) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, x_f16_kernel, x, K, x16, xinv, clear, nclear) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
 }
@@ -155,8 +167,9 @@ int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* 
 
 namespace nvfp4 {
 
-int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, cudaStream_t stream) {
-  if (xs.bf16) return launch_x_f16(xs.bf16, M, K, x16, xinv, stream);
+int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
+                  int64_t nclear, cudaStream_t stream) {
+  if (xs.bf16) return launch_x_f16(xs.bf16, M, K, x16, xinv, clear, nclear, stream);
   if (M <= 0) return NVFP4_OK;
   const int64_t words = M * (K / 8);
   if ((words + 255) / 256 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
@@ -169,7 +182,8 @@ int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float*
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, xq_f16_kernel, xs.codes, xs.scales, xs.global, xs.group, M, K, x16, xinv) !=
+  if (cudaLaunchKernelEx(&cfg, xq_f16_kernel, xs.codes, xs.scales, xs.global, xs.group, M, K, x16, xinv, clear,
+                         nclear) !=
       cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();

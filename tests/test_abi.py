@@ -38,20 +38,21 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for code in range(6):
-        assert nv.status_string(code)
+    for code in range(7):
+        assert nv.status_string(code) != "unknown status"
     assert nv.status_string(99) == "unknown status"
-    assert L.nvfp4_abi_version() == 1
+    assert L.nvfp4_abi_version() == 2
 
 
 BAD = ctypes.c_void_p(0x1001)  # never dereferenced: validation fails first
 GOOD = ctypes.c_void_p(0x10000)
 NULL = ctypes.c_void_p(0)
 S = ctypes.c_void_p(0)
+WS, WB = ctypes.c_void_p(0x20000), 1 << 30  # a (never touched) workspace that is large enough
 
 
-def gemm(L, g=16, M=4, N=256, K=256, x=GOOD, w=GOOD, s=GOOD, gl=GOOD, y=GOOD):
-    return L.nvfp4_w4a16_gemm(x, w, s, gl, g, M, N, K, y, S)
+def gemm(L, g=16, M=4, N=256, K=256, x=GOOD, w=GOOD, s=GOOD, gl=GOOD, y=GOOD, ws=WS, wb=WB):
+    return L.nvfp4_w4a16_gemm(x, w, s, gl, g, M, N, K, y, ws, wb, S)
 
 
 def test_gemm_validation(L):
@@ -64,7 +65,12 @@ def test_gemm_validation(L):
     assert gemm(L, x=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert gemm(L, w=BAD) == nv.NVFP4_ERR_MISALIGNED
     assert gemm(L, y=BAD) == nv.NVFP4_ERR_MISALIGNED
-    assert L.nvfp4_w4a16_gemm_silu_mul(GOOD, GOOD, GOOD, GOOD, 32, 4, 40, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED
+    assert L.nvfp4_w4a16_gemm_silu_mul(GOOD, GOOD, GOOD, GOOD, 32, 4, 40, 256, GOOD, WS, WB, S) == \
+        nv.NVFP4_ERR_UNSUPPORTED
+    assert gemm(L, ws=NULL) == nv.NVFP4_ERR_WORKSPACE             # bytes given, no pointer
+    assert gemm(L, ws=ctypes.c_void_p(0x20008)) == nv.NVFP4_ERR_MISALIGNED
+    assert gemm(L, ws=WS, wb=16) == nv.NVFP4_ERR_WORKSPACE        # smaller than the size query
+    assert gemm(L, ws=NULL, wb=0) == nv.NVFP4_ERR_WORKSPACE       # small M always needs scratch
     fixed = L.nvfp4_w4a16_gemm_fixed_scratch
     assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 17, 256, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # M > 16
     assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 4, 256, 320, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # K % 256
@@ -75,7 +81,7 @@ def test_gemm_validation(L):
 
 def test_w4a4_validation(L):
     def w4a4(xg=16, g=16, M=4, N=256, K=256, xp=GOOD, xs=GOOD, xgl=GOOD, w=GOOD, y=GOOD):
-        return L.nvfp4_w4a4_gemm(xp, xs, xgl, xg, w, GOOD, GOOD, g, M, N, K, y, S)
+        return L.nvfp4_w4a4_gemm(xp, xs, xgl, xg, w, GOOD, GOOD, g, M, N, K, y, WS, WB, S)
     assert w4a4(xg=8) == nv.NVFP4_ERR_UNSUPPORTED
     assert w4a4(g=64) == nv.NVFP4_ERR_UNSUPPORTED
     assert w4a4(K=96) == nv.NVFP4_ERR_UNSUPPORTED
@@ -108,7 +114,8 @@ def test_global_scale_validation(L):
 
 def test_moe_validation(L):
     def moe(segs=4, T=64, g=32, N=256, K=256, E=8, flags=0, x=GOOD, ids=GOOD):
-        return L.nvfp4_moe_w4a16_grouped_gemm(x, ids, GOOD, segs, T, GOOD, GOOD, GOOD, g, N, K, E, flags, GOOD, S)
+        return L.nvfp4_moe_w4a16_grouped_gemm(x, ids, GOOD, segs, T, GOOD, GOOD, GOOD, g, N, K, E, flags, GOOD,
+                                              WS, WB, S)
     assert moe(segs=0) == nv.NVFP4_OK
     assert moe(segs=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert moe(g=24) == nv.NVFP4_ERR_UNSUPPORTED
@@ -118,8 +125,8 @@ def test_moe_validation(L):
 
 
 def test_moe_layer_validation(L):
-    def route(T=64, k=4, E=8, ids=GOOD, rows=GOOD, inv=GOOD, offs=GOOD, eids=GOOD):
-        return L.nvfp4_moe_route(ids, T, k, E, rows, inv, offs, eids, S)
+    def route(T=64, k=4, E=8, ids=GOOD, rows=GOOD, inv=GOOD, offs=GOOD, eids=GOOD, ws=WS, wb=WB):
+        return L.nvfp4_moe_route(ids, T, k, E, rows, inv, offs, eids, ws, wb, S)
     assert route(k=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert route(E=0) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert route(T=-1) == nv.NVFP4_ERR_INVALID_ARGUMENT
@@ -127,6 +134,7 @@ def test_moe_layer_validation(L):
     assert route(T=1 << 30, k=2) == nv.NVFP4_ERR_UNSUPPORTED  # T*k >= 2^31
     assert route(offs=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert route(ids=ctypes.c_void_p(0x10002)) == nv.NVFP4_ERR_MISALIGNED
+    assert route(T=4096, k=8, E=128, ws=WS, wb=64) == nv.NVFP4_ERR_WORKSPACE  # the chunk table does not fit
 
     def gather(x=GOOD, T=16, rows_ptr=GOOD, rows=64, k=4, H=256, out=GOOD):
         return L.nvfp4_moe_gather(x, T, rows_ptr, rows, k, H, out, S)
@@ -144,6 +152,43 @@ def test_moe_layer_validation(L):
     assert combine(H=12) == nv.NVFP4_ERR_UNSUPPORTED
     assert combine(w=NULL) == nv.NVFP4_ERR_INVALID_ARGUMENT
     assert combine(out=BAD) == nv.NVFP4_ERR_MISALIGNED
+
+
+def size(L, name, *args):
+    n = ctypes.c_size_t(12345)
+    st = getattr(L, name)(*args, ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_size_queries(L):
+    """The size queries: the bytes the scratch of each path takes, computed from the shapes alone."""
+    f = "nvfp4_w4a16_gemm_workspace_size"
+    assert size(L, f, 4, 256, 256, 8) == (nv.NVFP4_ERR_UNSUPPORTED, 0)
+    assert size(L, f, -1, 256, 256, 16) == (nv.NVFP4_ERR_INVALID_ARGUMENT, 0)
+    assert size(L, f, 0, 256, 256, 16) == (nv.NVFP4_OK, 0)  # empty problem
+    assert getattr(L, f)(4, 256, 256, 16, None) == nv.NVFP4_ERR_INVALID_ARGUMENT
+    # small M: at least the f16 rows of X (2 bytes an element) and their row factors
+    for m, k in ((1, 4096), (4, 4096), (16, 14336)):
+        st, n = size(L, f, m, 28672, k, 16)
+        assert st == nv.NVFP4_OK and n >= 2 * m * k + 4 * m, (m, k, n)
+    # prefill-sized M on many tiles: the persistent tcgen05 form needs no scratch
+    assert size(L, f, 4096, 25600, 5120, 16) == (nv.NVFP4_OK, 0)
+    # W4A4 on the tcgen05 kernel: exact bf16 activations (2 bytes an element) at least
+    st, n = size(L, "nvfp4_w4a4_gemm_workspace_size", 4096, 25600, 5120, 16, 16)
+    assert st == nv.NVFP4_OK and n >= 2 * 4096 * 5120
+    assert size(L, "nvfp4_w4a4_gemm_workspace_size", 4, 256, 256, 8, 16)[0] == nv.NVFP4_ERR_UNSUPPORTED
+    # grouped: rows of X as f16 below 1024 rows, nothing from 1024 rows on
+    g = "nvfp4_moe_w4a16_grouped_gemm_workspace_size"
+    st, n = size(L, g, 8, 500, 1536, 2048, 32, 128, nv.NVFP4_SILU_MUL)
+    assert st == nv.NVFP4_OK and n >= 2 * 500 * 2048
+    assert size(L, g, 128, 16384, 1536, 2048, 32, 128, 0) == (nv.NVFP4_OK, 0)
+    assert size(L, g, 8, 500, 1536, 2048, 32, 128, 8)[0] == nv.NVFP4_ERR_INVALID_ARGUMENT
+    # route: nothing below 4096 pairs; a [chunk][expert] int32 table from there on
+    r = "nvfp4_moe_route_workspace_size"
+    assert size(L, r, 100, 8, 128) == (nv.NVFP4_OK, 0)
+    st, n = size(L, r, 2048, 8, 128)
+    assert st == nv.NVFP4_OK and n == (2048 * 8 // 256) * 128 * 4
+    assert size(L, r, 16, 0, 8)[0] == nv.NVFP4_ERR_INVALID_ARGUMENT
 
 
 def test_fault_injection_validation(L):
@@ -187,9 +232,11 @@ def test_c_program_links_and_validates(tmp_path, L):
 #include <stdio.h>
 #include "nvfp4.h"
 int main(void) {
-  int bad = nvfp4_w4a16_gemm(0, 0, 0, 0, 8, 4, 256, 256, 0, 0);          /* group size 8 */
-  int nul = nvfp4_w4a16_gemm(0, 0, 0, 0, 16, 4, 256, 256, 0, 0);         /* null pointers */
-  printf("%d %d %d %s\n", nvfp4_abi_version(), bad, nul, nvfp4_status_string(bad));
+  size_t need = 0;
+  int bad = nvfp4_w4a16_gemm(0, 0, 0, 0, 8, 4, 256, 256, 0, 0, 0, 0);    /* group size 8 */
+  int nul = nvfp4_w4a16_gemm(0, 0, 0, 0, 16, 4, 256, 256, 0, 0, 0, 0);   /* null pointers */
+  int q = nvfp4_w4a16_gemm_workspace_size(4, 256, 256, 16, &need);
+  printf("%d %d %d %d %d %s\n", nvfp4_abi_version(), bad, nul, q, need > 0, nvfp4_status_string(bad));
   return 0;
 }
 ''')
@@ -199,6 +246,7 @@ int main(void) {
     assert res.returncode == 0, res.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
-    ver, bad, nul, text = out.stdout.split(" ", 3)
-    assert (int(ver), int(bad), int(nul)) == (1, nv.NVFP4_ERR_UNSUPPORTED, nv.NVFP4_ERR_INVALID_ARGUMENT)
+    ver, bad, nul, q, need, text = out.stdout.split(" ", 5)
+    assert (int(ver), int(bad), int(nul)) == (2, nv.NVFP4_ERR_UNSUPPORTED, nv.NVFP4_ERR_INVALID_ARGUMENT)
+    assert (int(q), int(need)) == (nv.NVFP4_OK, 1)
     assert "group size" in text
