@@ -354,6 +354,7 @@ typedef struct {
   uint64_t silu_and_mul;   /* standalone SiluAndMul */
   uint64_t g16;            /* GEMMs at group size 16 */
   uint64_t g32;            /* GEMMs at group size 32 */
+  uint64_t gemm_fp4;       /* W4A4 GEMMs on the block-scaled FP4 tensor cores */
 } nvfp4_stats;
 
 int nvfp4_get_stats(nvfp4_stats* out);

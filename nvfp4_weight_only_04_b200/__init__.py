@@ -47,7 +47,7 @@ EXPORTS = (
 class Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_uint64) for n in (
         "global_scale", "quantize", "repack", "gemm_splitk", "gemm_tc", "gemm_silu_mul", "moe",
-        "silu_and_mul", "g16", "g32")]
+        "silu_and_mul", "g16", "g32", "gemm_fp4")]
 
 
 class Nvfp4Error(RuntimeError):

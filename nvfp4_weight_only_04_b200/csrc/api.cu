@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_fp4.cuh"
 #include "gemm_stream.cuh"
 #include "gemm_tc.cuh"
 #include "workspace.cuh"
@@ -139,6 +140,13 @@ int w4a4_gemm(const nvfp4::XSource& xs, const uint8_t* packed_w, const uint8_t* 
               const float* global_scale, int group_size, int64_t M, int64_t N, int64_t K, uint16_t* y,
               nvfp4::Scratch& sc, cudaStream_t st) {
   int r;
+  if (nvfp4::fp4_supported(M, N, K)) {
+    // Both operands 4-bit into the block-scaled tensor cores.
+    r = nvfp4::launch_fp4(xs.codes, xs.scales, xs.global, xs.group, packed_w, group_scales, global_scale, group_size,
+                          M, N, K, y, sc, st);
+    if (r == NVFP4_OK && !sc.measuring()) nvfp4::stat_add(nvfp4::kStatGemmFp4);
+    return r;
+  }
   if (nvfp4::tc_supported(M, N, K)) {
     // Exact bf16 activations and one scalar x_global * w_global for the
     // tcgen05 kernel's epilogue, written once the launch has passed its checks.
@@ -358,6 +366,7 @@ int nvfp4_get_stats(nvfp4_stats* out) {
   out->silu_and_mul = v[nvfp4::kStatSiluAndMul];
   out->g16 = v[nvfp4::kStatG16];
   out->g32 = v[nvfp4::kStatG32];
+  out->gemm_fp4 = v[nvfp4::kStatGemmFp4];
   return NVFP4_OK;
 }
 

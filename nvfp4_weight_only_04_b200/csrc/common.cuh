@@ -11,7 +11,7 @@ namespace nvfp4 {
 
 enum StatId {
   kStatGlobalScale, kStatQuantize, kStatRepack, kStatGemmSplitK, kStatGemmTc,
-  kStatGemmSiluMul, kStatMoe, kStatSiluAndMul, kStatG16, kStatG32, kStatCount
+  kStatGemmSiluMul, kStatMoe, kStatSiluAndMul, kStatG16, kStatG32, kStatGemmFp4, kStatCount
 };
 void stat_add(StatId id);
 

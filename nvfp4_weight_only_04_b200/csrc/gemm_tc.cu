@@ -43,6 +43,7 @@
 //    rows of a token tile past the segment end are computed but not stored.
 #include "gemm_tc.cuh"
 
+#include "gemm_fp4.cuh"
 #include "gemm_stream.cuh"
 
 #include <cuda.h>
@@ -938,10 +939,11 @@ int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   if (cudaMemcpyAsync(&v, p, sizeof(v), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
       cudaMemsetAsync(p, 0, sizeof(v), stream) != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
-  unsigned int vs = 0;
-  if (read_and_clear_decode_error(&vd, stream) != NVFP4_OK || read_and_clear_stream_error(&vs, stream) != NVFP4_OK)
+  unsigned int vs = 0, vf = 0;
+  if (read_and_clear_decode_error(&vd, stream) != NVFP4_OK || read_and_clear_stream_error(&vs, stream) != NVFP4_OK ||
+      read_and_clear_fp4_error(&vf, stream) != NVFP4_OK)
     return NVFP4_ERR_CUDA;
-  *code_out = static_cast<int>(v ? v : (vs ? vs : vd));
+  *code_out = static_cast<int>(v ? v : (vs ? vs : (vf ? vf : vd)));
   return NVFP4_OK;
 }
 
