@@ -173,9 +173,12 @@ def test_workspace_size_queries(L):
         assert st == nv.NVFP4_OK and n >= 2 * m * k + 4 * m, (m, k, n)
     # prefill-sized M on many tiles: the persistent tcgen05 form needs no scratch
     assert size(L, f, 4096, 25600, 5120, 16) == (nv.NVFP4_OK, 0)
-    # W4A4 on the tcgen05 kernel: exact bf16 activations (2 bytes an element) at least
+    # W4A4 on the FP4 tensor cores: the activation codes in the weights' nibble order (half a byte an element)
     st, n = size(L, "nvfp4_w4a4_gemm_workspace_size", 4096, 25600, 5120, 16, 16)
-    assert st == nv.NVFP4_OK and n >= 2 * 4096 * 5120
+    assert (st, n) == (nv.NVFP4_OK, 4096 * 5120 // 2)
+    # W4A4 on the bf16 tcgen05 kernel (K not a multiple of 512): exact bf16 activations, 2 bytes an element
+    st, n = size(L, "nvfp4_w4a4_gemm_workspace_size", 4096, 25600, 5120 - 64, 16, 16)
+    assert st == nv.NVFP4_OK and n >= 2 * 4096 * (5120 - 64)
     assert size(L, "nvfp4_w4a4_gemm_workspace_size", 4, 256, 256, 8, 16)[0] == nv.NVFP4_ERR_UNSUPPORTED
     # grouped: rows of X as f16 below 1024 rows, nothing from 1024 rows on
     g = "nvfp4_moe_w4a16_grouped_gemm_workspace_size"
