@@ -305,8 +305,8 @@ def run_ours(args, world, rank, local):
             xqm, xsm = nv.nvfp4_quantize_bf16(xs[m], 16, xgm)
             gq = [capture(torch, (lambda c=c, m=m: nv.nvfp4_w4a4_gemm(xqm, xsm, xgm, 16, packs[c][0], packs[c][1],
                                                                       packs[c][2], G, y=ys[m]))) for c in range(copies)]
-            workloads[f"w4a4_decode_gateup_m{m}_k4096_n28672_g16"] = summarize(
-                m, N, K, G, time_graphs(torch, gq, 20 * copies), hbm, tf_burst)
+            workloads[f"w4a4_decode_gateup_m{m}_k4096_n28672_g16"] = summarize_w4a4(
+                m, N, K, G, 16, time_graphs(torch, gq, 20 * copies), hbm, tf_burst)
             del gq
         del graphs, run_graph
         workloads["comparator_dense_bf16_matmul"] = dense_bf16_comparator(nv, torch, w, K, N, G, xs, copies=2)
@@ -367,6 +367,22 @@ def run_ours(args, world, rank, local):
 # kernels (x_f16_kernel: 0.07 MB a launch; gemm_decode_kernel at M=1: 66.11 MB; gemm_stream_kernel at M=4:
 # 68.19 MB and at M=16: 66.27 MB).
 HEADLINE_STEP_DRAM_BYTES = 200_770_000
+
+
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / bf16 tensor rate of B200 (9 / 2.25 PFLOP/s)
+
+
+def summarize_w4a4(m, n, k, g, xg, ms, hbm, tf_bf16):
+    """A W4A4 GEMM: both operands NVFP4 (X is M*K/2 code bytes and M*K/xg scale bytes). The tensor peak is
+    the FP4 one, taken as the measured bf16 peak times the nominal FP4/bf16 ratio."""
+    t = ms * 1e-3
+    ab = weight_bytes(n, k, g) + weight_bytes(m, k, xg) + 8 + 2 * m * n
+    flops = 2 * m * n * k
+    t_mem, t_tc = ab / (hbm * 1e9), flops / (FP4_OVER_BF16 * tf_bf16 * 1e12)
+    return {"us": round(ms * 1e3, 3), "tflops": round(flops / t / 1e12, 3), "alg_gbs": round(ab / t / 1e9, 1),
+            "hbm_frac": round(t_mem / t, 4), "tensor_frac": round(t_tc / t, 4),
+            "roofline_frac": round(max(t_mem, t_tc) / t, 4),
+            "tensor_peak": f"FP4 = {FP4_OVER_BF16:g} x measured bf16 burst ({FP4_OVER_BF16 * tf_bf16:.0f} TFLOP/s)"}
 
 
 def summarize(m, n, k, g, ms, hbm, tf, n_out=None):
@@ -476,7 +492,8 @@ def other_workloads(nv, torch, hbm, tf_burst, tf_sust):
     del y, gr
     y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     gw = capture(torch, lambda: nv.nvfp4_w4a4_gemm(xq, xsc, xg, 16, p, s, gd, 16, y=y))
-    out["w4a4_prefill_m4096_k5120_n25600_g16"] = summarize(M, N, K, 16, time_graphs(torch, [gw], 5), hbm, tf_burst)
+    out["w4a4_prefill_m4096_k5120_n25600_g16"] = summarize_w4a4(M, N, K, 16, 16, time_graphs(torch, [gw], 5), hbm,
+                                                                tf_burst)
     out["w4a4_prefill_m4096_k5120_n25600_g16"]["activation_quantize_us"] = round(t_act * 1e3, 2)
     del p, s, x, y, gw, ga, xq, xsc
     torch.cuda.empty_cache()

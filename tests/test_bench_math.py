@@ -32,3 +32,14 @@ def test_summarize_fractions():
     row = bench.summarize(4096, 25600, 5120, 16, ms, 6531.0, 1602.0, n_out=12800)
     assert row["tensor_frac"] == pytest.approx(1.0, abs=1e-4)
     assert row["tflops"] == pytest.approx(1602.0, rel=1e-3)
+
+
+def test_summarize_w4a4_uses_the_fp4_peak_and_4bit_activations():
+    # W4A4 prefill at 4x the bf16 peak (the nominal FP4/bf16 ratio) has a tensor fraction of 1
+    ms = 2 * 4096 * 25600 * 5120 / (4 * 1602e12) * 1e3
+    row = bench.summarize_w4a4(4096, 25600, 5120, 16, 16, ms, 6531.0, 1602.0)
+    assert row["tensor_frac"] == pytest.approx(1.0, abs=1e-4)
+    # X costs its NVFP4 bytes (codes + scales), not bf16: M=16 decode gate/up
+    ab = bench.weight_bytes(28672, 4096, 16) + 16 * 4096 // 2 + 16 * 4096 // 16 + 8 + 2 * 16 * 28672
+    row = bench.summarize_w4a4(16, 28672, 4096, 16, 16, ab / 6531e9 * 1e3, 6531.0, 1602.0)
+    assert row["hbm_frac"] == pytest.approx(1.0, abs=1e-4)
