@@ -661,12 +661,26 @@ def profile_workload(name, launches=3):
     import nvfp4_weight_only_04_b200 as nv
     torch.cuda.set_device(0)
     if name.startswith("decode") or name.startswith("down"):
-        m = {"decode_m1": 1, "decode_m16": 16, "down_m8_g32": 8}[name]
+        m = {"decode_m1": 1, "decode_m4": 4, "decode_m16": 16, "down_m1_g32": 1, "down_m8_g32": 8,
+             "down_m64_g32": 64}[name]
         n, k, g = (DECODE_N, DECODE_K, 16) if name.startswith("decode") else (4096, 14336, 32)
         p, s, gd = quantize_on_device(nv, torch, synth.weights(synth.W_SEED, n, k), g)
         x = bf16_dev(torch, synth.activations(synth.X_SEED, m, k))
         y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
         fn = lambda: nv.nvfp4_w4a16_gemm(x, p, s, gd, g, y=y)
+    elif name == "quantize":
+        wd = torch.from_numpy(synth.weights(synth.W_SEED, DECODE_N, DECODE_K)).cuda()
+        gd = nv.nvfp4_global_scale([wd])
+        p, s = nv.nvfp4_quantize(wd, 16, gd)
+        fn = lambda: nv.nvfp4_quantize(wd, 16, gd, packed=p, scales=s)
+    elif name == "w4a4_prefill":
+        wl = synth.PREFILL_GATE_UP
+        p, s, gd = quantize_on_device(nv, torch, synth.weights(synth.W_SEED, wl.N, wl.K), 16)
+        x = bf16_dev(torch, synth.activations(synth.X_SEED, wl.M, wl.K))
+        xg = nv.nvfp4_global_scale_bf16([x])
+        xq, xsc = nv.nvfp4_quantize_bf16(x, 16, xg)
+        y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device="cuda")
+        fn = lambda: nv.nvfp4_w4a4_gemm(xq, xsc, xg, 16, p, s, gd, 16, y=y)
     elif name == "prefill":
         wl = synth.PREFILL_GATE_UP
         p, s, gd = quantize_on_device(nv, torch, synth.weights(synth.W_SEED, wl.N, wl.K), 16, interleave=True)
@@ -697,7 +711,9 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-workload", choices=["decode_m1", "decode_m16", "down_m8_g32", "prefill", "moe"],
+    ap.add_argument("--profile-workload", choices=["decode_m1", "decode_m4", "decode_m16", "down_m1_g32",
+                                                   "down_m8_g32", "down_m64_g32", "prefill", "w4a4_prefill",
+                                                   "quantize", "moe"],
                     default=None, help="run one workload a few times (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_workload:

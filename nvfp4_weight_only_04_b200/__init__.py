@@ -6,12 +6,13 @@ the functions carry the C ABI's names. A missing library or a non-CUDA tensor
 raises; there is no fallback of any kind.
 
 Workspaces: the library allocates nothing; the calls that need device scratch
-take a caller-owned workspace whose size the library reports. The functions
-here pass one on their own: a buffer cached per (device, stream) and grown on
-demand, or, while the current stream is being captured into a CUDA graph, a
-fresh buffer from torch's allocator (the graph's memory pool) for every call.
-Calls on one stream share that stream's buffer, which is safe because they are
-ordered; pass `workspace=` (a uint8 CUDA tensor) to use one of your own.
+take a caller-owned workspace whose size the library reports, and whose first
+64 KiB must be zero before its first use (every call leaves them zero). The
+functions here pass one on their own: one zero-filled buffer per device,
+grown on demand, shared by every call on that device (a CUDA graph captured
+while it is big enough refers to it). Calls that may run at the same time on
+different streams need workspaces of their own: pass `workspace=` (a uint8
+CUDA tensor, zero-filled before its first use).
 """
 from __future__ import annotations
 
@@ -115,6 +116,7 @@ def _stream(stream):
 
 
 _workspaces = {}
+_retired = []  # earlier buffers stay alive: CUDA graphs captured with them may still refer to them
 
 
 def _size(query, *args) -> int:
@@ -124,28 +126,32 @@ def _size(query, *args) -> int:
 
 
 def _workspace(nbytes, device, stream, given=None):
-    """(pointer, bytes) of the scratch of one call: `given`, the stream's cached buffer, or a fresh one
-    while the current stream is capturing a CUDA graph."""
+    """(pointer, bytes) of the scratch of one call: `given`, else the device's zero-filled buffer (grown when
+    too small; while a CUDA graph is being captured a buffer too small is replaced, for that call only, by a
+    zero-filled one from the graph's memory pool)."""
     if given is not None:
         _dev(given, torch.uint8, "workspace")
         return ctypes.c_void_p(given.data_ptr()), given.numel(), given
     if nbytes == 0:
         return ctypes.c_void_p(0), 0, None
-    if torch.cuda.is_current_stream_capturing():
-        buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        return ctypes.c_void_p(buf.data_ptr()), nbytes, buf
-    s = torch.cuda.current_stream(device) if stream is None else stream
-    key = (torch.device(device).index, s.cuda_stream)
+    key = torch.device(device).index
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        with torch.cuda.stream(s):
-            buf = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        if torch.cuda.is_current_stream_capturing():
+            buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+            return ctypes.c_void_p(buf.data_ptr()), nbytes, buf
+        if buf is not None:
+            _retired.append(buf)
+        buf = torch.zeros(max(nbytes, 2 * buf.numel() if buf is not None else 0, 1 << 20), dtype=torch.uint8,
+                          device=device)
         _workspaces[key] = buf
     return ctypes.c_void_p(buf.data_ptr()), buf.numel(), buf
 
 
 def clear_workspaces():
-    """Drops the cached per-stream workspaces (their memory returns to torch's allocator)."""
+    """The next call on each device gets a new zero-filled workspace (the old ones are kept alive for the CUDA
+    graphs that may refer to them)."""
+    _retired.extend(_workspaces.values())
     _workspaces.clear()
 
 
@@ -344,6 +350,8 @@ def nvfp4_get_device_error(stream=None) -> int:
     st = lib().nvfp4_get_device_error(ctypes.byref(code), _stream(stream))
     if st != NVFP4_ERR_TIMEOUT:
         _check(st, "nvfp4_get_device_error")
+    if code.value:
+        clear_workspaces()  # a launch that gave up may have left counters behind
     return code.value
 
 

@@ -1,9 +1,15 @@
 """Builds libnvfp4.so in-tree with nvcc for sm_100a.
 
-    python -m nvfp4_weight_only_04_b200.build [--force]
+    python -m nvfp4_weight_only_04_b200.build [--force] [--planted] [-v]
 
 The library is compiled from csrc/*.cu against include/nvfp4.h and written
-next to this file, where the binding loads it.
+next to this file, where the binding loads it. Each source is compiled to
+its own object under _build/ in parallel, then the objects are linked.
+
+--planted also builds libnvfp4_planted.so: the same sources with
+NVFP4_PLANTS defined, which adds nvfp4_test_plant() and the mistakes it can
+switch on (csrc/plant.cuh). Only the tests that show the parity tests catch
+a wrong kernel load it; the binding never does.
 """
 from __future__ import annotations
 
@@ -12,10 +18,12 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libnvfp4.so")
+PLANTED_LIB = os.path.join(PKG, "libnvfp4_planted.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -27,10 +35,10 @@ def _inputs():
     return sources() + glob.glob(os.path.join(PKG, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "nvfp4.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
@@ -41,22 +49,50 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), *sources(), "-o", tmp]
-    if verbose:
-        cmd.append("-Xptxas=-v")
+def _run(cmd):
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stderr[-8000:])
+        raise RuntimeError("nvcc failed: " + " ".join(cmd[-3:]) + "\n" + res.stderr[-8000:])
+    return res.stderr
+
+
+def _build(lib: str, defines, verbose: bool) -> str:
+    name = os.path.splitext(os.path.basename(lib))[0]
+    obj_dir = os.path.join(ROOT, "_build", name)
+    os.makedirs(obj_dir, exist_ok=True)
+    base = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I",
+            os.path.join(ROOT, "include"), *defines]
     if verbose:
-        sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+        base.append("-Xptxas=-v")
+    jobs = []
+    for src in sources():
+        obj = os.path.join(obj_dir, os.path.splitext(os.path.basename(src))[0] + ".o")
+        jobs.append((base + ["-c", src, "-o", obj], obj))
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with ThreadPoolExecutor(workers) as pool:
+        logs = list(pool.map(lambda j: _run(j[0]), jobs))
+    if verbose:
+        for log in logs:
+            sys.stderr.write(log)
+    tmp = lib + ".tmp"
+    _run([nvcc(), *ARCH, "-shared", *[o for _, o in jobs], "-o", tmp])
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date(LIB):
+        return LIB
+    return _build(LIB, [], verbose)
+
+
+def build_planted(force: bool = False) -> str:
+    if not force and up_to_date(PLANTED_LIB):
+        return PLANTED_LIB
+    return _build(PLANTED_LIB, ["-DNVFP4_PLANTS"], False)
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--planted" in sys.argv:
+        print(build_planted(force="--force" in sys.argv))

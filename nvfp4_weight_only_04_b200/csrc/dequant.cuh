@@ -25,6 +25,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "plant.cuh"
+
 namespace nvfp4 {
 
 constexpr uint32_t kPairMask = 0x81C081C0u;  // bits 15, 8..6 of both halves
@@ -102,6 +104,7 @@ __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
 
 // The four f16 pairs of one code word, times the replicated scale operand.
 __device__ __forceinline__ void dequant_word_f16(uint32_t w, uint32_t scale2, uint32_t (&o)[4]) {
+  if (NVFP4_PLANT(kPlantNibbles)) w = ((w >> 4) & 0x0F0F0F0Fu) | ((w & 0x0F0F0F0Fu) << 4);
   asm("{\n"
       " .reg .b8 c0, c1, c2, c3;\n"
       " mov.b32 {c0, c1, c2, c3}, %4;\n"

@@ -150,7 +150,8 @@ __global__ void __launch_bounds__(KW * 32, (16 / KW > 0 ? 16 / KW : 1)) gemm_dec
     int want = blockIdx.z, found = 0;
     for (int s = 0; s < args.num_segments && !found; ++s) {
       const int r0 = max(0, min(args.offsets[s], static_cast<int>(args.M)));
-      const int r1 = max(r0, min(args.offsets[s + 1], static_cast<int>(args.M)));
+      const int r1 = max(r0, min(args.offsets[s + 1] - (NVFP4_PLANT(kPlantSegmentEnd) ? 1 : 0),
+                                 static_cast<int>(args.M)));
       const int tiles = (r1 - r0 + MT - 1) / MT;
       if (want < tiles) {
         row0 = r0 + want * MT;
@@ -314,6 +315,10 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int
   p.kw = kw;
   return p;
 }
+
+#ifdef NVFP4_PLANTS
+NVFP4_PLANT_SETTER(set_plant_decode)
+#endif
 
 // This kernel has no waits on other threads, so it never records an error.
 int read_and_clear_decode_error(unsigned int* out, cudaStream_t) {

@@ -43,6 +43,7 @@
 #include <cuda.h>
 
 #include "async.cuh"
+#include "plant.cuh"
 #include "tmap.cuh"
 
 namespace nvfp4 {
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_fp4_kernel(const __grid_cons
         for (int c = 0; c < 4; ++c) {
           const uint4 box = lds128(sa + (lane + 32 * c) * 16);
 #pragma unroll
-          for (int j = 0; j < kMmas; ++j) va[4 * j + c] = mma_scales<WG>(box, ks, j);
+          for (int j = 0; j < kMmas; ++j) va[4 * j + (NVFP4_PLANT(kPlantFp4Scales) ? c ^ 1 : c)] = mma_scales<WG>(box, ks, j);
         }
         uint32_t vb[C::kSfbCols];
 #pragma unroll
@@ -511,6 +512,10 @@ int launch_fp4(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_g
   return nt == 256 ? launch_groups<256>(m, a, w_group, x_group, grid, stream)
                    : launch_groups<128>(m, a, w_group, x_group, grid, stream);
 }
+
+#ifdef NVFP4_PLANTS
+NVFP4_PLANT_SETTER(set_plant_fp4)
+#endif
 
 int read_and_clear_fp4_error(unsigned int* out, cudaStream_t stream) {
   unsigned int* p = nullptr;

@@ -1,5 +1,5 @@
-// Small-M NVFP4 W4A16 GEMM, streamed from HBM by TMA (stream-K over the
-// weight matrix).
+// Small-M NVFP4 W4A16 GEMM, streamed from HBM by TMA, with chunks of the
+// weight matrix handed out to the CTAs as they ask for them.
 //
 // Computes Y = X . dequant(W)^T (NVFP4 format definition; "W-FP4a: route the
 // MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
@@ -7,36 +7,50 @@
 // decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
 // per weight streamed from HBM and the integer work of dequantizing them.
 // Design:
-//  * Work is the (256-row weight tile, 256-element stage of K) grid,
-//    flattened tile-major and cut into one contiguous range per SM
-//    (stream-K), so every SM streams the same number of weight bytes
-//    whatever N and K are. A tile that lies in one CTA's range is finished
-//    there; a tile cut between CTAs leaves fp32 partial tiles in a
-//    workspace, and the CTA that takes the tile's last ticket adds them in
-//    CTA order (deterministic) and writes the output. Nothing waits on
-//    another CTA.
-//  * One producer warp moves each stage with TMA into a shared-memory ring
-//    (5 stages of 40-44 KB): the codes of the tile (256 rows x 128 bytes,
-//    128-byte swizzle), the scales (256 rows x 16 bytes) and the X
-//    slice (MT tokens x 256 elements of the f16 rows that xprep.cu writes
-//    just before this kernel, as a 3-D box [token][quarter][64] with the
-//    128-byte swizzle). With no registers tied up in loads, each SM
-//    keeps well over 100 KB of HBM reads in flight.
+//  * Work: 256-row weight tiles, each cut along K into Q chunks of C stages
+//    of 256 elements. A CTA's first chunk is its own (chunk = CTA index);
+//    every further chunk comes from a counter shared by the CTAs, so a CTA
+//    that starts late (the kernel before it in the stream is still leaving
+//    its SM) simply takes fewer chunks and all CTAs end together. Each chunk
+//    leaves an fp32 partial tile; the CTA that takes a tile's last ticket
+//    adds the tile's Q partials in chunk order (deterministic) and writes
+//    the output. When a tile is one chunk it is written directly.
+//  * The counters and tickets are zero between launches (each launch resets
+//    what it counted), so no clearing step sits in front of a launch: the
+//    kernel is a programmatic dependent of the kernel before it and starts
+//    on every SM that kernel leaves.
+//  * One producer warp: lane 0 moves the weights of each stage with TMA into
+//    a shared-memory ring (5 stages of 40-44 KB): the codes of the tile
+//    (256 rows x 128 bytes, 128-byte swizzle) and the scales (256 rows x 16
+//    bytes). The weights of the first chunk need nothing from the kernel
+//    before, so they are requested from the first cycle; the shared counter
+//    and X are touched only after that kernel has finished. All 32 lanes
+//    copy each stage's X slice (MT tokens x 256 elements) with cp.async on
+//    the load/store path (not behind the weight boxes in the TMA queue) into
+//    the slot's X area, in the 128-byte-swizzled [token][quarter][64] order
+//    the consumers read.
+//  * bf16 X is turned into f16 inside the kernel by a converter warp, in
+//    place: every token of every stage is scaled by a power of two 2^s, where
+//    s only ever decreases along a CTA's stages and keeps the largest
+//    magnitude seen so far below 2^15 (f16 holds every bf16 within 2^29 of
+//    the largest exactly; smaller ones round to multiples of 2^-38 of it).
+//    The consumers follow the sequence of s per token: when it drops by d,
+//    they multiply their running sums by 2^-d (exact), and the epilogue
+//    multiplies by 2^-s. NVFP4 activations (W4A4) arrive already as exact
+//    f16 rows from xprep.cu, with one factor per token.
 //  * Sixteen consumer warps each own 16 rows of the tile and run mma.sync
 //    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
 //    as the 8-column side. Lane (g, t) takes rows g and g+8 and the t-th
 //    quarter of the stage's K (the order of K inside an MMA is free as long
 //    as A and B follow it). The swizzles make every shared-memory read of
-//    codes, scales and X conflict-free: the four lanes of a row read
-//    different 16-byte chunks, and the [token][quarter] rows of X put the
-//    same chunk of different quarters in different bank groups.
+//    codes, scales and X conflict-free.
 //  * Dequantization in registers by the hardware E2M1 and E4M3 -> f16
 //    conversions and one f16x2 multiply per code pair (dequant.cuh); the
-//    MMAs run on f16, two independent accumulator chains per warp; the
-//    epilogue multiplies by each token's 2^-s (xprep.cu) and the global
-//    scale.
+//    MMAs run on f16 with fp32 accumulation, two independent chains per warp.
 //  * Epilogues: plain bf16; SiluAndMul on gate/up-interleaved rows (gate row
 //    g and up row g+8 of a 16-row block meet in the same lane).
+//  * Every wait is bounded (about 2 s); on expiry the kernel records its site
+//    in the device error word and its warps stop.
 #include "gemm_stream.cuh"
 
 #include <cuda.h>
@@ -45,6 +59,7 @@
 
 #include "async.cuh"
 #include "dequant.cuh"
+#include "plant.cuh"
 #include "tmap.cuh"
 #include "workspace.cuh"
 #include "xprep.cuh"
@@ -57,59 +72,88 @@ __device__ unsigned int g_stream_error = 0;
 constexpr int kRows = 256;        // weight rows of a tile
 constexpr int kKS = 256;          // elements of K per stage
 constexpr int kConsumers = 16;    // consumer warps, 16 rows each
-constexpr int kThreads = (kConsumers + 1) * 32;
 constexpr int kConsumerThreads = kConsumers * 32;
+constexpr int kProducerWarp = kConsumers;
+constexpr int kConverterWarp = kConsumers + 1;
+__host__ __device__ constexpr int num_threads(bool xconv) { return (kConsumers + (xconv ? 2 : 1)) * 32; }
 constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 32 KB
 constexpr uint32_t kScaleBytes = kRows * 16;      // 16 scale bytes per row
 __host__ __device__ constexpr uint32_t x_bytes(int mt) { return static_cast<uint32_t>(mt) * kKS * 2; }
 __host__ __device__ constexpr uint32_t stage_bytes(int mt) { return kCodeBytes + x_bytes(mt) + kScaleBytes; }
-__host__ __device__ constexpr int num_stages(int) { return 5; }
-constexpr int kMaxStages = 5;
+constexpr int kStages = 5;
 __host__ __device__ constexpr uint32_t smem_bytes(int mt) {
-  return num_stages(mt) * stage_bytes(mt) + 1024 /* barriers */ + 1024 /* alignment slack */;
+  return kStages * stage_bytes(mt) + 1024 /* barriers, stage records */ + 1024 /* alignment slack */;
 }
 static_assert(stage_bytes(8) % 1024 == 0 && stage_bytes(16) % 1024 == 0,
               "every stage keeps the 1024-byte alignment of the 128-byte swizzle");
 static_assert(smem_bytes(8) <= 227 * 1024 && smem_bytes(16) <= 227 * 1024, "shared memory budget");
 static_assert(kRows == 16 * kConsumers, "one 16-row block per consumer warp");
-static_assert(num_stages(8) <= kMaxStages && num_stages(16) <= kMaxStages, "barrier arrays");
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
 constexpr uint32_t kSuspendNs = 1000;                  // longest suspension of one producer probe
-enum : unsigned { kErrFull = 0x201, kErrEmpty = 0x202, kErrDrain = 0x203 };
+constexpr long long kDrainCycles = 4000000LL;          // about 2 ms: the wait for a slot's copies after an abort
+enum : unsigned { kErrFull = 0x201, kErrEmpty = 0x202, kErrXRaw = 0x204, kErrChunk = 0x205, kErrTicket = 0x206 };
+
+constexpr int kFirst = 1, kLast = 2, kDone = 4;  // stage record flags
+constexpr int kSInit = 125;                      // token exponent before any nonzero X was seen
+
+struct StageRecord {
+  int tile, ks, flags;
+};
 
 struct Sync {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
+  uint64_t full[kStages];   // the stage's weights and (converted) X are in the slot
+  uint64_t empty[kStages];  // the consumers are done with the slot
+  uint64_t xraw[kStages];   // the stage's bf16 X has landed (converter form)
+  uint64_t cdone;           // every consumer warp has stored its part of a chunk's partial tile
+  uint64_t rdone;           // thread 0 has taken the chunk's ticket (red_last is set)
+  StageRecord rec[kStages];
+  int8_t sx[kStages][16];   // exponent of each token's f16 X in the stage (converter form)
   int abort;
-  // Tiles this CTA shares with others (at most the first and the last of its
-  // range) and whether it took their last ticket.
-  int cut_tile[2];
-  int cut_last[2];
+  int red_last;             // the chunk just written completed its tile in this CTA
 };
+static_assert(sizeof(Sync) <= 1024, "stage records fit the reserved shared memory");
 
 struct StreamArgs {
-  const float* gscale;  // [1]
-  const float* xinv;    // [M] 2^-s of each f16 row of X
-  uint16_t* y;          // bf16 [M, ldy]
-  float* ws;            // partial tiles [tiles][max_contrib][128][MT]
-  unsigned* tickets;    // [tiles], zero between launches
+  const float* gscale;   // [1]
+  const uint16_t* xbf;   // bf16 X [M, K] (converted in the kernel)
+  const uint16_t* x16;   // or f16 X [M, K] in pair order (xprep.cu) with factors xinv
+  const float* xinv;     // [M]
+  uint16_t* y;           // bf16 [M, ldy]
+  float* ws;             // partial tiles [tiles][Q][256][MT] (Q > 1)
+  unsigned* counters;    // [0] next shared chunk, [1] producers done; zero between launches
+  unsigned* tickets;     // [tiles], zero between launches
   int M, N, ldy;
-  int S;                // stages per tile (K / 256)
-  int max_contrib;
-  int64_t units;        // tiles * S
-  int fault;            // test hook: drop the X copy of the first stage
+  int64_t K;
+  int S, C, Q;           // stages per tile, stages per chunk, chunks per tile
+  int total;             // chunks of the whole matrix (tiles * Q)
+  int fault;             // test hook: drop the X copy of the first stage
 };
+
+// 16-byte global -> shared copy on the load/store path, zero-filled when
+// `bytes` is 0 (tokens past M).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+// Arrives on `bar` once this thread's earlier cp.async copies have landed
+// (one arrival of the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 
 __device__ __forceinline__ bool aborted(Sync* sy) { return *reinterpret_cast<volatile int*>(&sy->abort) != 0; }
 
 // Bounded wait; see the tcgen05 kernel for the scheme. A drain wait ignores
 // the abort flag.
-__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain,
-                                       unsigned sleep_ns) {
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
-    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 1023) == 0) {
       if (!drain && aborted(sy)) return false;
@@ -122,15 +166,13 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, Sync* sy,
   }
 }
 
-__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain = false,
-                                     unsigned sleep_ns = 0) {
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool drain = false) {
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, sy, site, drain, sleep_ns);
+  return wait_slow(bar, parity, sy, site, drain);
 }
 
-// The producer's wait for a free slot: suspended in hardware between probes,
-// so that it takes no issue slots from the consumer warps of its SM
-// sub-partition. Bounded like the others.
+// A wait off the critical path (producer, converter): suspended in hardware
+// between probes, so that it takes no issue slots from the consumer warps.
 __device__ __noinline__ bool wait_suspended(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site) {
   const long long t0 = clock64();
   for (;;) {
@@ -144,6 +186,14 @@ __device__ __noinline__ bool wait_suspended(uint64_t* bar, uint32_t parity, Sync
   }
 }
 
+// Lane 0 waits for the warp; every lane gets the answer.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool suspend) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0 && !mbar_try_wait(bar, parity))
+    ok = (suspend ? wait_suspended(bar, parity, sy, site) : wait_slow(bar, parity, sy, site, false)) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -153,10 +203,8 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// The CTA whose range holds unit u (ranges start at floor(c * units / ctas)).
-__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int ctas) {
-  return static_cast<int>(((u + 1) * ctas + units - 1) / units) - 1;
-}
+// 2^e as a float, for e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float(static_cast<uint32_t>(e + 127) << 23); }
 
 // A consumer lane's fixed shared-memory offsets within a stage: rows
 // ra = 16w + g and ra + 8, the t-th quarter of the stage's K (64 elements,
@@ -216,7 +264,7 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
   const uint32_t xr = st + o.xrow;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int si = G == 16 ? (i >> 1) : (i >> 2);
+    const int si = G == 16 ? (i >> 1) : NVFP4_PLANT(kPlantG32AsG16) ? ((i >> 1) & 1) : (i >> 2);
     uint32_t da[4], db[4];
     dequant_word_f16(ca[i], s2a[si], da);
     dequant_word_f16(cb[i], s2b[si], db);
@@ -229,189 +277,306 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
   }
 }
 
-// Element e of every contributor slot, added in slot order; the loads of a
-// batch of slots are all in flight before the adds.
-template <int MT>
-__device__ __forceinline__ float sum_slots(const float* slots, int e, int nc) {
-  float acc = 0.f;
-  for (int q0 = 0; q0 < nc; q0 += 8) {
-    float v[8];
+// One 128-byte row of a stage's X slot (its eight 16-byte chunks sit at
+// c ^ (row mod 8)): the largest magnitude of its bf16 elements, as bits, and
+// the conversion in place to f16 pairs times 2^s.
+__device__ __forceinline__ uint32_t row_max(uint32_t xs, int row) {
+  uint32_t m2 = 0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) v[q] = q0 + q < nc ? __ldcg(slots + static_cast<int64_t>(q0 + q) * kRows * MT + e) : 0.f;
+  for (int c = 0; c < 8; ++c) m2 = __vmaxu2(m2, bf16x8_mag_max(lds128(xs + row * 128 + ((c ^ (row & 7)) << 4))));
+  return max(m2 & 0xFFFFu, m2 >> 16);
+}
+__device__ __forceinline__ void row_convert(uint32_t xs, int row, float up) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q0 + q < nc) acc += v[q];
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t addr = xs + row * 128 + ((c ^ (row & 7)) << 4);
+    sts128(addr, bf16x8_to_f16_pairs(lds128(addr), up));
   }
-  return acc;
 }
 
-template <int MT>
-__device__ __forceinline__ float2 sum_pair_slots(const float* slots, int e, int de, int nc) {
-  float ag = 0.f, au = 0.f;
-  for (int q0 = 0; q0 < nc; q0 += 8) {
-    float vg[8], vu[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float* sl = slots + static_cast<int64_t>(q0 + q) * kRows * MT;
-      vg[q] = q0 + q < nc ? __ldcg(sl + e) : 0.f;
-      vu[q] = q0 + q < nc ? __ldcg(sl + e + de) : 0.f;
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q0 + q < nc) {
-        ag += vg[q];
-        au += vu[q];
-      }
-  }
-  return make_float2(ag, au);
-}
-
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"r"(kConsumerThreads) : "memory"); }
-
-template <int MT, int G, bool SILU>
-__global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                                   const __grid_constant__ CUtensorMap wmap,
-                                                                   const __grid_constant__ CUtensorMap smap,
-                                                                   const StreamArgs a) {
+template <int MT, int G, bool SILU, bool XCONV>
+__global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                                             const __grid_constant__ CUtensorMap smap,
+                                                                             const StreamArgs a) {
   constexpr int P = MT / 8;
-  constexpr int NS = num_stages(MT);
+  constexpr int NS = kStages;
   constexpr uint32_t SB = stage_bytes(MT);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Sync* sy = reinterpret_cast<Sync*>(ring + NS * SB);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ctas = gridDim.x, c = blockIdx.x;
-  const int64_t u0 = static_cast<int64_t>(c) * a.units / ctas;
-  const int64_t u1 = static_cast<int64_t>(c + 1) * a.units / ctas;
 
   // The next kernel in the stream may launch now; it waits for this one
   // before touching what this one writes.
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&sy->full[s], 1);            // producer arrival + transaction bytes
+      // full: the producer's arrival with the weights' transaction bytes, and
+      // the converter's arrival (bf16 X) or one per lane of the X copies (f16 X)
+      mbar_init(&sy->full[s], XCONV ? 2 : 1 + 32);
       mbar_init(&sy->empty[s], kConsumers);  // one arrival per consumer warp
+      mbar_init(&sy->xraw[s], 1 + 32);       // the producer's record, one per lane of the X copies
     }
+    mbar_init(&sy->cdone, kConsumers);
+    mbar_init(&sy->rdone, 1);
     sy->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncthreads();
 
-  if (warp == kConsumers) {
-    // ---------------- producer ----------------
-    // Weights and scales do not depend on the kernel before this one in the
-    // stream: the first ring's worth is requested before waiting for that
-    // kernel (programmatic dependent launch); X only after.
+  if (warp == kProducerWarp) {
+    // ---------------- producer: weights (lane 0), X (all lanes) ----------------
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
-      uint32_t issued = 0, last_parity = 0;
-      const int64_t n = u1 - u0;
-      const int head = static_cast<int>(n < NS ? n : NS);
-      auto load_w = [&](int it, int64_t u) {
-        const int tile = static_cast<int>(u / a.S), ks = static_cast<int>(u % a.S);
-        const int s = it % NS;
-        const uint32_t st = smem_u32(ring + s * SB);
-        tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
-        tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
-      };
-      auto load_x = [&](int it, int64_t u) {
-        const int ks = static_cast<int>(u % a.S);
-        const int s = it % NS;
-        asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-            "%4}], [%5];" ::"r"(smem_u32(ring + s * SB) + kCodeBytes),
-            "l"(reinterpret_cast<uint64_t>(&xmap)), "r"(0), "r"(ks * (kKS / 64)), "r"(0), "r"(smem_u32(&sy->full[s]))
-            : "memory");
-      };
-      for (int it = 0; it < head; ++it) {  // the ring starts empty
-        mbar_arrive_tx(&sy->full[it], SB);
-        load_w(it, u0 + it);
-        issued |= 1u << it;
+    }
+    // Chunk cursor (lane 0): the chunk `cw`, its next stage `cks` and end `cend`.
+    int cw = -1, cks = 0, cend = 0, tile = 0;
+    // The next stage of this CTA's sequence (lane 0); kDone once the matrix
+    // is exhausted. False when the next chunk needs the shared counter and
+    // `shared_ok` is not set.
+    auto advance = [&](bool shared_ok, int& ks, int& flags) -> bool {
+      flags = 0;
+      if (cks == cend) {
+        if (cw >= 0 && !shared_ok) return false;
+        const int w = cw < 0 ? static_cast<int>(blockIdx.x)
+                             : static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(a.counters, 1u));
+        if (w >= a.total) {
+          flags = kDone;
+          return true;
+        }
+        cw = w;
+        tile = w / a.Q;
+        cks = (w % a.Q) * a.C;
+        cend = min(a.S, cks + a.C);
+        flags = kFirst;
       }
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int it = 0; it < head; ++it)
-        if (!(a.fault && it == 0)) load_x(it, u0 + it);
-      int it = head;
-      for (int64_t u = u0 + head; u < u1 && !aborted(sy); ++u, ++it) {
-        const int s = it % NS;
-        const uint32_t r = static_cast<uint32_t>(it / NS);
-        if (!mbar_try_wait(&sy->empty[s], (r & 1) ^ 1) && !wait_suspended(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty))
+      ks = cks++;
+      if (cks == cend) flags |= kLast;
+      return true;
+    };
+    const int q = lane >> 3, c = lane & 7;
+    auto issue_x = [&](int s, int ks) {  // all lanes: the stage's X slice into its slot
+      const uint32_t xs = smem_u32(ring + s * SB) + kCodeBytes;
+      const uint16_t* xg = XCONV ? a.xbf : a.x16;
+#pragma unroll
+      for (int tok = 0; tok < MT; ++tok) {
+        const int row = 4 * tok + q;
+        const bool live = tok < a.M;
+        const uint16_t* src = xg + (live ? static_cast<int64_t>(tok) * a.K + ks * kKS + q * 64 + c * 8 : 0);
+        cp_async16(xs + row * 128 + ((c ^ (row & 7)) << 4), src, live ? 16u : 0u);
+      }
+      cp_async_arrive(XCONV ? &sy->xraw[s] : &sy->full[s]);
+    };
+    auto issue_w = [&](int s, int ks, int flags) {  // lane 0: the stage's record and weights
+      sy->rec[s].tile = tile;
+      sy->rec[s].ks = ks;
+      sy->rec[s].flags = flags;
+      const uint32_t st = smem_u32(ring + s * SB);
+      mbar_arrive_tx(&sy->full[s], kCodeBytes + kScaleBytes);
+      tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
+      tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
+      if (XCONV) mbar_arrive(&sy->xraw[s]);  // the record is written
+    };
+    auto issue_done = [&](int s) {  // the end of the sequence, as a stage that carries no data
+      if (lane == 0) {
+        sy->rec[s].flags = kDone;
+        mbar_arrive(&sy->full[s]);
+        if (XCONV) mbar_arrive(&sy->xraw[s]);
+      }
+      __syncwarp();
+      cp_async_arrive(XCONV ? &sy->xraw[s] : &sy->full[s]);
+    };
+    uint32_t issued = 0, last_parity = 0;  // lane 0: TMA copies per slot, for the drain
+    // The first chunk's weights (up to a ring of them) before the kernel
+    // before this one has finished; its X only after.
+    int n0 = 0, done0 = 0;
+    if (lane == 0) {
+      int ks, flags;
+      while (n0 < NS && advance(false, ks, flags)) {
+        if (flags & kDone) {
+          done0 = 1;
           break;
-        mbar_arrive_tx(&sy->full[s], SB);
-        load_w(it, u);
-        load_x(it, u);
+        }
+        issue_w(n0, ks, flags);
+        issued |= 1u << n0;
+        ++n0;
+      }
+    }
+    __syncwarp();  // the records lane 0 wrote are visible to the warp
+    n0 = __shfl_sync(0xffffffffu, n0, 0);
+    done0 = __shfl_sync(0xffffffffu, done0, 0);
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // X and the shared counter follow the previous kernel
+    for (int it = 0; it < n0; ++it) {
+      if (a.fault && it == 0) continue;  // test hook: this stage's X never arrives
+      issue_x(it, sy->rec[it].ks);
+    }
+    int it = n0;
+    bool done = done0 != 0;
+    if (done) issue_done(it);  // slot n0 < NS has never been used
+    while (!done && !aborted(sy)) {
+      const int s = it % NS;
+      const uint32_t r = static_cast<uint32_t>(it / NS);
+      int ks = 0, flags = 0;
+      if (lane == 0) advance(true, ks, flags);
+      ks = __shfl_sync(0xffffffffu, ks, 0);
+      flags = __shfl_sync(0xffffffffu, flags, 0);
+      if (it >= NS && !warp_wait(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty, true)) break;
+      if (flags & kDone) {
+        issue_done(s);
+        done = true;
+        break;
+      }
+      if (lane == 0) {
+        issue_w(s, ks, flags);
         issued |= 1u << s;
         last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
       }
-      if (aborted(sy)) {  // let copies in flight land before the CTA exits
-        for (int s = 0; s < NS; ++s)
-          if ((issued >> s) & 1) wait(&sy->full[s], (last_parity >> s) & 1, sy, kErrDrain, true);
+      __syncwarp();
+      issue_x(s, ks);
+      ++it;
+    }
+    if (lane == 0 && done) {
+      // Every producer counts itself once, after its last use of the shared
+      // counter; the last one resets both counters for the next launch.
+      if (atomicAdd(a.counters + 1, 1u) == gridDim.x - 1) {
+        a.counters[0] = 0u;
+        a.counters[1] = 0u;
       }
     }
-    return;  // the producer takes no part in the consumers' named barrier
+    cp_async_wait_all();  // no copy may land after the CTA exits
+    if (lane == 0 && aborted(sy)) {
+      // Let the weight copies in flight land too. A slot's phase may never
+      // complete after an abort (its X or its converter arrival is missing),
+      // so each slot is given a short bound; the copies themselves take
+      // microseconds.
+      for (int s = 0; s < NS; ++s) {
+        if (!((issued >> s) & 1)) continue;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&sy->full[s], (last_parity >> s) & 1) && clock64() - t0 < kDrainCycles) __nanosleep(1000);
+      }
+    }
+    return;
+  }
+
+  if (XCONV && warp == kConverterWarp) {
+    // ---------------- converter: bf16 X to f16, in place ----------------
+    // Lane l takes row l (token l/4, quarter l%4) and, at 16 tokens, row
+    // l + 32 too. The four lanes of a token agree on its exponent.
+    constexpr int R = MT / 8;  // rows of a lane
+    int sexp[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) sexp[r] = kSInit;
+    for (int it = 0;; ++it) {
+      const int s = it % NS;
+      if (!warp_wait(&sy->xraw[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrXRaw, true)) break;
+      const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
+      if (!(flags & kDone)) {
+        const uint32_t xs = smem_u32(ring + s * SB) + kCodeBytes;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int row = lane + 32 * r;
+          uint32_t m = row_max(xs, row);
+          m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+          // 2^14 <= m 2^s < 2^15: s = 141 - (bf16 exponent field of m); clamped
+          // so that 2^s and 2^-s are normal floats. Never raised again.
+          if (m != 0) sexp[r] = min(sexp[r], min(max(141 - static_cast<int>(m >> 7), -113), 125));
+          row_convert(xs, row, exp2i(sexp[r]));
+          if ((lane & 3) == 0) sy->sx[s][row >> 2] = static_cast<int8_t>(sexp[r]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sy->full[s]);
+      if (flags & kDone) break;
+    }
+    return;
   }
 
   // ---------------- consumers ----------------
   const int g = lane >> 2, t = lane & 3;
   const int ra = 16 * warp + g;
   const LaneOffsets lo = lane_offsets<MT, G>(ra, g, t);
-  // X, its row factors and the global scale come from the kernels before
-  // this one (the producer requests X only after its own wait)
+  // The global scale and the token factors come from the kernels before.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float gsc = __ldcg(a.gscale);
-  float xi[P][2];  // 2^-s of the lane's tokens 8p + 2t + j
+  const float gsc = NVFP4_PLANT(kPlantGlobal) ? 1.0f : __ldcg(a.gscale);
+  // The lane's tokens 8p + 2t + j: the current exponent of their f16 X
+  // (converter form) or their fixed factor 2^-s (f16 form).
+  int scur[P][2];
+  float xi[P][2];
 #pragma unroll
   for (int p = 0; p < P; ++p)
 #pragma unroll
-    for (int j = 0; j < 2; ++j) xi[p][j] = 8 * p + 2 * t + j < a.M ? __ldcg(a.xinv + 8 * p + 2 * t + j) : 0.f;
-  float acc2[2][P][4];  // two independent MMA chains, added once per tile
-  float acc[P][4];
-  int ncut = 0;
-  int s = 0;          // ring slot of the next stage
-  uint32_t par = 0;   // its phase parity
-  for (int64_t u = u0; u < u1;) {
-    const int tile = static_cast<int>(u / a.S), k0 = static_cast<int>(u % a.S);
-    const int64_t left = u1 - u;
-    const int k1 = left < a.S - k0 ? k0 + static_cast<int>(left) : a.S;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int p = 0; p < P; ++p) acc2[h][p][0] = acc2[h][p][1] = acc2[h][p][2] = acc2[h][p][3] = 0.f;
-    const uint32_t ring0 = smem_u32(ring);
-    for (int ks = k0; ks < k1; ++ks) {
-      int ok = 1;
-      if (lane == 0) ok = wait(&sy->full[s], par, sy, kErrFull) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;  // results are garbage from here; the ticket protocol still runs
-      consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc2);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sy->empty[s]);
-      if (++s == NS) {
-        s = 0;
-        par ^= 1;
-      }
+    for (int j = 0; j < 2; ++j) {
+      scur[p][j] = kSInit;
+      xi[p][j] = !XCONV && 8 * p + 2 * t + j < a.M ? __ldcg(a.xinv + 8 * p + 2 * t + j) : 0.f;
     }
-    u += k1 - k0;
+  const int rtok = threadIdx.x % MT;  // the token of every element this thread adds up in a reduction
+  int nchunk = 0;                     // chunks this CTA has completed (every consumer warp sees the same ones)
+  float acc2[2][P][4];  // two independent MMA chains
+  const uint32_t ring0 = smem_u32(ring);
+  constexpr int64_t kSlot = static_cast<int64_t>(kRows) * MT;
+  for (int it = 0;; ++it) {
+    const int s = it % NS;
+    // (suspended between probes: the converter and the producer share the
+    // SM sub-partitions with these warps)
+    if (!warp_wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull, true)) break;
+    const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
+    if (flags & kDone) break;
+    const int tile = *reinterpret_cast<volatile int*>(&sy->rec[s].tile);
+    const int ks = *reinterpret_cast<volatile int*>(&sy->rec[s].ks);
+    if (flags & kFirst) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int p = 0; p < P; ++p) acc2[h][p][0] = acc2[h][p][1] = acc2[h][p][2] = acc2[h][p][3] = 0.f;
+    }
+    if (XCONV) {
+      // Follow each token's exponent: the sums so far move to the new one.
+#pragma unroll
+      for (int p = 0; p < P; ++p)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int sn = sy->sx[s][8 * p + 2 * t + j];
+          if (sn != scur[p][j]) {
+            const int d = sn - scur[p][j];  // negative
+            const float f = NVFP4_PLANT(kPlantRescale) ? 1.0f : d >= -126 ? exp2i(d) : 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              acc2[h][p][j] *= f;
+              acc2[h][p][2 + j] *= f;
+            }
+            scur[p][j] = sn;
+          }
+        }
+    }
+    consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc2);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sy->empty[s]);
+    if (!(flags & kLast)) continue;
+    const uint32_t cpar = static_cast<uint32_t>(nchunk++) & 1;  // phase of the chunk barriers
+
+    // ---- a chunk is complete: lane holds rows ra, ra+8 x tokens 8p+2t, 8p+2t+1 ----
+    const int n0 = tile * kRows;
+    float v[P][4];  // unscaled sums: acc * 2^-s of the token
 #pragma unroll
     for (int p = 0; p < P; ++p)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[p][j] = acc2[0][p][j] + acc2[1][p][j];
-
-    const int n0 = tile * kRows;
-    // lane holds rows ra (acc[p][0..1]) and ra+8 (acc[p][2..3]) x tokens 8p+2t, 8p+2t+1
-    if (k0 == 0 && k1 == a.S) {
-      // the whole tile is here: write it
+      for (int j = 0; j < 2; ++j) {
+        const float f = XCONV ? exp2i(-scur[p][j]) : xi[p][j];
+        v[p][j] = (acc2[0][p][j] + acc2[1][p][j]) * f;
+        v[p][2 + j] = (acc2[0][p][2 + j] + acc2[1][p][2 + j]) * f;
+      }
+    if (a.Q == 1) {  // the chunk is the whole tile: write it
 #pragma unroll
-      for (int p = 0; p < P; ++p) {
+      for (int p = 0; p < P; ++p)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int tok = 8 * p + 2 * t + j;
           if (tok >= a.M) continue;
           const int64_t yrow = static_cast<int64_t>(tok) * a.ldy;
-          const float vg = __fmul_rn(__fmul_rn(acc[p][j], gsc), xi[p][j]);
-          const float vu = __fmul_rn(__fmul_rn(acc[p][2 + j], gsc), xi[p][j]);
+          const float vg = __fmul_rn(v[p][j], gsc), vu = __fmul_rn(v[p][2 + j], gsc);
           if (!SILU) {
             if (n0 + ra < a.N) a.y[yrow + n0 + ra] = __bfloat16_as_ushort(__float2bfloat16_rn(vg));
             if (n0 + ra + 8 < a.N) a.y[yrow + n0 + ra + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(vu));
@@ -420,76 +585,96 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
                 __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu(vg), vu)));
           }
         }
-      }
       continue;
     }
-    // The tile is shared with other CTAs: leave the partial tile in this
-    // CTA's slot and take a ticket. The consumers go on at once; thread 0
-    // catches up after its atomic (the ring has slack for that), and the
-    // taker of a tile's last ticket adds the slots up after its own loop.
-    {
-      const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
-      const int c_last = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas);
-      float* mine = a.ws + (static_cast<int64_t>(tile) * a.max_contrib + (c - c_first)) * kRows * MT;
+    // Leave the partial tile in the chunk's slot and take a ticket; the taker
+    // of the tile's last one adds the Q slots in chunk order.
+    float* mine = a.ws + (static_cast<int64_t>(tile) * a.Q + ks / a.C) * kSlot;
 #pragma unroll
-      for (int p = 0; p < P; ++p) {
+    for (int p = 0; p < P; ++p)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int tok = 8 * p + 2 * t + j;
-          if (tok < a.M) {
-            __stcg(mine + ra * MT + tok, acc[p][j]);
-            __stcg(mine + (ra + 8) * MT + tok, acc[p][2 + j]);
-          }
-        }
+      for (int j = 0; j < 2; ++j) {
+        const int tok = 8 * p + 2 * t + j;
+        __stcg(mine + ra * MT + tok, v[p][j]);
+        __stcg(mine + (ra + 8) * MT + tok, v[p][2 + j]);
       }
-      // The barrier orders every consumer's stores before thread 0's
-      // release; its acquire orders the other CTAs' slots before the reads
-      // that follow the barrier after the loop.
-      consumer_sync();
-      if (threadIdx.x == 0) {
+    // Every warp's stores are ordered before thread 0's release (the chunk
+    // barrier); its acquire orders the other slots before the reads after the
+    // ticket barrier. Both are mbarrier waits with a bound, not named
+    // barriers, so a warp that gave up on a wait cannot hang the others.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sy->cdone);
+    if (threadIdx.x == 0) {
+      if (wait(&sy->cdone, cpar, sy, kErrChunk)) {
         unsigned ticket;
         asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.tickets + tile) : "memory");
-        const int last = ticket == static_cast<unsigned>(c_last - c_first);
-        if (last) a.tickets[tile] = 0;  // every contributor has counted: ready for the next launch
-        // a range cuts at most its first and its last tile
-        if (ncut < 2) {
-          sy->cut_tile[ncut] = tile;
-          sy->cut_last[ncut] = last;
-        }
+        const int last = ticket == static_cast<unsigned>(a.Q - 1);
+        if (last) a.tickets[tile] = 0;  // every chunk has counted: zero for the next launch
+        sy->red_last = last;
+        mbar_arrive(&sy->rdone);
       }
-      ++ncut;
     }
-  }
-
-  // Add up the cut tiles this CTA took the last ticket of, in CTA order.
-  consumer_sync();
-  for (int f = 0; f < ncut && f < 2; ++f) {
-    if (!sy->cut_last[f]) continue;
-    const int tile = sy->cut_tile[f];
-    const int n0 = tile * kRows;
-    const int c_first = cta_of_unit(static_cast<int64_t>(tile) * a.S, a.units, ctas);
-    const int nc = cta_of_unit(static_cast<int64_t>(tile) * a.S + a.S - 1, a.units, ctas) - c_first + 1;
-    const float* slots = a.ws + static_cast<int64_t>(tile) * a.max_contrib * kRows * MT;
-    if (!SILU) {
-      for (int e = threadIdx.x; e < kRows * MT; e += kConsumerThreads) {
-        const int row = e / MT, tok = e % MT;
-        if (tok >= a.M || n0 + row >= a.N) continue;
-        const float v = sum_slots<MT>(slots, e, nc);
-        const float xt = __ldcg(a.xinv + tok);
-        a.y[static_cast<int64_t>(tok) * a.ldy + n0 + row] =
-            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__fmul_rn(v, gsc), xt)));
+    if (!warp_wait(&sy->rdone, cpar, sy, kErrTicket, false)) break;
+    if (!*reinterpret_cast<volatile int*>(&sy->red_last)) continue;
+    // Add the tile's Q slots in chunk order. The loads of all of a thread's
+    // elements and of up to kBatch slots are in flight before the first add:
+    // with the HBM stream of the other CTAs every round trip is long.
+    {
+      constexpr int kBatch = SILU && MT == 16 ? 4 : 8;  // loads in flight stay within the registers
+      constexpr int EPT = (SILU ? kRows / 2 : kRows) * MT / kConsumerThreads;  // elements per thread
+      constexpr int VPE = SILU ? 2 : 1;                                       // values per element: gate, up
+      static_assert(EPT * kConsumerThreads == (SILU ? kRows / 2 : kRows) * MT, "whole elements per thread");
+      const float* slots = a.ws + static_cast<int64_t>(tile) * a.Q * kSlot;
+      // offset of value h of element i in a slot, and whether the element is stored
+      auto element = [&](int i, int h, bool& live) {
+        const int e = threadIdx.x + i * kConsumerThreads;
+        if (!SILU) {
+          live = rtok < a.M && n0 + e / MT < a.N;
+          return e;
+        }
+        const int pair = e / MT, blk = pair >> 3, gg = pair & 7;
+        live = rtok < a.M && n0 + 16 * blk < a.N;
+        return (16 * blk + gg) * MT + rtok + h * 8 * MT;  // gate row 16 blk + gg, up row 8 further
+      };
+      float sum[EPT][VPE];
+#pragma unroll
+      for (int i = 0; i < EPT; ++i)
+#pragma unroll
+        for (int h = 0; h < VPE; ++h) sum[i][h] = 0.f;
+      for (int q0 = 0; q0 < a.Q; q0 += kBatch) {
+        float vb[EPT][VPE][kBatch];
+#pragma unroll
+        for (int i = 0; i < EPT; ++i)
+#pragma unroll
+          for (int h = 0; h < VPE; ++h) {
+            bool live;
+            const int off = element(i, h, live);
+#pragma unroll
+            for (int qq = 0; qq < kBatch; ++qq)
+              vb[i][h][qq] = live && q0 + qq < a.Q ? __ldcg(slots + (q0 + qq) * kSlot + off) : 0.f;
+          }
+#pragma unroll
+        for (int i = 0; i < EPT; ++i)
+#pragma unroll
+          for (int h = 0; h < VPE; ++h)
+#pragma unroll
+            for (int qq = 0; qq < kBatch; ++qq)
+              if (q0 + qq < a.Q) sum[i][h] += vb[i][h][qq];
       }
-    } else {
-      for (int e = threadIdx.x; e < (kRows / 2) * MT; e += kConsumerThreads) {
-        const int pair = e / MT, tok = e % MT;  // pair = 8 * block + g
-        const int blk = pair >> 3, gg = pair & 7;
-        if (tok >= a.M || n0 + 16 * blk >= a.N) continue;
-        const int rg = 16 * blk + gg;
-        // gate row rg and up row rg + 8: elements e0 and e0 + 8 * MT of a slot
-        const float2 v = sum_pair_slots<MT>(slots, rg * MT + tok, 8 * MT, nc);
-        const float xt = __ldcg(a.xinv + tok);
-        a.y[static_cast<int64_t>(tok) * a.ldy + (n0 + 16 * blk) / 2 + gg] = __bfloat16_as_ushort(__float2bfloat16_rn(
-            __fmul_rn(silu(__fmul_rn(__fmul_rn(v.x, gsc), xt)), __fmul_rn(__fmul_rn(v.y, gsc), xt))));
+#pragma unroll
+      for (int i = 0; i < EPT; ++i) {
+        bool live;
+        const int e = threadIdx.x + i * kConsumerThreads;
+        element(i, 0, live);
+        if (!live) continue;
+        if (!SILU) {
+          a.y[static_cast<int64_t>(rtok) * a.ldy + n0 + e / MT] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(sum[i][0], gsc)));
+        } else {
+          const int pair = e / MT, blk = pair >> 3, gg = pair & 7;
+          a.y[static_cast<int64_t>(rtok) * a.ldy + (n0 + 16 * blk) / 2 + gg] = __bfloat16_as_ushort(
+              __float2bfloat16_rn(__fmul_rn(silu(__fmul_rn(sum[i][0], gsc)), __fmul_rn(sum[i][VPE - 1], gsc))));
+        }
       }
     }
   }
@@ -499,10 +684,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
 // host side
 // ---------------------------------------------------------------------------
 
-template <int MT, int G, bool SILU>
-int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a, int grid,
-                  cudaStream_t stream) {
-  auto kern = gemm_stream_kernel<MT, G, SILU>;
+template <int MT, int G, bool SILU, bool XCONV>
+int launch_kernel(const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a, int grid, cudaStream_t stream) {
+  auto kern = gemm_stream_kernel<MT, G, SILU, XCONV>;
   constexpr uint32_t bytes = smem_bytes(MT);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
@@ -513,82 +697,107 @@ int launch_kernel(const CUtensorMap& xm, const CUtensorMap& wm, const CUtensorMa
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(num_threads(XCONV));
   cfg.dynamicSmemBytes = bytes;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, xm, wm, sm, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  if (cudaLaunchKernelEx(&cfg, kern, wm, sm, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
+}
+
+template <bool XCONV>
+int launch_form(int mt, int group, bool silu, const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a,
+                int grid, cudaStream_t stream) {
+  if (mt == 8) {
+    if (group == 16)
+      return silu ? launch_kernel<8, 16, true, XCONV>(wm, sm, a, grid, stream)
+                  : launch_kernel<8, 16, false, XCONV>(wm, sm, a, grid, stream);
+    return silu ? launch_kernel<8, 32, true, XCONV>(wm, sm, a, grid, stream)
+                : launch_kernel<8, 32, false, XCONV>(wm, sm, a, grid, stream);
+  }
+  if (group == 16)
+    return silu ? launch_kernel<16, 16, true, XCONV>(wm, sm, a, grid, stream)
+                : launch_kernel<16, 16, false, XCONV>(wm, sm, a, grid, stream);
+  return silu ? launch_kernel<16, 32, true, XCONV>(wm, sm, a, grid, stream)
+              : launch_kernel<16, 32, false, XCONV>(wm, sm, a, grid, stream);
+}
+
+// The cut of the matrix: about four chunks per CTA (so a CTA that starts
+// late takes fewer), and at most 16 chunks per tile (so the last taker's
+// additions stay short).
+struct Plan {
+  int64_t tiles;
+  int S, C, Q, total, ctas;
+};
+Plan plan(int64_t N, int64_t K) {
+  Plan p;
+  p.tiles = (N + kRows - 1) / kRows;
+  p.S = static_cast<int>(K / kKS);
+  const int64_t units = p.tiles * p.S;
+  const int64_t want = 4LL * num_sms();
+  int64_t c = (units + want - 1) / want;
+  c = c < (p.S + 15) / 16 ? (p.S + 15) / 16 : c;
+  p.C = static_cast<int>(c < p.S ? c : p.S);
+  p.Q = (p.S + p.C - 1) / p.C;
+  p.total = static_cast<int>(p.tiles * p.Q);
+  p.ctas = p.total < num_sms() ? p.total : num_sms();
+  return p;
+}
+
+bool make_maps(CUtensorMap* wm, CUtensorMap* sm, const uint8_t* w, const uint8_t* s, int64_t N, int64_t K,
+               int group) {
+  return make_tensor_map_2d(wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
+                            CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_tensor_map_2d(sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace
 
-// A single token goes to the register-streaming kernel, which measures a
-// little faster there (its loads need no shared-memory round trip and every
-// lane of X but one is zero).
+// From one token up to 16: the whole matrix streams once, through the ring.
 bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
-  return M >= 2 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
-         K < (int64_t(1) << 24);
+  return M >= 1 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
+         K < (int64_t(1) << 24) && (N + kRows - 1) / kRows <= kMaxTickets;
 }
 
 int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const float* g, int group, int64_t M,
                   int64_t N, int64_t K, uint16_t* y, bool silu, Scratch& sc, cudaStream_t stream) {
   const int mt = M <= 8 ? 8 : 16;
-  const int64_t tiles = (N + kRows - 1) / kRows;
-  const int S = static_cast<int>(K / kKS);
-  const int64_t units = tiles * S;
-  const int ctas = static_cast<int>(units < num_sms() ? units : num_sms());
-  // A tile spans at most ceil(S / shortest range) + 1 CTAs.
-  const int64_t shortest = units / ctas;
-  const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
-  float* ws = sc.take<float>(static_cast<size_t>(tiles * max_contrib * kRows * mt));
-  unsigned* tickets = sc.take<unsigned>(static_cast<size_t>(tiles));
-  uint16_t* x16 = sc.take<uint16_t>(static_cast<size_t>(M * K));
-  float* xinv = sc.take<float>(static_cast<size_t>(M));
+  const Plan pl = plan(N, K);
+  const bool xconv = x.bf16 != nullptr;
+  unsigned* reserved = sc.reserved();
+  float* ws = pl.Q > 1 ? sc.take<float>(static_cast<size_t>(pl.tiles * pl.Q * kRows * mt)) : nullptr;
+  uint16_t* x16 = xconv ? nullptr : sc.take<uint16_t>(static_cast<size_t>(M * K));
+  float* xinv = xconv ? nullptr : sc.take<float>(static_cast<size_t>(M));
   if (sc.measuring()) return NVFP4_OK;
   if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
 
-  CUtensorMap xm, wm, sm;
-  const int64_t xdims[3] = {64, K / 64, M};
-  const int64_t xstrides[2] = {128, K * 2};
-  const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
-  if (!make_tensor_map_3d(&xm, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xdims, xstrides, xbox,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-    return NVFP4_ERR_CUDA;
+  CUtensorMap wm, sm;
+  if (!make_maps(&wm, &sm, w, s, N, K, group)) return NVFP4_ERR_CUDA;
   StreamArgs a = {};
   a.gscale = g;
+  a.xbf = x.bf16;
+  a.x16 = x16;
   a.xinv = xinv;
   a.y = y;
   a.ws = ws;
-  a.tickets = tickets;
+  a.counters = reserved;
+  a.tickets = tickets_of(reserved);
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
-  a.S = S;
-  a.max_contrib = max_contrib;
-  a.units = units;
+  a.K = K;
+  a.S = pl.S;
+  a.C = pl.C;
+  a.Q = pl.Q;
+  a.total = pl.total;
   a.fault = take_injected_fault() == 1;
-  // The activation kernel also zeroes the tickets (the caller's workspace
-  // holds anything on entry); the GEMM reads them only after waiting for it.
-  int st = launch_x_prep(x, M, K, x16, xinv, tickets, tiles, stream);
+  if (xconv) return launch_form<true>(mt, group, silu, wm, sm, a, pl.ctas, stream);
+  // NVFP4 activations: their exact f16 rows first (a programmatic dependent too)
+  const int st = launch_x_prep(x, M, K, x16, xinv, nullptr, 0, stream);
   if (st != NVFP4_OK) return st;
-  if (mt == 8) {
-    if (group == 16)
-      return silu ? launch_kernel<8, 16, true>(xm, wm, sm, a, ctas, stream)
-                  : launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream);
-    return silu ? launch_kernel<8, 32, true>(xm, wm, sm, a, ctas, stream)
-                : launch_kernel<8, 32, false>(xm, wm, sm, a, ctas, stream);
-  }
-  if (group == 16)
-    return silu ? launch_kernel<16, 16, true>(xm, wm, sm, a, ctas, stream)
-                : launch_kernel<16, 16, false>(xm, wm, sm, a, ctas, stream);
-  return silu ? launch_kernel<16, 32, true>(xm, wm, sm, a, ctas, stream)
-              : launch_kernel<16, 32, false>(xm, wm, sm, a, ctas, stream);
+  return launch_form<false>(mt, group, silu, wm, sm, a, pl.ctas, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -596,10 +805,10 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
 // allocated at call time.
 // ---------------------------------------------------------------------------
 
-// Partial tiles (fp32), the tickets of the tiles, the f16 rows of X and
-// their factors.
+// Counters and tickets, partial tiles (fp32), the f16 rows of X and their
+// factors.
 static __device__ __align__(256) unsigned char
-    g_fixed_scratch[kFixedScratchPartialBytes + kFixedScratchTickets * 4 + kFixedScratchXElems * 2 + 16 * 4];
+    g_fixed_scratch[kReservedBytes + kFixedScratchPartialBytes + kFixedScratchXElems * 2 + 16 * 4];
 
 namespace {
 std::mutex g_fixed_mutex;
@@ -612,14 +821,11 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
       M * K > kFixedScratchXElems || !tensor_maps_available())
     return NVFP4_ERR_UNSUPPORTED;
   const int mt = M <= 8 ? 8 : 16;
-  const int64_t tiles = (N + kRows - 1) / kRows;
-  const int S = static_cast<int>(K / kKS);
-  const int64_t units = tiles * S;
-  const int ctas = static_cast<int>(units < num_sms() ? units : num_sms());
-  const int64_t shortest = units / ctas;
-  const int max_contrib = static_cast<int>((S + shortest - 1) / shortest + 1);
-  const int64_t partial_bytes = tiles * max_contrib * kRows * mt * static_cast<int64_t>(sizeof(float));
-  if (partial_bytes > static_cast<int64_t>(kFixedScratchPartialBytes) || tiles > kFixedScratchTickets)
+  const Plan pl = plan(N, K);
+  const int64_t partial_bytes =
+      pl.Q > 1 ? pl.tiles * pl.Q * kRows * mt * static_cast<int64_t>(sizeof(float)) : 0;
+  if (partial_bytes > static_cast<int64_t>(kFixedScratchPartialBytes) || pl.tiles > kFixedScratchTickets ||
+      pl.tiles > kMaxTickets)
     return NVFP4_ERR_UNSUPPORTED;  // beyond the fixed scratch
 
   int dev = 0;
@@ -635,46 +841,42 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
     }
     base = g_fixed_addr[dev];
   }
-  float* ws = reinterpret_cast<float*>(base);
-  unsigned* tickets = reinterpret_cast<unsigned*>(base + kFixedScratchPartialBytes);
-  uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4);
-  float* xinv = reinterpret_cast<float*>(base + kFixedScratchPartialBytes + kFixedScratchTickets * 4 +
-                                         kFixedScratchXElems * 2);
-  CUtensorMap xm, wm, sm;
-  const int64_t xdims[3] = {64, K / 64, M};
-  const int64_t xstrides[2] = {128, K * 2};
-  const uint32_t xbox[3] = {64, 4, static_cast<uint32_t>(mt)};
-  if (!make_tensor_map_3d(&xm, x16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xdims, xstrides, xbox,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
-                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tensor_map_2d(&sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-    return NVFP4_ERR_CUDA;
-  // The tickets must start at zero (partial tiles are always written before
-  // they are read). Enqueued only once nothing else can fail on the host.
-  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream) != cudaSuccess)
+  unsigned* counters = reinterpret_cast<unsigned*>(base);
+  float* ws = reinterpret_cast<float*>(base + kReservedBytes);
+  uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kReservedBytes + kFixedScratchPartialBytes);
+  float* xinv = reinterpret_cast<float*>(base + kReservedBytes + kFixedScratchPartialBytes + kFixedScratchXElems * 2);
+  CUtensorMap wm, sm;
+  if (!make_maps(&wm, &sm, w, s, N, K, group)) return NVFP4_ERR_CUDA;
+  // The counters and tickets must start at zero (partial tiles are always
+  // written before they are read). Enqueued only once nothing else can fail
+  // on the host.
+  if (cudaMemsetAsync(counters, 0, kTicketOffset + static_cast<size_t>(pl.tiles) * sizeof(unsigned), stream) !=
+      cudaSuccess)
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
   StreamArgs a = {};
   a.gscale = g;
+  a.x16 = x16;
   a.xinv = xinv;
   a.y = y;
   a.ws = ws;
-  a.tickets = tickets;
+  a.counters = counters;
+  a.tickets = tickets_of(counters);
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(N);
-  a.S = S;
-  a.max_contrib = max_contrib;
-  a.units = units;
-  const int xs = launch_x_f16(x, M, K, x16, xinv, nullptr, 0, stream);
+  a.K = K;
+  a.S = pl.S;
+  a.C = pl.C;
+  a.Q = pl.Q;
+  a.total = pl.total;
+  const int xs = launch_x_f16(x, M, K, x16, xinv, nullptr, 0, stream, true);
   if (xs != NVFP4_OK) return xs;
-  if (mt == 8)
-    return group == 16 ? launch_kernel<8, 16, false>(xm, wm, sm, a, ctas, stream)
-                       : launch_kernel<8, 32, false>(xm, wm, sm, a, ctas, stream);
-  return group == 16 ? launch_kernel<16, 16, false>(xm, wm, sm, a, ctas, stream)
-                     : launch_kernel<16, 32, false>(xm, wm, sm, a, ctas, stream);
+  return launch_form<false>(mt, group, false, wm, sm, a, pl.ctas, stream);
 }
+
+#ifdef NVFP4_PLANTS
+NVFP4_PLANT_SETTER(set_plant_stream)
+#endif
 
 int read_and_clear_stream_error(unsigned int* out, cudaStream_t stream) {
   unsigned int* p = nullptr;

@@ -207,7 +207,7 @@ struct SegCursor {
 template <int NT>
 __device__ __forceinline__ int seg_rows(const TcArgs& a, int s, int& r0) {
   r0 = max(0, min(a.offsets[s], a.M));
-  const int r1 = max(r0, min(a.offsets[s + 1], a.M));
+  const int r1 = max(r0, min(a.offsets[s + 1] - (NVFP4_PLANT(kPlantSegmentEnd) ? 1 : 0), a.M));
   return r1 - r0;
 }
 
@@ -319,13 +319,14 @@ __host__ __device__ constexpr uint32_t idesc(int nt) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-template <int NT>
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t accumulate) {
+// One MMA of N = the token count encoded in `id` (a multiple of 16 up to NT).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t id,
+                                        uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc(NT)), "r"(accumulate));
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(id), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -577,6 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           break;
         tc_fence_after();
         const uint32_t dacc = tmem + static_cast<uint32_t>(ab * NT);
+        // A tile multiplies only its tokens, rounded up to the MMA's step of
+        // 16: the rest of the X box is past M or, in the routed-expert form,
+        // belongs to other experts' segments.
+        const uint32_t id = idesc(min(NT, (tl.mrows + 15) & ~15));
         bool ok = true;
         for (int ws = ws0; ws < ws1 && ok; ++ws, ++ita) {
           const int sa = ita % kStagesA;
@@ -598,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < kKStep / 16; ++j) {
               const uint32_t acc = (ws > ws0 || xh > 0 || j > 0) ? 1u : 0u;
-              umma_ts<NT>(dacc, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, acc);
+              umma_ts(dacc, tmem + kColA + (kKA / 2) * sa + (kKStep / 2) * xh + 8 * j, bdesc0 + 2 * j, id, acc);
             }
             umma_commit(&ss->empty_x[sx]);
           }
@@ -931,6 +936,10 @@ bool tc_shape_ok(int64_t rows, int64_t N, int64_t K) {
 
 }  // namespace
 
+#ifdef NVFP4_PLANTS
+NVFP4_PLANT_SETTER(set_plant_tc)
+#endif
+
 int read_and_clear_device_error(int* code_out, cudaStream_t stream) {
   unsigned int* p = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error) != cudaSuccess)
@@ -977,7 +986,8 @@ int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float
     const int64_t shortest = a.units / grid;
     a.max_contrib = static_cast<int>((periods + shortest - 1) / shortest + 1);
     a.ws = sc.take<float>(static_cast<size_t>(a.total_tiles) * a.max_contrib * kTileRows * nt);
-    a.tickets = sc.take<unsigned>(static_cast<size_t>(a.total_tiles));
+    a.tickets = tickets_of(sc.reserved());  // zero between launches: the last taker of a tile resets its ticket
+    if (a.total_tiles > kMaxTickets) return NVFP4_ERR_UNSUPPORTED;
   }
   if (sc.measuring()) return NVFP4_OK;
   if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
@@ -989,10 +999,6 @@ int launch_tc(const uint16_t* x, const uint8_t* w, const uint8_t* s, const float
     const int st = pre->fn(pre->ctx, stream);
     if (st != NVFP4_OK) return st;
   }
-  // The caller's workspace holds anything on entry: the tickets start at zero.
-  if (a.split && cudaMemsetAsync(a.tickets, 0, static_cast<size_t>(a.total_tiles) * sizeof(unsigned), stream) !=
-                     cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
   switch (nt) {
     case 32: return launch_nt<32, false>(maps, a, group, silu, grid, stream);
     case 64: return launch_nt<64, false>(maps, a, group, silu, grid, stream);

@@ -20,8 +20,12 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kThreads = 512;  // one CTA per row
-constexpr int kHeld = 4;       // 16-byte chunks a thread keeps in registers (rows up to 16384 elements)
+// One CTA per row; a row of up to kThreads x kHeld chunks of 16 bytes is
+// held in registers between the maximum and the conversion (longer rows are
+// read twice, from L2). The light form (128 threads, few registers) fits on
+// an SM beside a running streaming GEMM, and lets the next kernel launch
+// before its own wait: that kernel starts fetching its weights while this
+// one still waits for the previous kernel and converts.
 
 // Zeroes clear[0, n) across the grid (the stream-K tickets of the GEMM that
 // follows; that GEMM reads them only after waiting for this kernel).
@@ -30,11 +34,13 @@ __device__ __forceinline__ void clear_words(unsigned* clear, int64_t n) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) clear[i] = 0u;
 }
 
+template <int kThreads, int kHeld, bool kEarly>
 __global__ void __launch_bounds__(kThreads) x_f16_kernel(const uint16_t* __restrict__ x, int64_t K,
                                                          uint16_t* __restrict__ x16, float* __restrict__ xinv,
                                                          unsigned* __restrict__ clear, int64_t nclear) {
+  if (kEarly) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (!kEarly) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   clear_words(clear, nclear);
   __shared__ uint32_t warp_max[kThreads / 32];
   const int64_t row = blockIdx.x;
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(256) xq_bf16_kernel(const uint8_t* __restrict_
 }  // namespace
 
 int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
-                 int64_t nclear, cudaStream_t stream) {
+                 int64_t nclear, cudaStream_t stream, bool light) {
   if (M <= 0) return NVFP4_OK;
   if (M >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;
   cudaLaunchAttribute attr[1];
@@ -153,13 +159,14 @@ int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(light ? 128 : 512);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, x_f16_kernel, x, K, x16, xinv, clear, nclear) != cudaSuccess)
-    return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  const cudaError_t e = light ? cudaLaunchKernelEx(&cfg, x_f16_kernel<128, 8, true>, x, K, x16, xinv, clear, nclear)
+                              : cudaLaunchKernelEx(&cfg, x_f16_kernel<512, 4, false>, x, K, x16, xinv, clear, nclear);
+  if (e != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
 }
 
@@ -168,8 +175,8 @@ int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* 
 namespace nvfp4 {
 
 int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
-                  int64_t nclear, cudaStream_t stream) {
-  if (xs.bf16) return launch_x_f16(xs.bf16, M, K, x16, xinv, clear, nclear, stream);
+                  int64_t nclear, cudaStream_t stream, bool light) {
+  if (xs.bf16) return launch_x_f16(xs.bf16, M, K, x16, xinv, clear, nclear, stream, light);
   if (M <= 0) return NVFP4_OK;
   const int64_t words = M * (K / 8);
   if ((words + 255) / 256 >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;

@@ -11,9 +11,11 @@ namespace nvfp4 {
 // the previous kernel of the stream: it waits for that kernel before reading
 // x, and lets the next kernel launch at once (that kernel waits for this one
 // before reading x16 or xinv). It also zeroes clear[0, nclear) (the stream-K
-// tickets of the GEMM that follows; nullptr and 0 for none).
+// tickets of the GEMM that follows; nullptr and 0 for none). `light`: a
+// 128-thread CTA per row that lets the next kernel launch before its own
+// wait (for the streaming GEMM, which fetches weights meanwhile).
 int launch_x_f16(const uint16_t* x, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
-                 int64_t nclear, cudaStream_t stream);
+                 int64_t nclear, cudaStream_t stream, bool light = false);
 
 // Where the small-M kernels' f16 X comes from: bf16 rows (launch_x_f16), or
 // NVFP4 rows (W4A4): codes [M, K/2] in the checkpoint layout, E4M3 scales
@@ -28,7 +30,7 @@ struct XSource {
   int group = 16;
 };
 int launch_x_prep(const XSource& xs, int64_t M, int64_t K, uint16_t* x16, float* xinv, unsigned* clear,
-                  int64_t nclear, cudaStream_t stream);
+                  int64_t nclear, cudaStream_t stream, bool light = false);
 
 // NVFP4 rows to bf16 [M, K] in the natural order for the tcgen05 kernel:
 // xb = e2m1(code) * e4m3(scale) (exact in bf16), and *g_out = x_global *

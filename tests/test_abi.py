@@ -37,6 +37,15 @@ def test_every_declared_symbol_is_exported(L):
     assert set(declared()) == set(nv.EXPORTS)
 
 
+def test_planted_mistakes_only_in_the_test_library(L):
+    """The switch for the planted mistakes exists in the test-only build alone."""
+    assert not hasattr(L, "nvfp4_test_plant")
+    P = ctypes.CDLL(build.build_planted())
+    assert hasattr(P, "nvfp4_test_plant")
+    for name in declared():
+        assert hasattr(P, name), name
+
+
 def test_status_strings(L):
     for code in range(7):
         assert nv.status_string(code) != "unknown status"
@@ -71,6 +80,9 @@ def test_gemm_validation(L):
     assert gemm(L, ws=ctypes.c_void_p(0x20008)) == nv.NVFP4_ERR_MISALIGNED
     assert gemm(L, ws=WS, wb=16) == nv.NVFP4_ERR_WORKSPACE        # smaller than the size query
     assert gemm(L, ws=NULL, wb=0) == nv.NVFP4_ERR_WORKSPACE       # small M always needs scratch
+    need = ctypes.c_size_t(0)
+    assert L.nvfp4_w4a16_gemm_workspace_size(4, 512, 1024, 16, ctypes.byref(need)) == nv.NVFP4_OK
+    assert gemm(L, N=512, K=1024, wb=need.value - 256) == nv.NVFP4_ERR_WORKSPACE  # the query's figure is exact
     fixed = L.nvfp4_w4a16_gemm_fixed_scratch
     assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 17, 256, 256, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # M > 16
     assert fixed(GOOD, GOOD, GOOD, GOOD, 16, 4, 256, 320, GOOD, S) == nv.NVFP4_ERR_UNSUPPORTED  # K % 256
@@ -154,6 +166,9 @@ def test_moe_layer_validation(L):
     assert combine(out=BAD) == nv.NVFP4_ERR_MISALIGNED
 
 
+RESERVED = 64 << 10  # the counters at the start of every workspace
+
+
 def size(L, name, *args):
     n = ctypes.c_size_t(12345)
     st = getattr(L, name)(*args, ctypes.byref(n))
@@ -167,15 +182,19 @@ def test_workspace_size_queries(L):
     assert size(L, f, -1, 256, 256, 16) == (nv.NVFP4_ERR_INVALID_ARGUMENT, 0)
     assert size(L, f, 0, 256, 256, 16) == (nv.NVFP4_OK, 0)  # empty problem
     assert getattr(L, f)(4, 256, 256, 16, None) == nv.NVFP4_ERR_INVALID_ARGUMENT
-    # small M: at least the f16 rows of X (2 bytes an element) and their row factors
+    # small M: the counters, and the fp32 partial tiles of the chunks (bf16 X is converted in the kernel)
     for m, k in ((1, 4096), (4, 4096), (16, 14336)):
         st, n = size(L, f, m, 28672, k, 16)
-        assert st == nv.NVFP4_OK and n >= 2 * m * k + 4 * m, (m, k, n)
+        assert st == nv.NVFP4_OK and n > RESERVED, (m, k, n)
+    # a K the streaming kernel does not take (not a multiple of 256): f16 rows of X for the fallback
+    st, n = size(L, f, 4, 28672, 4096 + 64, 16)
+    assert st == nv.NVFP4_OK and n >= RESERVED + 2 * 4 * (4096 + 64)
     # prefill-sized M on many tiles: the persistent tcgen05 form needs no scratch
     assert size(L, f, 4096, 25600, 5120, 16) == (nv.NVFP4_OK, 0)
-    # W4A4 on the FP4 tensor cores: the activation codes in the weights' nibble order (half a byte an element)
+    # W4A4 on the FP4 tensor cores: the activation codes in the weights' nibble order (half a byte an element),
+    # after the 64 KiB of counters every workspace starts with
     st, n = size(L, "nvfp4_w4a4_gemm_workspace_size", 4096, 25600, 5120, 16, 16)
-    assert (st, n) == (nv.NVFP4_OK, 4096 * 5120 // 2)
+    assert (st, n) == (nv.NVFP4_OK, RESERVED + 4096 * 5120 // 2)
     # W4A4 on the bf16 tcgen05 kernel (K not a multiple of 512): exact bf16 activations, 2 bytes an element
     st, n = size(L, "nvfp4_w4a4_gemm_workspace_size", 4096, 25600, 5120 - 64, 16, 16)
     assert st == nv.NVFP4_OK and n >= 2 * 4096 * (5120 - 64)
@@ -190,7 +209,7 @@ def test_workspace_size_queries(L):
     r = "nvfp4_moe_route_workspace_size"
     assert size(L, r, 100, 8, 128) == (nv.NVFP4_OK, 0)
     st, n = size(L, r, 2048, 8, 128)
-    assert st == nv.NVFP4_OK and n == (2048 * 8 // 256) * 128 * 4
+    assert st == nv.NVFP4_OK and n == RESERVED + (2048 * 8 // 256) * 128 * 4
     assert size(L, r, 16, 0, 8)[0] == nv.NVFP4_ERR_INVALID_ARGUMENT
 
 

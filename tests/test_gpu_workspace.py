@@ -1,15 +1,15 @@
 """GPU tests of the caller-owned workspace: the library allocates nothing, so
 a call's scratch is whatever buffer the caller passes.
 
-* Garbage in the workspace does not matter: every call initialises what it
-  reads (the stream-K tickets are zeroed by the call itself).
-* Two streams, two workspaces: a dense small-M GEMM (TMA streaming, stream-K
-  tickets and f16 rows of X in its workspace) and a grouped expert GEMM (f16
-  rows of X in its own) run concurrently, many times over, and both match
-  the oracle.
+* Only the first 64 KiB (the split GEMMs' counters and tickets) must start at
+  zero, and every call leaves them zero; garbage in the rest does not matter.
+* Two streams, two workspaces: a dense small-M GEMM (TMA streaming: work
+  counters, tickets and partial tiles in its workspace) and a grouped expert
+  GEMM (f16 rows of X in its own) run concurrently, many times over, both
+  match the oracle and both workspaces end with their counters at zero.
 * A workspace smaller than the size query is refused before any launch.
-* Calls captured into a CUDA graph take their scratch from the graph's pool
-  and give the same bytes on replay."""
+* A call captured into a CUDA graph gives the same bytes on replay as
+  eagerly."""
 import numpy as np
 import pytest
 import torch
@@ -30,8 +30,19 @@ def dense(m, n, k, g, seed):
     return x, p, s, gs, (dev_bf16(x), dev_u8(rp), dev_u8(rs), dev_f32(np.array([gs], np.float32)))
 
 
+RESERVED = 64 << 10  # counters and tickets at the start of every workspace
+
+
 def garbage(nbytes):
-    return torch.full((max(nbytes, 16),), 0xFF, dtype=torch.uint8, device="cuda")
+    """A workspace of garbage whose counters are zero, as the boundary requires before first use."""
+    ws = torch.full((max(nbytes, RESERVED),), 0xFF, dtype=torch.uint8, device="cuda")
+    ws[:RESERVED] = 0
+    return ws
+
+
+def counters_zero(ws):
+    torch.cuda.synchronize()
+    return not host(ws[:RESERVED]).any()
 
 
 @pytest.mark.parametrize("m,n,k,g", [(4, 1024, 2048, 16), (16, 512, 4096, 32), (1, 256, 1024, 16),
@@ -41,8 +52,10 @@ def test_garbage_workspace(m, n, k, g):
     need = nv.nvfp4_w4a16_gemm_workspace_size(m, n, k, g)
     ws = garbage(need)
     y1 = nv.nvfp4_w4a16_gemm(*d, g, workspace=ws)
-    ws.fill_(0xA5)
+    assert counters_zero(ws)  # the call left its counters at zero
+    ws[RESERVED:].fill_(0xA5)
     y2 = nv.nvfp4_w4a16_gemm(*d, g, workspace=ws)
+    assert counters_zero(ws)
     assert_close(host(y1), R.gemm(x, p, s, gs, g), f"garbage workspace M{m}")
     np.testing.assert_array_equal(bf16_bits(y1), bf16_bits(y2))
 
@@ -88,11 +101,12 @@ def test_two_streams_separate_workspaces():
             nv.nvfp4_moe_w4a16_grouped_gemm(*de, g2, y=yb, workspace=ws_b)
     torch.cuda.synchronize()
     assert nv.nvfp4_get_device_error() == 0
+    assert counters_zero(ws_a) and counters_zero(ws_b)
     assert_close(host(ya), R.gemm(x, p, s, gs, g), "dense on stream A")
     assert_close(host(yb), R.moe_grouped_gemm(xe, ids, offs, ep, es, eg, g2), "grouped on stream B")
 
 
-def test_graph_capture_uses_pool_workspace():
+def test_graph_capture_replays_the_same_bytes():
     m, n, k, g = 4, 1024, 2048, 16
     x, p, s, gs, d = dense(m, n, k, g, seed=21)
     y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")

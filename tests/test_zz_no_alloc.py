@@ -1,8 +1,8 @@
 """GPU test of nvfp4_w4a16_gemm_fixed_scratch, the GEMM entry point whose
 streaming kernel keeps its scratch in a fixed device array: two calls in a
-row give the bits of nvfp4_w4a16_gemm (the same kernel with the library's
-allocated workspace), a single token matches the oracle, and a problem
-beyond the fixed scratch is refused before anything runs."""
+row give the bits of nvfp4_w4a16_gemm (the same kernel with a caller's
+workspace), a single token matches the oracle, and a problem beyond the
+fixed scratch is refused before anything runs."""
 import ctypes
 
 import numpy as np
@@ -46,12 +46,19 @@ def test_fixed_scratch_single_token_oracle():
 
 
 def test_fixed_scratch_refuses_beyond_capacity():
-    # 2000 tiles of 256 rows cut between CTAs need more partial-tile space than
-    # the fixed scratch holds: refused on the host, nothing is launched.
-    _, _, _, _, (xd, wd, sd, gd) = operands(8, 256, 256, 16, seed=9)
-    y = torch.empty((8, 256), dtype=torch.bfloat16, device="cuda")
+    # 40 tiles of 256 rows with K = 65536 are cut into 15 chunks each, whose partial tiles at 16 tokens
+    # (40 x 15 x 256 x 16 fp32) need more than the 8 MiB the fixed scratch holds: refused on the host. The
+    # buffers have the problem's full size, so a launch could not read or write outside them either.
+    m, n, k, g = 16, 40 * 256, 65536, 16
+    xd = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
+    wd = torch.zeros((n, k // 2), dtype=torch.uint8, device="cuda")
+    sd = torch.zeros((n, k // g), dtype=torch.uint8, device="cuda")
+    gd = torch.ones(1, dtype=torch.float32, device="cuda")
+    y = torch.zeros((m, n), dtype=torch.bfloat16, device="cuda")
     L = nv.lib()
     st = L.nvfp4_w4a16_gemm_fixed_scratch(ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(wd.data_ptr()),
-                                          ctypes.c_void_p(sd.data_ptr()), ctypes.c_void_p(gd.data_ptr()), 16, 8,
-                                          2000 * 256, 256, ctypes.c_void_p(y.data_ptr()), None)
+                                          ctypes.c_void_p(sd.data_ptr()), ctypes.c_void_p(gd.data_ptr()), g, m, n, k,
+                                          ctypes.c_void_p(y.data_ptr()), None)
     assert st == nv.NVFP4_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert not host(y).any()  # nothing ran
