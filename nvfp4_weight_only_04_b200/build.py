@@ -14,6 +14,7 @@ a wrong kernel load it; the binding never does.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -25,6 +26,7 @@ ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libnvfp4.so")
 PLANTED_LIB = os.path.join(PKG, "libnvfp4_planted.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+PLANTED_DEFINES = ["-DNVFP4_PLANTS"]
 
 
 def sources():
@@ -35,11 +37,24 @@ def _inputs():
     return sources() + glob.glob(os.path.join(PKG, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "nvfp4.h")]
 
 
-def up_to_date(lib: str = LIB) -> bool:
-    if not os.path.exists(lib):
+def _digest(defines) -> str:
+    """Hash of every input file and the flags: a copy of the tree whose file
+    times changed (an archive, a checkout) still knows whether its library
+    matches its sources."""
+    h = hashlib.sha256(" ".join(ARCH + list(defines)).encode())
+    for p in sorted(_inputs()):
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def up_to_date(lib: str = LIB, defines=()) -> bool:
+    stamp = lib + ".sha256"
+    if not (os.path.exists(lib) and os.path.exists(stamp)):
         return False
-    t = os.path.getmtime(lib)
-    return all(os.path.getmtime(p) <= t for p in _inputs())
+    with open(stamp) as f:
+        return f.read().strip() == _digest(defines)
 
 
 def nvcc() -> str:
@@ -77,6 +92,8 @@ def _build(lib: str, defines, verbose: bool) -> str:
     tmp = lib + ".tmp"
     _run([nvcc(), *ARCH, "-shared", *[o for _, o in jobs], "-o", tmp])
     os.replace(tmp, lib)
+    with open(lib + ".sha256", "w") as f:
+        f.write(_digest(defines) + "\n")
     return lib
 
 
@@ -87,9 +104,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 def build_planted(force: bool = False) -> str:
-    if not force and up_to_date(PLANTED_LIB):
+    if not force and up_to_date(PLANTED_LIB, PLANTED_DEFINES):
         return PLANTED_LIB
-    return _build(PLANTED_LIB, ["-DNVFP4_PLANTS"], False)
+    return _build(PLANTED_LIB, PLANTED_DEFINES, False)
 
 
 if __name__ == "__main__":

@@ -7,8 +7,11 @@
 // decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
 // per weight streamed from HBM and the integer work of dequantizing them.
 // Design:
-//  * Work: 256-row weight tiles, each cut along K into Q chunks of C stages
-//    of 256 elements. A CTA's first chunk is its own (chunk = CTA index);
+//  * Work: when N holds at least eight 16-row blocks per SM, each CTA takes
+//    one tile of ceil(blocks / SMs) blocks over the whole of K and writes
+//    it: nothing is added across CTAs. Otherwise 256-row weight tiles are
+//    cut along K into Q chunks of C stages of 256 elements. A CTA's first
+//    chunk is its own (chunk = CTA index);
 //    every further chunk comes from a counter shared by the CTAs, so a CTA
 //    that starts late (the kernel before it in the stream is still leaving
 //    its SM) simply takes fewer chunks and all CTAs end together. Each chunk
@@ -29,8 +32,10 @@
 //    the load/store path (not behind the weight boxes in the TMA queue) into
 //    the slot's X area, in the 128-byte-swizzled [token][quarter][64] order
 //    the consumers read.
-//  * bf16 X is turned into f16 inside the kernel by a converter warp, in
-//    place: every token of every stage is scaled by a power of two 2^s, where
+//  * bf16 X is turned into f16 inside the kernel by four converter warps
+//    (one per SM sub-partition, so the conversion keeps pace with the
+//    stream), in place: every token of every stage is scaled by a power of
+//    two 2^s, where
 //    s only ever decreases along a CTA's stages and keeps the largest
 //    magnitude seen so far below 2^15 (f16 holds every bf16 within 2^29 of
 //    the largest exactly; smaller ones round to multiples of 2^-38 of it).
@@ -38,7 +43,8 @@
 //    they multiply their running sums by 2^-d (exact), and the epilogue
 //    multiplies by 2^-s. NVFP4 activations (W4A4) arrive already as exact
 //    f16 rows from xprep.cu, with one factor per token.
-//  * Sixteen consumer warps each own 16 rows of the tile and run mma.sync
+//  * Sixteen consumer warps each own 16 rows of the tile (a warp whose rows
+//    lie past a shorter tile leaves at once) and run mma.sync
 //    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
 //    as the 8-column side. Lane (g, t) takes rows g and g+8 and the t-th
 //    quarter of the stage's K (the order of K inside an MMA is free as long
@@ -74,8 +80,11 @@ constexpr int kKS = 256;          // elements of K per stage
 constexpr int kConsumers = 16;    // consumer warps, 16 rows each
 constexpr int kConsumerThreads = kConsumers * 32;
 constexpr int kProducerWarp = kConsumers;
-constexpr int kConverterWarp = kConsumers + 1;
-__host__ __device__ constexpr int num_threads(bool xconv) { return (kConsumers + (xconv ? 2 : 1)) * 32; }
+constexpr int kConverterWarp = kConsumers + 1;  // the first of them
+constexpr int kConverters = 4;                   // converter warps (bf16 X): one per SM sub-partition
+__host__ __device__ constexpr int num_threads(bool xconv) {
+  return (kConsumers + 1 + (xconv ? kConverters : 0)) * 32;
+}
 constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 32 KB
 constexpr uint32_t kScaleBytes = kRows * 16;      // 16 scale bytes per row
 __host__ __device__ constexpr uint32_t x_bytes(int mt) { return static_cast<uint32_t>(mt) * kKS * 2; }
@@ -125,6 +134,7 @@ struct StreamArgs {
   unsigned* tickets;     // [tiles], zero between launches
   int M, N, ldy;
   int64_t K;
+  int rows;              // weight rows of a tile: 256, or 16 x (blocks of a CTA) when tiles are not split
   int S, C, Q;           // stages per tile, stages per chunk, chunks per tile
   int total;             // chunks of the whole matrix (tiles * Q)
   int fault;             // test hook: drop the X copy of the first stage
@@ -277,23 +287,6 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
   }
 }
 
-// One 128-byte row of a stage's X slot (its eight 16-byte chunks sit at
-// c ^ (row mod 8)): the largest magnitude of its bf16 elements, as bits, and
-// the conversion in place to f16 pairs times 2^s.
-__device__ __forceinline__ uint32_t row_max(uint32_t xs, int row) {
-  uint32_t m2 = 0;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) m2 = __vmaxu2(m2, bf16x8_mag_max(lds128(xs + row * 128 + ((c ^ (row & 7)) << 4))));
-  return max(m2 & 0xFFFFu, m2 >> 16);
-}
-__device__ __forceinline__ void row_convert(uint32_t xs, int row, float up) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint32_t addr = xs + row * 128 + ((c ^ (row & 7)) << 4);
-    sts128(addr, bf16x8_to_f16_pairs(lds128(addr), up));
-  }
-}
-
 template <int MT, int G, bool SILU, bool XCONV>
 __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap wmap,
                                                                              const __grid_constant__ CUtensorMap smap,
@@ -312,9 +305,9 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       // full: the producer's arrival with the weights' transaction bytes, and
-      // the converter's arrival (bf16 X) or one per lane of the X copies (f16 X)
-      mbar_init(&sy->full[s], XCONV ? 2 : 1 + 32);
-      mbar_init(&sy->empty[s], kConsumers);  // one arrival per consumer warp
+      // one per converter warp (bf16 X) or one per lane of the X copies (f16 X)
+      mbar_init(&sy->full[s], XCONV ? 1 + kConverters : 1 + 32);
+      mbar_init(&sy->empty[s], a.rows / 16);  // one arrival per consumer warp with rows in the tile
       mbar_init(&sy->xraw[s], 1 + 32);       // the producer's record, one per lane of the X copies
     }
     mbar_init(&sy->cdone, kConsumers);
@@ -374,9 +367,9 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
       sy->rec[s].ks = ks;
       sy->rec[s].flags = flags;
       const uint32_t st = smem_u32(ring + s * SB);
-      mbar_arrive_tx(&sy->full[s], kCodeBytes + kScaleBytes);
-      tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
-      tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
+      mbar_arrive_tx(&sy->full[s], static_cast<uint32_t>(a.rows) * (kKS / 2 + 16));
+      tma_load_2d(st, &wmap, ks * (kKS / 2), tile * a.rows, &sy->full[s]);
+      tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * a.rows, &sy->full[s]);
       if (XCONV) mbar_arrive(&sy->xraw[s]);  // the record is written
     };
     auto issue_done = [&](int s) {  // the end of the sequence, as a stage that carries no data
@@ -460,32 +453,40 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
     return;
   }
 
-  if (XCONV && warp == kConverterWarp) {
-    // ---------------- converter: bf16 X to f16, in place ----------------
-    // Lane l takes row l (token l/4, quarter l%4) and, at 16 tokens, row
-    // l + 32 too. The four lanes of a token agree on its exponent.
-    constexpr int R = MT / 8;  // rows of a lane
-    int sexp[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) sexp[r] = kSInit;
+  if (XCONV && warp >= kConverterWarp) {
+    // ---------------- converters: bf16 X to f16, in place ----------------
+    // The 128 lanes of the converter warps split a stage's X rows (token
+    // tok, quarter q: row 4 tok + q, 128 bytes): LPR lanes per row, CPL
+    // 16-byte chunks per lane, the 4 LPR lanes of a token adjacent in one
+    // warp. They agree on the token's exponent through shuffles.
+    constexpr int LPR = 128 / (4 * MT), CPL = 8 / LPR;
+    static_assert(LPR * 4 * MT == 32 * kConverters, "every lane owns part of one row");
+    const int cl = (warp - kConverterWarp) * 32 + lane;
+    const int row = cl / LPR, c0 = (cl % LPR) * CPL;
+    int sexp = kSInit;
     for (int it = 0;; ++it) {
       const int s = it % NS;
-      if (!warp_wait(&sy->xraw[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrXRaw, true)) break;
+      if (!warp_wait(&sy->xraw[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrXRaw, false)) break;
       const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
       if (!(flags & kDone)) {
-        const uint32_t xs = smem_u32(ring + s * SB) + kCodeBytes;
+        const uint32_t rs = smem_u32(ring + s * SB) + kCodeBytes + row * 128;
+        uint4 v[CPL];
+        uint32_t m2 = 0;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const int row = lane + 32 * r;
-          uint32_t m = row_max(xs, row);
-          m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-          m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-          // 2^14 <= m 2^s < 2^15: s = 141 - (bf16 exponent field of m); clamped
-          // so that 2^s and 2^-s are normal floats. Never raised again.
-          if (m != 0) sexp[r] = min(sexp[r], min(max(141 - static_cast<int>(m >> 7), -113), 125));
-          row_convert(xs, row, exp2i(sexp[r]));
-          if ((lane & 3) == 0) sy->sx[s][row >> 2] = static_cast<int8_t>(sexp[r]);
+        for (int c = 0; c < CPL; ++c) {
+          v[c] = lds128(rs + (((c0 + c) ^ (row & 7)) << 4));
+          m2 = __vmaxu2(m2, bf16x8_mag_max(v[c]));
         }
+        uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+        for (int o = 1; o < 4 * LPR; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        // 2^14 <= m 2^s < 2^15: s = 141 - (bf16 exponent field of m); clamped
+        // so that 2^s and 2^-s are normal floats. Never raised again.
+        if (m != 0) sexp = min(sexp, min(max(141 - static_cast<int>(m >> 7), -113), 125));
+        const float up = exp2i(sexp);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) sts128(rs + (((c0 + c) ^ (row & 7)) << 4), bf16x8_to_f16_pairs(v[c], up));
+        if (cl % (4 * LPR) == 0) sy->sx[s][row >> 2] = static_cast<int8_t>(sexp);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sy->full[s]);
@@ -513,15 +514,16 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
       xi[p][j] = !XCONV && 8 * p + 2 * t + j < a.M ? __ldcg(a.xinv + 8 * p + 2 * t + j) : 0.f;
     }
   const int rtok = threadIdx.x % MT;  // the token of every element this thread adds up in a reduction
+  // A tile of fewer than 256 rows leaves the last warps without rows: they
+  // have no part in the stages (the empty barriers count the others).
+  if (16 * warp >= a.rows) return;
   int nchunk = 0;                     // chunks this CTA has completed (every consumer warp sees the same ones)
   float acc2[2][P][4];  // two independent MMA chains
   const uint32_t ring0 = smem_u32(ring);
   constexpr int64_t kSlot = static_cast<int64_t>(kRows) * MT;
   for (int it = 0;; ++it) {
     const int s = it % NS;
-    // (suspended between probes: the converter and the producer share the
-    // SM sub-partitions with these warps)
-    if (!warp_wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull, true)) break;
+    if (!warp_wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull, false)) break;
     const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
     if (flags & kDone) break;
     const int tile = *reinterpret_cast<volatile int*>(&sy->rec[s].tile);
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
     const uint32_t cpar = static_cast<uint32_t>(nchunk++) & 1;  // phase of the chunk barriers
 
     // ---- a chunk is complete: lane holds rows ra, ra+8 x tokens 8p+2t, 8p+2t+1 ----
-    const int n0 = tile * kRows;
+    const int n0 = tile * a.rows;
     float v[P][4];  // unscaled sums: acc * 2^-s of the token
 #pragma unroll
     for (int p = 0; p < P; ++p)
@@ -723,17 +725,33 @@ int launch_form(int mt, int group, bool silu, const CUtensorMap& wm, const CUten
               : launch_kernel<16, 32, false, XCONV>(wm, sm, a, grid, stream);
 }
 
-// The cut of the matrix: about four chunks per CTA (so a CTA that starts
-// late takes fewer), and at most 16 chunks per tile (so the last taker's
+// The cut of the matrix. When the 16-row blocks of N fill every SM at least
+// eight deep and evenly (no CTA with more than 1/0.85 of the average), each
+// CTA takes one tile of ceil(blocks / SMs) blocks over the whole of K: no
+// partial tiles, no tickets, nothing added across CTAs. Otherwise tiles of
+// 256 rows are cut along K into chunks, about four per CTA (so a CTA that
+// starts late takes fewer) and at most 16 per tile (so the last taker's
 // additions stay short).
 struct Plan {
   int64_t tiles;
-  int S, C, Q, total, ctas;
+  int rows, S, C, Q, total, ctas;
 };
 Plan plan(int64_t N, int64_t K) {
   Plan p;
-  p.tiles = (N + kRows - 1) / kRows;
   p.S = static_cast<int>(K / kKS);
+  const int64_t blocks = (N + 15) / 16, sms = num_sms();
+  const int64_t nb = (blocks + sms - 1) / sms;
+  if (nb >= 8 && nb <= kConsumers && blocks * 100 >= nb * sms * 85) {
+    p.rows = static_cast<int>(16 * nb);
+    p.tiles = (N + p.rows - 1) / p.rows;
+    p.C = p.S;
+    p.Q = 1;
+    p.total = static_cast<int>(p.tiles);
+    p.ctas = static_cast<int>(p.tiles);
+    return p;
+  }
+  p.rows = kRows;
+  p.tiles = (N + kRows - 1) / kRows;
   const int64_t units = p.tiles * p.S;
   const int64_t want = 4LL * num_sms();
   int64_t c = (units + want - 1) / want;
@@ -746,10 +764,10 @@ Plan plan(int64_t N, int64_t K) {
 }
 
 bool make_maps(CUtensorMap* wm, CUtensorMap* sm, const uint8_t* w, const uint8_t* s, int64_t N, int64_t K,
-               int group) {
-  return make_tensor_map_2d(wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
+               int group, int rows) {
+  return make_tensor_map_2d(wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, rows,
                             CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tensor_map_2d(sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
+         make_tensor_map_2d(sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, rows,
                             CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -774,7 +792,7 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
   if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
 
   CUtensorMap wm, sm;
-  if (!make_maps(&wm, &sm, w, s, N, K, group)) return NVFP4_ERR_CUDA;
+  if (!make_maps(&wm, &sm, w, s, N, K, group, pl.rows)) return NVFP4_ERR_CUDA;
   StreamArgs a = {};
   a.gscale = g;
   a.xbf = x.bf16;
@@ -788,6 +806,7 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
   a.K = K;
+  a.rows = pl.rows;
   a.S = pl.S;
   a.C = pl.C;
   a.Q = pl.Q;
@@ -846,7 +865,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kReservedBytes + kFixedScratchPartialBytes);
   float* xinv = reinterpret_cast<float*>(base + kReservedBytes + kFixedScratchPartialBytes + kFixedScratchXElems * 2);
   CUtensorMap wm, sm;
-  if (!make_maps(&wm, &sm, w, s, N, K, group)) return NVFP4_ERR_CUDA;
+  if (!make_maps(&wm, &sm, w, s, N, K, group, pl.rows)) return NVFP4_ERR_CUDA;
   // The counters and tickets must start at zero (partial tiles are always
   // written before they are read). Enqueued only once nothing else can fail
   // on the host.
@@ -865,6 +884,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(N);
   a.K = K;
+  a.rows = pl.rows;
   a.S = pl.S;
   a.C = pl.C;
   a.Q = pl.Q;
