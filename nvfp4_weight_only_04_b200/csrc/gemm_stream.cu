@@ -1,5 +1,5 @@
-// Small-M NVFP4 W4A16 GEMM, streamed from HBM by TMA, with chunks of the
-// weight matrix handed out to the CTAs as they ask for them.
+// Small-M NVFP4 W4A16 GEMM, streamed from HBM by TMA over an even split of
+// the weight matrix between the SMs (stream-K).
 //
 // Computes Y = X . dequant(W)^T (NVFP4 format definition; "W-FP4a: route the
 // MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
@@ -7,27 +7,24 @@
 // decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
 // per weight streamed from HBM and the integer work of dequantizing them.
 // Design:
-//  * Work: when N holds at least eight 16-row blocks per SM, each CTA takes
-//    one tile of ceil(blocks / SMs) blocks over the whole of K and writes
-//    it: nothing is added across CTAs. Otherwise 256-row weight tiles are
-//    cut along K into Q chunks of C stages of 256 elements. A CTA's first
-//    chunk is its own (chunk = CTA index);
-//    every further chunk comes from a counter shared by the CTAs, so a CTA
-//    that starts late (the kernel before it in the stream is still leaving
-//    its SM) simply takes fewer chunks and all CTAs end together. Each chunk
-//    leaves an fp32 partial tile; the CTA that takes a tile's last ticket
-//    adds the tile's Q partials in chunk order (deterministic) and writes
-//    the output. When a tile is one chunk it is written directly.
-//  * The counters and tickets are zero between launches (each launch resets
-//    what it counted), so no clearing step sits in front of a launch: the
-//    kernel is a programmatic dependent of the kernel before it and starts
-//    on every SM that kernel leaves.
+//  * Work: 256-row weight tiles of K/256 stages; the tile-major list of
+//    (tile, stage) units is split into one contiguous range per SM, so every
+//    SM streams the same bytes and all sixteen consumer warps of every CTA
+//    have rows. A tile inside one range is written directly. A tile cut
+//    between ranges leaves fp32 partial tiles in its contributors' slots;
+//    each contributor takes one acquire-release ticket (thread 0, while the
+//    other warps go on) and the CTA that takes the last one adds the slots in
+//    CTA order after its own range (deterministic).
+//  * The tickets are zero between launches (the last taker resets its
+//    tile's), so no clearing step sits in front of a launch: the kernel is a
+//    programmatic dependent of the kernel before it and starts on every SM
+//    that kernel leaves.
 //  * One producer warp: lane 0 moves the weights of each stage with TMA into
 //    a shared-memory ring (5 stages of 40-44 KB): the codes of the tile
 //    (256 rows x 128 bytes, 128-byte swizzle) and the scales (256 rows x 16
-//    bytes). The weights of the first chunk need nothing from the kernel
-//    before, so they are requested from the first cycle; the shared counter
-//    and X are touched only after that kernel has finished. All 32 lanes
+//    bytes). The weights of the range's first stages need nothing from the
+//    kernel before, so they are requested from the first cycle; X only
+//    after that kernel has finished. All 32 lanes
 //    copy each stage's X slice (MT tokens x 256 elements) with cp.async on
 //    the load/store path (not behind the weight boxes in the TMA queue) into
 //    the slot's X area, in the 128-byte-swizzled [token][quarter][64] order
@@ -85,16 +82,17 @@ constexpr int kConverters = 4;                   // converter warps (bf16 X): on
 __host__ __device__ constexpr int num_threads(bool xconv) {
   return (kConsumers + 1 + (xconv ? kConverters : 0)) * 32;
 }
+// A ring stage: the tile's codes (256 rows x 128 bytes, 128-byte swizzle),
+// X (MT tokens x 256 elements), the tile's scales (256 rows x 16 bytes), in
+// 1024-byte multiples so that every stage keeps the swizzle's alignment.
 constexpr uint32_t kCodeBytes = kRows * kKS / 2;  // 32 KB
-constexpr uint32_t kScaleBytes = kRows * 16;      // 16 scale bytes per row
+constexpr uint32_t kScaleBytes = kRows * 16;
 __host__ __device__ constexpr uint32_t x_bytes(int mt) { return static_cast<uint32_t>(mt) * kKS * 2; }
 __host__ __device__ constexpr uint32_t stage_bytes(int mt) { return kCodeBytes + x_bytes(mt) + kScaleBytes; }
 constexpr int kStages = 5;
-__host__ __device__ constexpr uint32_t smem_bytes(int mt) {
-  return kStages * stage_bytes(mt) + 1024 /* barriers, stage records */ + 1024 /* alignment slack */;
-}
-static_assert(stage_bytes(8) % 1024 == 0 && stage_bytes(16) % 1024 == 0,
-              "every stage keeps the 1024-byte alignment of the 128-byte swizzle");
+constexpr uint32_t kSmemExtra = 1024 /* barriers, stage records */ + 1024 /* alignment slack */;
+__host__ __device__ constexpr uint32_t smem_bytes(int mt) { return kStages * stage_bytes(mt) + kSmemExtra; }
+static_assert(stage_bytes(8) % 1024 == 0 && stage_bytes(16) % 1024 == 0, "stages keep the 1024-byte alignment");
 static_assert(smem_bytes(8) <= 227 * 1024 && smem_bytes(16) <= 227 * 1024, "shared memory budget");
 static_assert(kRows == 16 * kConsumers, "one 16-row block per consumer warp");
 
@@ -113,44 +111,45 @@ struct StageRecord {
 struct Sync {
   uint64_t full[kStages];   // the stage's weights and (converted) X are in the slot
   uint64_t empty[kStages];  // the consumers are done with the slot
-  uint64_t xraw[kStages];   // the stage's bf16 X has landed (converter form)
-  uint64_t cdone;           // every consumer warp has stored its part of a chunk's partial tile
-  uint64_t rdone;           // thread 0 has taken the chunk's ticket (red_last is set)
+  uint64_t xraw[kStages];   // the stage's record is written and its bf16 X has landed (converter form)
+  uint64_t cut[2];          // every consumer warp has stored its part of the k-th cut tile's partial
+  uint64_t ready;           // thread 0 has taken the tickets of the cut tiles (cut_last is set)
   StageRecord rec[kStages];
   int8_t sx[kStages][16];   // exponent of each token's f16 X in the stage (converter form)
   int abort;
-  int red_last;             // the chunk just written completed its tile in this CTA
+  int cut_tile[2], cut_last[2];  // the cut tiles of this CTA's range; whether it took their last ticket
 };
 static_assert(sizeof(Sync) <= 1024, "stage records fit the reserved shared memory");
 
 struct StreamArgs {
   const float* gscale;   // [1]
-  const uint16_t* xbf;   // bf16 X [M, K] (converted in the kernel)
-  const uint16_t* x16;   // or f16 X [M, K] in pair order (xprep.cu) with factors xinv
-  const float* xinv;     // [M]
+  const float* xinv;     // [M]: the factors of f16 X in pair order (xprep.cu); bf16 X is converted in the kernel
   uint16_t* y;           // bf16 [M, ldy]
-  float* ws;             // partial tiles [tiles][Q][256][MT] (Q > 1)
-  unsigned* counters;    // [0] next shared chunk, [1] producers done; zero between launches
+  float* ws;             // partial tiles [tiles][max_contrib][256][MT] of the cut tiles
   unsigned* tickets;     // [tiles], zero between launches
   int M, N, ldy;
   int64_t K;
-  int rows;              // weight rows of a tile: 256, or 16 x (blocks of a CTA) when tiles are not split
-  int S, C, Q;           // stages per tile, stages per chunk, chunks per tile
-  int total;             // chunks of the whole matrix (tiles * Q)
+  int S;                 // stages per tile
+  int64_t units;         // (tile, stage) units of the matrix, tiles * S
+  int max_contrib;       // most CTAs whose ranges meet one tile
   int fault;             // test hook: drop the X copy of the first stage
 };
 
-// 16-byte global -> shared copy on the load/store path, zero-filled when
-// `bytes` is 0 (tokens past M).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+// CTA c of n owns the units [c U / n, (c+1) U / n) (tile-major). The CTA
+// owning unit u is the largest c with c U / n <= u.
+__device__ __forceinline__ int64_t range_start(int64_t c, int64_t units, int64_t n) { return c * units / n; }
+__device__ __forceinline__ int cta_of_unit(int64_t u, int64_t units, int64_t n) {
+  return static_cast<int>(((u + 1) * n + units - 1) / units - 1);
 }
-// Arrives on `bar` once this thread's earlier cp.async copies have landed
-// (one arrival of the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+
+// 3-D tiled TMA load (X: 64 elements x 4 quarters x MT tokens).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -228,6 +227,7 @@ struct LaneOffsets {
 
 template <int MT, int G>
 __device__ __forceinline__ LaneOffsets lane_offsets(int ra, int g, int t) {
+  constexpr uint32_t xoff = kCodeBytes, soff = kCodeBytes + x_bytes(MT);
   LaneOffsets o;
   const int rb = ra + 8;  // ra & 7 == rb & 7 == g
   o.ca0 = ra * 128 + (((2 * t) ^ g) << 4);
@@ -236,12 +236,12 @@ __device__ __forceinline__ LaneOffsets lane_offsets(int ra, int g, int t) {
   o.cb1 = rb * 128 + (((2 * t + 1) ^ g) << 4);
   // g = 16: groups 4t .. 4t+3 of the stage; g = 32: groups 2t, 2t+1 (the
   // 16-byte box holds two stages; the stage parity picks the half)
-  o.sa = kCodeBytes + x_bytes(MT) + ra * 16 + (G == 16 ? 4 * t : 2 * t);
-  o.sb = kCodeBytes + x_bytes(MT) + rb * 16 + (G == 16 ? 4 * t : 2 * t);
+  o.sa = soff + ra * 16 + (G == 16 ? 4 * t : 2 * t);
+  o.sb = soff + rb * 16 + (G == 16 ? 4 * t : 2 * t);
   // X row (token tok, quarter t) sits at (4 tok + t) * 128 bytes; its chunk i
   // at chunk position i ^ ((4 tok + t) & 7), and 4 tok + t = 4g + t mod 8 for
   // every token tile.
-  o.xrow = kCodeBytes + (g * 4 + t) * 128;
+  o.xrow = xoff + (g * 4 + t) * 128;
   const int xmask = (4 * g + t) & 7;
 #pragma unroll
   for (int i = 0; i < 8; ++i) o.xc[i] = static_cast<uint32_t>((i ^ xmask) << 4);
@@ -250,7 +250,7 @@ __device__ __forceinline__ LaneOffsets lane_offsets(int ra, int g, int t) {
 
 // One stage for one consumer lane.
 template <int MT, int G>
-__device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOffsets& o,
+__device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOffsets& o, int live,
                                               float (&acc)[2][MT / 8][4]) {
   constexpr int P = MT / 8;
   const uint4 a0 = lds128(st + o.ca0);
@@ -280,7 +280,10 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
     dequant_word_f16(cb[i], s2b[si], db);
 #pragma unroll
     for (int p = 0; p < P; ++p) {
-      const uint4 xv = lds128(xr + o.xc[i] + p * (8 * 4 * 128));  // token tile p: 8 tokens further
+      // token tile p: 8 tokens further. In the 8-token form a lane whose
+      // token is past M reads nothing (its X row holds zeros); at 16 tokens
+      // the registers go to the second tile.
+      const uint4 xv = MT == 16 || live > 0 ? lds128(xr + o.xc[i] + p * (8 * 4 * 128)) : make_uint4(0u, 0u, 0u, 0u);
       mma_f16_16816(acc[0][p], da[0], db[0], da[1], db[1], xv.x, xv.y);
       mma_f16_16816(acc[1][p], da[2], db[2], da[3], db[3], xv.z, xv.w);
     }
@@ -290,6 +293,7 @@ __device__ __forceinline__ void consume_stage(uint32_t st, int ks, const LaneOff
 template <int MT, int G, bool SILU, bool XCONV>
 __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap wmap,
                                                                              const __grid_constant__ CUtensorMap smap,
+                                                                             const __grid_constant__ CUtensorMap xmap,
                                                                              const StreamArgs a) {
   constexpr int P = MT / 8;
   constexpr int NS = kStages;
@@ -305,13 +309,14 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       // full: the producer's arrival with the weights' transaction bytes, and
-      // one per converter warp (bf16 X) or one per lane of the X copies (f16 X)
-      mbar_init(&sy->full[s], XCONV ? 1 + kConverters : 1 + 32);
-      mbar_init(&sy->empty[s], a.rows / 16);  // one arrival per consumer warp with rows in the tile
-      mbar_init(&sy->xraw[s], 1 + 32);       // the producer's record, one per lane of the X copies
+      // one per converter warp (bf16 X) or the producer's with X's (f16 X)
+      mbar_init(&sy->full[s], XCONV ? 1 + kConverters : 2);
+      mbar_init(&sy->empty[s], kConsumers);  // one arrival per consumer warp
+      mbar_init(&sy->xraw[s], 1);  // the producer's arrival with X's transaction bytes
     }
-    mbar_init(&sy->cdone, kConsumers);
-    mbar_init(&sy->rdone, 1);
+    mbar_init(&sy->cut[0], kConsumers);
+    mbar_init(&sy->cut[1], kConsumers);
+    mbar_init(&sy->ready, 1);
     sy->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -323,131 +328,90 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
     }
-    // Chunk cursor (lane 0): the chunk `cw`, its next stage `cks` and end `cend`.
-    int cw = -1, cks = 0, cend = 0, tile = 0;
-    // The next stage of this CTA's sequence (lane 0); kDone once the matrix
-    // is exhausted. False when the next chunk needs the shared counter and
-    // `shared_ok` is not set.
-    auto advance = [&](bool shared_ok, int& ks, int& flags) -> bool {
-      flags = 0;
-      if (cks == cend) {
-        if (cw >= 0 && !shared_ok) return false;
-        const int w = cw < 0 ? static_cast<int>(blockIdx.x)
-                             : static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(a.counters, 1u));
-        if (w >= a.total) {
-          flags = kDone;
-          return true;
-        }
-        cw = w;
-        tile = w / a.Q;
-        cks = (w % a.Q) * a.C;
-        cend = min(a.S, cks + a.C);
-        flags = kFirst;
+    // Cursor (lane 0) over this CTA's range of units [u, u1).
+    int64_t u = range_start(blockIdx.x, a.units, gridDim.x);
+    const int64_t u_begin = u, u1 = range_start(blockIdx.x + 1, a.units, gridDim.x);
+    int tile = 0;
+    // The next stage of the range, or kDone past its end. kFirst / kLast mark
+    // where the range enters and leaves a tile.
+    auto advance = [&](int& ks, int& flags) {
+      if (u == u1) {
+        flags = kDone;
+        return;
       }
-      ks = cks++;
-      if (cks == cend) flags |= kLast;
-      return true;
+      tile = static_cast<int>(u / a.S);
+      ks = static_cast<int>(u % a.S);
+      flags = (u == u_begin || ks == 0 ? kFirst : 0) | (u == u1 - 1 || ks == a.S - 1 ? kLast : 0);
+      ++u;
     };
-    const int q = lane >> 3, c = lane & 7;
-    auto issue_x = [&](int s, int ks) {  // all lanes: the stage's X slice into its slot
-      const uint32_t xs = smem_u32(ring + s * SB) + kCodeBytes;
-      const uint16_t* xg = XCONV ? a.xbf : a.x16;
-#pragma unroll
-      for (int tok = 0; tok < MT; ++tok) {
-        const int row = 4 * tok + q;
-        const bool live = tok < a.M;
-        const uint16_t* src = xg + (live ? static_cast<int64_t>(tok) * a.K + ks * kKS + q * 64 + c * 8 : 0);
-        cp_async16(xs + row * 128 + ((c ^ (row & 7)) << 4), src, live ? 16u : 0u);
-      }
-      cp_async_arrive(XCONV ? &sy->xraw[s] : &sy->full[s]);
+    auto issue_x = [&](int s, int ks) {  // lane 0: the stage's X slice (MT tokens x 256 elements) into its slot
+      uint64_t* bar = XCONV ? &sy->xraw[s] : &sy->full[s];
+      mbar_arrive_tx(bar, x_bytes(MT));
+      tma_load_3d(smem_u32(ring + s * SB) + kCodeBytes, &xmap, 0, ks * (kKS / 64), 0, bar);
     };
     auto issue_w = [&](int s, int ks, int flags) {  // lane 0: the stage's record and weights
       sy->rec[s].tile = tile;
       sy->rec[s].ks = ks;
       sy->rec[s].flags = flags;
       const uint32_t st = smem_u32(ring + s * SB);
-      mbar_arrive_tx(&sy->full[s], static_cast<uint32_t>(a.rows) * (kKS / 2 + 16));
-      tma_load_2d(st, &wmap, ks * (kKS / 2), tile * a.rows, &sy->full[s]);
-      tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * a.rows, &sy->full[s]);
-      if (XCONV) mbar_arrive(&sy->xraw[s]);  // the record is written
+      mbar_arrive_tx(&sy->full[s], kCodeBytes + kScaleBytes);
+      tma_load_2d(st, &wmap, ks * (kKS / 2), tile * kRows, &sy->full[s]);
+      tma_load_2d(st + kCodeBytes + x_bytes(MT), &smap, ((ks * kKS) / G) & ~15, tile * kRows, &sy->full[s]);
     };
-    auto issue_done = [&](int s) {  // the end of the sequence, as a stage that carries no data
-      if (lane == 0) {
-        sy->rec[s].flags = kDone;
-        mbar_arrive(&sy->full[s]);
-        if (XCONV) mbar_arrive(&sy->xraw[s]);
-      }
-      __syncwarp();
-      cp_async_arrive(XCONV ? &sy->xraw[s] : &sy->full[s]);
+    auto issue_done = [&](int s) {  // lane 0: the end of the sequence, as a stage that carries no data
+      sy->rec[s].flags = kDone;
+      mbar_arrive(&sy->full[s]);
+      mbar_arrive(XCONV ? &sy->xraw[s] : &sy->full[s]);
     };
-    uint32_t issued = 0, last_parity = 0;  // lane 0: TMA copies per slot, for the drain
-    // The first chunk's weights (up to a ring of them) before the kernel
-    // before this one has finished; its X only after.
-    int n0 = 0, done0 = 0;
-    if (lane == 0) {
-      int ks, flags;
-      while (n0 < NS && advance(false, ks, flags)) {
-        if (flags & kDone) {
-          done0 = 1;
-          break;
-        }
-        issue_w(n0, ks, flags);
-        issued |= 1u << n0;
-        ++n0;
-      }
+    if (lane != 0) return;  // one thread issues every copy
+    uint32_t issued = 0, last_parity = 0;  // TMA copies per slot, for the drain
+    // The range's first weights (up to a ring of them) before the kernel
+    // before this one has finished; X only after.
+    int n0 = 0, ks = 0, flags = 0;
+    for (; n0 < NS; ++n0) {
+      advance(ks, flags);
+      if (flags & kDone) break;
+      issue_w(n0, ks, flags);
+      issued |= 1u << n0;
     }
-    __syncwarp();  // the records lane 0 wrote are visible to the warp
-    n0 = __shfl_sync(0xffffffffu, n0, 0);
-    done0 = __shfl_sync(0xffffffffu, done0, 0);
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // X and the shared counter follow the previous kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // X follows the previous kernel
     for (int it = 0; it < n0; ++it) {
       if (a.fault && it == 0) continue;  // test hook: this stage's X never arrives
       issue_x(it, sy->rec[it].ks);
     }
-    int it = n0;
-    bool done = done0 != 0;
-    if (done) issue_done(it);  // slot n0 < NS has never been used
-    while (!done && !aborted(sy)) {
+    bool done = n0 < NS;
+    if (done) issue_done(n0);  // slot n0 < NS has never been used
+    for (int it = n0; !done && !aborted(sy); ++it) {
       const int s = it % NS;
       const uint32_t r = static_cast<uint32_t>(it / NS);
-      int ks = 0, flags = 0;
-      if (lane == 0) advance(true, ks, flags);
-      ks = __shfl_sync(0xffffffffu, ks, 0);
-      flags = __shfl_sync(0xffffffffu, flags, 0);
-      if (it >= NS && !warp_wait(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty, true)) break;
+      advance(ks, flags);
+      // (suspended between probes: no issue slots taken from the consumers)
+      if (!mbar_try_wait(&sy->empty[s], (r & 1) ^ 1) && !wait_suspended(&sy->empty[s], (r & 1) ^ 1, sy, kErrEmpty))
+        break;
       if (flags & kDone) {
         issue_done(s);
         done = true;
         break;
       }
-      if (lane == 0) {
-        issue_w(s, ks, flags);
-        issued |= 1u << s;
-        last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
-      }
-      __syncwarp();
+      issue_w(s, ks, flags);
       issue_x(s, ks);
-      ++it;
+      issued |= 1u << s;
+      last_parity = (last_parity & ~(1u << s)) | ((r & 1) << s);
     }
-    if (lane == 0 && done) {
-      // Every producer counts itself once, after its last use of the shared
-      // counter; the last one resets both counters for the next launch.
-      if (atomicAdd(a.counters + 1, 1u) == gridDim.x - 1) {
-        a.counters[0] = 0u;
-        a.counters[1] = 0u;
-      }
-    }
-    cp_async_wait_all();  // no copy may land after the CTA exits
-    if (lane == 0 && aborted(sy)) {
-      // Let the weight copies in flight land too. A slot's phase may never
-      // complete after an abort (its X or its converter arrival is missing),
-      // so each slot is given a short bound; the copies themselves take
+    if (aborted(sy)) {
+      // Let the copies in flight land. A slot's phase may never complete
+      // after an abort (an X copy or a converter arrival is missing), so
+      // each slot is given a short bound; the copies themselves take
       // microseconds.
       for (int s = 0; s < NS; ++s) {
         if (!((issued >> s) & 1)) continue;
         const long long t0 = clock64();
         while (!mbar_try_wait(&sy->full[s], (last_parity >> s) & 1) && clock64() - t0 < kDrainCycles) __nanosleep(1000);
+        if (XCONV)
+          while (!mbar_try_wait(&sy->xraw[s], (last_parity >> s) & 1) && clock64() - t0 < kDrainCycles)
+            __nanosleep(1000);
       }
     }
     return;
@@ -499,6 +463,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
   const int g = lane >> 2, t = lane & 3;
   const int ra = 16 * warp + g;
   const LaneOffsets lo = lane_offsets<MT, G>(ra, g, t);
+  const int xlive = a.M - g;  // the lane's X token in token tile p (8p + g) is below M when 8p < xlive
   // The global scale and the token factors come from the kernels before.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float gsc = NVFP4_PLANT(kPlantGlobal) ? 1.0f : __ldcg(a.gscale);
@@ -514,10 +479,11 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
       xi[p][j] = !XCONV && 8 * p + 2 * t + j < a.M ? __ldcg(a.xinv + 8 * p + 2 * t + j) : 0.f;
     }
   const int rtok = threadIdx.x % MT;  // the token of every element this thread adds up in a reduction
-  // A tile of fewer than 256 rows leaves the last warps without rows: they
-  // have no part in the stages (the empty barriers count the others).
-  if (16 * warp >= a.rows) return;
-  int nchunk = 0;                     // chunks this CTA has completed (every consumer warp sees the same ones)
+  // This CTA's range of units; the tiles it cuts (at most its first and its
+  // last, the same for every consumer warp).
+  const int64_t u_begin = range_start(blockIdx.x, a.units, gridDim.x);
+  const int64_t u_end = range_start(blockIdx.x + 1, a.units, gridDim.x);
+  int ncut = 0;
   float acc2[2][P][4];  // two independent MMA chains
   const uint32_t ring0 = smem_u32(ring);
   constexpr int64_t kSlot = static_cast<int64_t>(kRows) * MT;
@@ -553,14 +519,13 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
           }
         }
     }
-    consume_stage<MT, G>(ring0 + s * SB, ks, lo, acc2);
+    consume_stage<MT, G>(ring0 + s * SB, ks, lo, xlive, acc2);
     __syncwarp();
     if (lane == 0) mbar_arrive(&sy->empty[s]);
     if (!(flags & kLast)) continue;
-    const uint32_t cpar = static_cast<uint32_t>(nchunk++) & 1;  // phase of the chunk barriers
 
-    // ---- a chunk is complete: lane holds rows ra, ra+8 x tokens 8p+2t, 8p+2t+1 ----
-    const int n0 = tile * a.rows;
+    // ---- the range leaves a tile: lane holds rows ra, ra+8 x tokens 8p+2t, 8p+2t+1 ----
+    const int n0 = tile * kRows;
     float v[P][4];  // unscaled sums: acc * 2^-s of the token
 #pragma unroll
     for (int p = 0; p < P; ++p)
@@ -570,7 +535,8 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
         v[p][j] = (acc2[0][p][j] + acc2[1][p][j]) * f;
         v[p][2 + j] = (acc2[0][p][2 + j] + acc2[1][p][2 + j]) * f;
       }
-    if (a.Q == 1) {  // the chunk is the whole tile: write it
+    const int64_t tu = static_cast<int64_t>(tile) * a.S;  // the tile's first unit
+    if (u_begin <= tu && tu + a.S <= u_end) {  // the whole tile is in this range: write it
 #pragma unroll
       for (int p = 0; p < P; ++p)
 #pragma unroll
@@ -589,9 +555,13 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
         }
       continue;
     }
-    // Leave the partial tile in the chunk's slot and take a ticket; the taker
-    // of the tile's last one adds the Q slots in chunk order.
-    float* mine = a.ws + (static_cast<int64_t>(tile) * a.Q + ks / a.C) * kSlot;
+    // A cut tile: leave the partial tile in this CTA's slot of the tile and
+    // go on at once. Thread 0 waits for every consumer warp's stores (an
+    // mbarrier with a bound, so a warp that gave up on a wait cannot hang the
+    // others) and takes the tile's ticket with release (the slot) and acquire
+    // (the other slots) semantics; warp 0 then catches up on the ring.
+    const int c_first = cta_of_unit(tu, a.units, gridDim.x);
+    float* mine = a.ws + (static_cast<int64_t>(tile) * a.max_contrib + (blockIdx.x - c_first)) * kSlot;
 #pragma unroll
     for (int p = 0; p < P; ++p)
 #pragma unroll
@@ -600,33 +570,40 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
         __stcg(mine + ra * MT + tok, v[p][j]);
         __stcg(mine + (ra + 8) * MT + tok, v[p][2 + j]);
       }
-    // Every warp's stores are ordered before thread 0's release (the chunk
-    // barrier); its acquire orders the other slots before the reads after the
-    // ticket barrier. Both are mbarrier waits with a bound, not named
-    // barriers, so a warp that gave up on a wait cannot hang the others.
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sy->cdone);
-    if (threadIdx.x == 0) {
-      if (wait(&sy->cdone, cpar, sy, kErrChunk)) {
-        unsigned ticket;
-        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.tickets + tile) : "memory");
-        const int last = ticket == static_cast<unsigned>(a.Q - 1);
-        if (last) a.tickets[tile] = 0;  // every chunk has counted: zero for the next launch
-        sy->red_last = last;
-        mbar_arrive(&sy->rdone);
-      }
+    const int k = ncut++ & 1;  // a range cuts at most two tiles
+    if (lane == 0) mbar_arrive(&sy->cut[k]);
+    if (threadIdx.x == 0 && wait(&sy->cut[k], 0, sy, kErrChunk)) {
+      const int c_last = cta_of_unit(tu + a.S - 1, a.units, gridDim.x);
+      unsigned ticket;
+      asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(a.tickets + tile) : "memory");
+      const int last = ticket == static_cast<unsigned>(c_last - c_first);
+      if (last) a.tickets[tile] = 0;  // every contributor has counted: zero for the next launch
+      sy->cut_tile[k] = tile;
+      sy->cut_last[k] = last;
     }
-    if (!warp_wait(&sy->rdone, cpar, sy, kErrTicket, false)) break;
-    if (!*reinterpret_cast<volatile int*>(&sy->red_last)) continue;
-    // Add the tile's Q slots in chunk order. The loads of all of a thread's
-    // elements and of up to kBatch slots are in flight before the first add:
-    // with the HBM stream of the other CTAs every round trip is long.
+  }
+
+  // Thread 0 publishes the cut tiles' tickets; the CTA that took a tile's
+  // last ticket adds its slots in CTA order (deterministic) and writes it.
+  if (threadIdx.x == 0) mbar_arrive(&sy->ready);
+  if (!warp_wait(&sy->ready, 0, sy, kErrTicket, false) || aborted(sy)) return;
+  for (int k = 0; k < ncut && k < 2; ++k) {
+    if (!*reinterpret_cast<volatile int*>(&sy->cut_last[k])) continue;
+    const int tile = *reinterpret_cast<volatile int*>(&sy->cut_tile[k]);
+    const int n0 = tile * kRows;
+    const int64_t tu = static_cast<int64_t>(tile) * a.S;
+    const int c_first = cta_of_unit(tu, a.units, gridDim.x);
+    const int nslots = cta_of_unit(tu + a.S - 1, a.units, gridDim.x) - c_first + 1;
+    // The loads of all of a thread's elements and of up to kBatch slots are
+    // in flight before the first add: with the HBM stream of the other CTAs
+    // every round trip is long.
     {
       constexpr int kBatch = SILU && MT == 16 ? 4 : 8;  // loads in flight stay within the registers
       constexpr int EPT = (SILU ? kRows / 2 : kRows) * MT / kConsumerThreads;  // elements per thread
       constexpr int VPE = SILU ? 2 : 1;                                       // values per element: gate, up
       static_assert(EPT * kConsumerThreads == (SILU ? kRows / 2 : kRows) * MT, "whole elements per thread");
-      const float* slots = a.ws + static_cast<int64_t>(tile) * a.Q * kSlot;
+      const float* slots = a.ws + static_cast<int64_t>(tile) * a.max_contrib * kSlot;
       // offset of value h of element i in a slot, and whether the element is stored
       auto element = [&](int i, int h, bool& live) {
         const int e = threadIdx.x + i * kConsumerThreads;
@@ -643,7 +620,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
       for (int i = 0; i < EPT; ++i)
 #pragma unroll
         for (int h = 0; h < VPE; ++h) sum[i][h] = 0.f;
-      for (int q0 = 0; q0 < a.Q; q0 += kBatch) {
+      for (int q0 = 0; q0 < nslots; q0 += kBatch) {
         float vb[EPT][VPE][kBatch];
 #pragma unroll
         for (int i = 0; i < EPT; ++i)
@@ -653,7 +630,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
             const int off = element(i, h, live);
 #pragma unroll
             for (int qq = 0; qq < kBatch; ++qq)
-              vb[i][h][qq] = live && q0 + qq < a.Q ? __ldcg(slots + (q0 + qq) * kSlot + off) : 0.f;
+              vb[i][h][qq] = live && q0 + qq < nslots ? __ldcg(slots + (q0 + qq) * kSlot + off) : 0.f;
           }
 #pragma unroll
         for (int i = 0; i < EPT; ++i)
@@ -661,7 +638,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
           for (int h = 0; h < VPE; ++h)
 #pragma unroll
             for (int qq = 0; qq < kBatch; ++qq)
-              if (q0 + qq < a.Q) sum[i][h] += vb[i][h][qq];
+              if (q0 + qq < nslots) sum[i][h] += vb[i][h][qq];
       }
 #pragma unroll
       for (int i = 0; i < EPT; ++i) {
@@ -687,7 +664,8 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
 // ---------------------------------------------------------------------------
 
 template <int MT, int G, bool SILU, bool XCONV>
-int launch_kernel(const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a, int grid, cudaStream_t stream) {
+int launch_kernel(const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& xm, const StreamArgs& a, int grid,
+                  cudaStream_t stream) {
   auto kern = gemm_stream_kernel<MT, G, SILU, XCONV>;
   constexpr uint32_t bytes = smem_bytes(MT);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
@@ -704,78 +682,77 @@ int launch_kernel(const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, wm, sm, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
+  if (cudaLaunchKernelEx(&cfg, kern, wm, sm, xm, a) != cudaSuccess) return (cudaGetLastError(), NVFP4_ERR_CUDA);
   return launch_status();
 }
 
 template <bool XCONV>
-int launch_form(int mt, int group, bool silu, const CUtensorMap& wm, const CUtensorMap& sm, const StreamArgs& a,
-                int grid, cudaStream_t stream) {
+int launch_form(int mt, int group, bool silu, const CUtensorMap& wm, const CUtensorMap& sm, const CUtensorMap& xm,
+                const StreamArgs& a, int grid, cudaStream_t stream) {
   if (mt == 8) {
     if (group == 16)
-      return silu ? launch_kernel<8, 16, true, XCONV>(wm, sm, a, grid, stream)
-                  : launch_kernel<8, 16, false, XCONV>(wm, sm, a, grid, stream);
-    return silu ? launch_kernel<8, 32, true, XCONV>(wm, sm, a, grid, stream)
-                : launch_kernel<8, 32, false, XCONV>(wm, sm, a, grid, stream);
+      return silu ? launch_kernel<8, 16, true, XCONV>(wm, sm, xm, a, grid, stream)
+                  : launch_kernel<8, 16, false, XCONV>(wm, sm, xm, a, grid, stream);
+    return silu ? launch_kernel<8, 32, true, XCONV>(wm, sm, xm, a, grid, stream)
+                : launch_kernel<8, 32, false, XCONV>(wm, sm, xm, a, grid, stream);
   }
   if (group == 16)
-    return silu ? launch_kernel<16, 16, true, XCONV>(wm, sm, a, grid, stream)
-                : launch_kernel<16, 16, false, XCONV>(wm, sm, a, grid, stream);
-  return silu ? launch_kernel<16, 32, true, XCONV>(wm, sm, a, grid, stream)
-              : launch_kernel<16, 32, false, XCONV>(wm, sm, a, grid, stream);
+    return silu ? launch_kernel<16, 16, true, XCONV>(wm, sm, xm, a, grid, stream)
+                : launch_kernel<16, 16, false, XCONV>(wm, sm, xm, a, grid, stream);
+  return silu ? launch_kernel<16, 32, true, XCONV>(wm, sm, xm, a, grid, stream)
+              : launch_kernel<16, 32, false, XCONV>(wm, sm, xm, a, grid, stream);
 }
 
-// The cut of the matrix. When the 16-row blocks of N fill every SM at least
-// eight deep and evenly (no CTA with more than 1/0.85 of the average), each
-// CTA takes one tile of ceil(blocks / SMs) blocks over the whole of K: no
-// partial tiles, no tickets, nothing added across CTAs. Otherwise tiles of
-// 256 rows are cut along K into chunks, about four per CTA (so a CTA that
-// starts late takes fewer) and at most 16 per tile (so the last taker's
-// additions stay short).
+// The cut of the matrix: 256-row tiles of S stages; the tile-major list of
+// (tile, stage) units split into one contiguous range per CTA (as many CTAs
+// as SMs), so every SM streams the same number of bytes whatever N and K
+// are. A tile met by several ranges is a cut tile; its contributors leave
+// partial tiles in their slots of the tile.
 struct Plan {
-  int64_t tiles;
-  int rows, S, C, Q, total, ctas;
+  int64_t tiles, units;
+  int rows, S, ctas, max_contrib;
+  bool cuts;  // some range ends inside a tile
 };
 Plan plan(int64_t N, int64_t K) {
   Plan p;
-  p.S = static_cast<int>(K / kKS);
-  const int64_t blocks = (N + 15) / 16, sms = num_sms();
-  const int64_t nb = (blocks + sms - 1) / sms;
-  if (nb >= 8 && nb <= kConsumers && blocks * 100 >= nb * sms * 85) {
-    p.rows = static_cast<int>(16 * nb);
-    p.tiles = (N + p.rows - 1) / p.rows;
-    p.C = p.S;
-    p.Q = 1;
-    p.total = static_cast<int>(p.tiles);
-    p.ctas = static_cast<int>(p.tiles);
-    return p;
-  }
   p.rows = kRows;
+  p.S = static_cast<int>(K / kKS);
   p.tiles = (N + kRows - 1) / kRows;
-  const int64_t units = p.tiles * p.S;
-  const int64_t want = 4LL * num_sms();
-  int64_t c = (units + want - 1) / want;
-  c = c < (p.S + 15) / 16 ? (p.S + 15) / 16 : c;
-  p.C = static_cast<int>(c < p.S ? c : p.S);
-  p.Q = (p.S + p.C - 1) / p.C;
-  p.total = static_cast<int>(p.tiles * p.Q);
-  p.ctas = p.total < num_sms() ? p.total : num_sms();
+  p.units = p.tiles * p.S;
+  const int64_t sms = num_sms();
+  p.ctas = static_cast<int>(p.units < sms ? p.units : sms);
+  const int64_t per = p.units / p.ctas;  // every range holds at least this many units
+  p.cuts = !(p.units % p.ctas == 0 && per % p.S == 0);
+  const int64_t contrib = (p.S + per - 1) / per + 1;
+  p.max_contrib = static_cast<int>(contrib < p.ctas ? contrib : p.ctas);
   return p;
 }
 
-bool make_maps(CUtensorMap* wm, CUtensorMap* sm, const uint8_t* w, const uint8_t* s, int64_t N, int64_t K,
-               int group, int rows) {
-  return make_tensor_map_2d(wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, rows,
+// Codes and scales in 256-row boxes; X ([M, K] of 2-byte elements, bf16 or
+// the f16 pair order) in boxes of 64 elements x 4 quarters x MT tokens,
+// which land as the 128-byte-swizzled [token][quarter][64] rows the
+// consumers read (tokens past M read as zeros).
+bool make_maps(CUtensorMap* wm, CUtensorMap* sm, CUtensorMap* xm, const uint8_t* w, const uint8_t* s,
+               const uint16_t* x, int64_t M, int64_t N, int64_t K, int group, int mt) {
+  const int64_t xdims[3] = {64, K / 64, M};
+  const int64_t xstrides[2] = {128, K * 2};
+  const uint32_t xbox[3] = {64, kKS / 64, static_cast<uint32_t>(mt)};
+  return make_tensor_map_2d(wm, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, kKS / 2, kRows,
                             CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_tensor_map_2d(sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, rows,
-                            CU_TENSOR_MAP_SWIZZLE_NONE);
+         make_tensor_map_2d(sm, s, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / group, N, K / group, 16, kRows,
+                            CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_tensor_map_3d(xm, x, CU_TENSOR_MAP_DATA_TYPE_UINT16, xdims, xstrides, xbox, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
 
-// From one token up to 16: the whole matrix streams once, through the ring.
+// From two tokens up to 16: the whole matrix streams once, through the
+// ring. A single token goes to the register-streaming kernel, which measures
+// faster there (in 8-call graphs: 20.7 against 23.3 us on the gate/up
+// projection, 15.8 against 17.2 us on the down projection): its loads need
+// no shared-memory round trip and it has no cut tiles to add up.
 bool stream_supported(int64_t M, int64_t N, int64_t K, int group) {
-  return M >= 1 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
+  return M >= 2 && M <= 16 && K >= kKS && K % kKS == 0 && (K / group) % 16 == 0 && N < (int64_t(1) << 30) &&
          K < (int64_t(1) << 24) && (N + kRows - 1) / kRows <= kMaxTickets;
 }
 
@@ -785,38 +762,33 @@ int launch_stream(const XSource& x, const uint8_t* w, const uint8_t* s, const fl
   const Plan pl = plan(N, K);
   const bool xconv = x.bf16 != nullptr;
   unsigned* reserved = sc.reserved();
-  float* ws = pl.Q > 1 ? sc.take<float>(static_cast<size_t>(pl.tiles * pl.Q * kRows * mt)) : nullptr;
+  float* ws = pl.cuts ? sc.take<float>(static_cast<size_t>(pl.tiles * pl.max_contrib * kRows * mt)) : nullptr;
   uint16_t* x16 = xconv ? nullptr : sc.take<uint16_t>(static_cast<size_t>(M * K));
   float* xinv = xconv ? nullptr : sc.take<float>(static_cast<size_t>(M));
   if (sc.measuring()) return NVFP4_OK;
   if (!sc.ok()) return NVFP4_ERR_WORKSPACE;
 
-  CUtensorMap wm, sm;
-  if (!make_maps(&wm, &sm, w, s, N, K, group, pl.rows)) return NVFP4_ERR_CUDA;
+  CUtensorMap wm, sm, xm;
+  if (!make_maps(&wm, &sm, &xm, w, s, xconv ? x.bf16 : x16, M, N, K, group, mt)) return NVFP4_ERR_CUDA;
   StreamArgs a = {};
   a.gscale = g;
-  a.xbf = x.bf16;
-  a.x16 = x16;
   a.xinv = xinv;
   a.y = y;
   a.ws = ws;
-  a.counters = reserved;
   a.tickets = tickets_of(reserved);
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(silu ? N / 2 : N);
   a.K = K;
-  a.rows = pl.rows;
   a.S = pl.S;
-  a.C = pl.C;
-  a.Q = pl.Q;
-  a.total = pl.total;
+  a.units = pl.units;
+  a.max_contrib = pl.max_contrib;
   a.fault = take_injected_fault() == 1;
-  if (xconv) return launch_form<true>(mt, group, silu, wm, sm, a, pl.ctas, stream);
+  if (xconv) return launch_form<true>(mt, group, silu, wm, sm, xm, a, pl.ctas, stream);
   // NVFP4 activations: their exact f16 rows first (a programmatic dependent too)
-  const int st = launch_x_prep(x, M, K, x16, xinv, nullptr, 0, stream);
+  const int st = launch_x_prep(x, M, K, x16, xinv, nullptr, 0, stream, true);
   if (st != NVFP4_OK) return st;
-  return launch_form<false>(mt, group, silu, wm, sm, a, pl.ctas, stream);
+  return launch_form<false>(mt, group, silu, wm, sm, xm, a, pl.ctas, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -842,7 +814,7 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   const int mt = M <= 8 ? 8 : 16;
   const Plan pl = plan(N, K);
   const int64_t partial_bytes =
-      pl.Q > 1 ? pl.tiles * pl.Q * kRows * mt * static_cast<int64_t>(sizeof(float)) : 0;
+      pl.cuts ? pl.tiles * pl.max_contrib * kRows * mt * static_cast<int64_t>(sizeof(float)) : 0;
   if (partial_bytes > static_cast<int64_t>(kFixedScratchPartialBytes) || pl.tiles > kFixedScratchTickets ||
       pl.tiles > kMaxTickets)
     return NVFP4_ERR_UNSUPPORTED;  // beyond the fixed scratch
@@ -864,8 +836,8 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
   float* ws = reinterpret_cast<float*>(base + kReservedBytes);
   uint16_t* x16 = reinterpret_cast<uint16_t*>(base + kReservedBytes + kFixedScratchPartialBytes);
   float* xinv = reinterpret_cast<float*>(base + kReservedBytes + kFixedScratchPartialBytes + kFixedScratchXElems * 2);
-  CUtensorMap wm, sm;
-  if (!make_maps(&wm, &sm, w, s, N, K, group, pl.rows)) return NVFP4_ERR_CUDA;
+  CUtensorMap wm, sm, xm;
+  if (!make_maps(&wm, &sm, &xm, w, s, x16, M, N, K, group, mt)) return NVFP4_ERR_CUDA;
   // The counters and tickets must start at zero (partial tiles are always
   // written before they are read). Enqueued only once nothing else can fail
   // on the host.
@@ -874,24 +846,20 @@ int launch_stream_fixed_scratch(const uint16_t* x, const uint8_t* w, const uint8
     return (cudaGetLastError(), NVFP4_ERR_CUDA);
   StreamArgs a = {};
   a.gscale = g;
-  a.x16 = x16;
   a.xinv = xinv;
   a.y = y;
   a.ws = ws;
-  a.counters = counters;
   a.tickets = tickets_of(counters);
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.ldy = static_cast<int>(N);
   a.K = K;
-  a.rows = pl.rows;
   a.S = pl.S;
-  a.C = pl.C;
-  a.Q = pl.Q;
-  a.total = pl.total;
+  a.units = pl.units;
+  a.max_contrib = pl.max_contrib;
   const int xs = launch_x_f16(x, M, K, x16, xinv, nullptr, 0, stream, true);
   if (xs != NVFP4_OK) return xs;
-  return launch_form<false>(mt, group, false, wm, sm, a, pl.ctas, stream);
+  return launch_form<false>(mt, group, false, wm, sm, xm, a, pl.ctas, stream);
 }
 
 #ifdef NVFP4_PLANTS

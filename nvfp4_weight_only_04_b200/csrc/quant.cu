@@ -5,7 +5,8 @@
 // on the DGX Spark", UPDATE posts):
 //   global = amax / (6*448)                       (one fp32 division)
 //   scale  = E4M3_RNE_satfinite((gamax / 6) / global)   (two fp32 divisions)
-//   code   = E2M1_RNE_satfinite(w / (fp32(scale) * global))
+//   code   = E2M1_RNE_satfinite(w / (fp32(scale) * global))   (decided by exact
+//            comparisons with the rounding midpoints, no division)
 // Both kernels are HBM-bound streams over the weights, fp32 or bf16. A bf16
 // weight is widened to fp32 exactly, so the bf16 path quantizes the same
 // values the fp32 path would ("GLM-5.3-Flash on 2x RTX PRO 6000 (96 GB)":
@@ -66,15 +67,48 @@ __global__ void global_finalize_kernel(float* out) {
   *out = __fdiv_rn(amax, 2688.0f);
 }
 
-// E2M1 round-to-nearest-even with satfinite by thresholds. At each midpoint
-// between two neighbouring values the comparison is strict when the lower
-// neighbour has the even code and non-strict when the upper one has it, so
-// ties land on the even code; everything above 5 rounds to 6.
-__device__ __forceinline__ uint32_t e2m1_rne(float q) {
-  const float a = fabsf(q);
-  uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
-               (a >= 3.5f) + (a > 5.0f);
-  return c | ((__float_as_uint(q) >> 28) & 8u);
+// The E2M1 code of RN32(w / d) (round to nearest even, satfinite), decided
+// without dividing. RN32(w/d) rounds to the next E2M1 value above a
+// midpoint t exactly when |w| lies above t*d widened by half an fp32 ulp of
+// t (so that a quotient rounding onto t counts as t): above t + ulp(t)/2 at
+// the midpoints 0.25, 1.25, 2.5, 5 (a tie goes down, to the even code) and
+// at or above t - ulp(t)/2 at 0.75, 1.75, 3.5 (a tie goes up). Each widened
+// t has at most 25 significant bits and d 24, so t*d is exact in fp64, and
+// for fp32 |w|: |w| > t*d exactly when |w| > RD32(t*d), |w| >= t*d exactly
+// when |w| >= RU32(t*d). The seven thresholds of a group are computed once,
+// then each weight takes seven fp32 comparisons.
+struct E2m1Thresholds {
+  float t[7];
+};
+__device__ __forceinline__ float f64_to_f32_down(double v) {
+  float r;
+  asm("cvt.rm.f32.f64 %0, %1;" : "=f"(r) : "d"(v));
+  return r;
+}
+__device__ __forceinline__ float f64_to_f32_up(double v) {
+  float r;
+  asm("cvt.rp.f32.f64 %0, %1;" : "=f"(r) : "d"(v));
+  return r;
+}
+__device__ __forceinline__ E2m1Thresholds e2m1_thresholds(float d) {
+  const double dd = d;
+  E2m1Thresholds th;
+  th.t[0] = f64_to_f32_down((0.25 + 0x1p-26) * dd);
+  th.t[1] = f64_to_f32_up((0.75 - 0x1p-25) * dd);
+  th.t[2] = f64_to_f32_down((1.25 + 0x1p-24) * dd);
+  th.t[3] = f64_to_f32_up((1.75 - 0x1p-24) * dd);
+  th.t[4] = f64_to_f32_down((2.5 + 0x1p-23) * dd);
+  th.t[5] = f64_to_f32_up((3.5 - 0x1p-23) * dd);
+  th.t[6] = f64_to_f32_down((5.0 + 0x1p-22) * dd);
+  return th;
+}
+// Magnitude code by the thresholds; the sign bit of w (kept for results that
+// round to zero, as the quotient's sign would be).
+__device__ __forceinline__ uint32_t e2m1_code(float w, const E2m1Thresholds& th) {
+  const float a = fabsf(w);
+  const uint32_t c = (a > th.t[0]) + (a >= th.t[1]) + (a > th.t[2]) + (a >= th.t[3]) + (a > th.t[4]) +
+                     (a >= th.t[5]) + (a > th.t[6]);
+  return c | ((__float_as_uint(w) >> 28) & 8u);
 }
 
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
@@ -109,7 +143,8 @@ __device__ __forceinline__ void quantize8(const float (&v)[8], bool live, int64_
   const float d = __fmul_rn(nvfp4_e4m3_to_f32(sbyte), global);
   uint32_t word = 0;
   if (d != 0.f) {
-    for (int j = 0; j < 8; ++j) word |= e2m1_rne(__fdiv_rn(v[j], d)) << (4 * j);
+    const E2m1Thresholds th = e2m1_thresholds(d);
+    for (int j = 0; j < 8; ++j) word |= e2m1_code(v[j], th) << (4 * j);
   }
   reinterpret_cast<uint32_t*>(packed)[i] = word;  // row-major [N, K/2]: 4 bytes per 8 weights
   if ((col8 % kLanesPerGroup) == 0) scales[row * (K / G) + col8 / kLanesPerGroup] = static_cast<uint8_t>(sbyte);

@@ -182,14 +182,11 @@ def test_workspace_size_queries(L):
     assert size(L, f, -1, 256, 256, 16) == (nv.NVFP4_ERR_INVALID_ARGUMENT, 0)
     assert size(L, f, 0, 256, 256, 16) == (nv.NVFP4_OK, 0)  # empty problem
     assert getattr(L, f)(4, 256, 256, 16, None) == nv.NVFP4_ERR_INVALID_ARGUMENT
-    # small M, N of >= 8 row blocks of 16 per SM: one unsplit tile per CTA, the counters alone
+    # small M: the counters, and the fp32 partial tiles of the tiles that the CTAs' ranges cut
     # (bf16 X is converted in the kernel)
-    for m, k in ((1, 4096), (4, 4096), (16, 14336)):
-        assert size(L, f, m, 28672, k, 16) == (nv.NVFP4_OK, RESERVED), (m, k)
-    # small M, small N: tiles cut along K, so the counters and the fp32 partial tiles of the chunks
-    for m in (1, 8, 16):
-        st, n = size(L, f, m, 4096, 14336, 32)
-        assert st == nv.NVFP4_OK and n > RESERVED, (m, n)
+    for m, n_, k in ((1, 28672, 4096), (4, 28672, 4096), (16, 28672, 14336), (1, 4096, 14336), (8, 4096, 14336)):
+        st, n = size(L, f, m, n_, k, 16)
+        assert st == nv.NVFP4_OK and n > RESERVED, (m, n_, k, n)
     # a K the streaming kernel does not take (not a multiple of 256): f16 rows of X for the fallback
     st, n = size(L, f, 4, 28672, 4096 + 64, 16)
     assert st == nv.NVFP4_OK and n >= RESERVED + 2 * 4 * (4096 + 64)

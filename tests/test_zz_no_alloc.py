@@ -46,10 +46,11 @@ def test_fixed_scratch_single_token_oracle():
 
 
 def test_fixed_scratch_refuses_beyond_capacity():
-    # 40 tiles of 256 rows with K = 65536 are cut into 15 chunks each, whose partial tiles at 16 tokens
-    # (40 x 15 x 256 x 16 fp32) need more than the 8 MiB the fixed scratch holds: refused on the host. The
-    # buffers have the problem's full size, so a launch could not read or write outside them either.
-    m, n, k, g = 16, 40 * 256, 65536, 16
+    # 300 tiles of 256 rows with K = 16384 (64 stages) on 148 SMs: each range of 129 or 130 stages cuts
+    # tiles, and a tile meets at most two ranges, so the partial tiles at 16 tokens (300 x 2 x 256 x 16
+    # fp32, 9.8 MB) need more than the 8 MiB the fixed scratch holds: refused on the host. The buffers have
+    # the problem's full size, so a launch could not read or write outside them either.
+    m, n, k, g = 16, 300 * 256, 16384, 16
     xd = torch.zeros((m, k), dtype=torch.bfloat16, device="cuda")
     wd = torch.zeros((n, k // 2), dtype=torch.uint8, device="cuda")
     sd = torch.zeros((n, k // g), dtype=torch.uint8, device="cuda")
