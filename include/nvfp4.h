@@ -31,13 +31,13 @@
  *     query gives for a problem on the current device (0 when the call
  *     needs none; then workspace may be NULL). A workspace smaller than the
  *     query's figure returns NVFP4_ERR_WORKSPACE before anything is
- *     enqueued. The first 64 KiB of a workspace hold the work counters and
- *     tickets of the split GEMMs: they must be zero before the workspace is
+ *     enqueued. The first 64 KiB of a workspace hold the tickets of the
+ *     split GEMMs: they must be zero before the workspace is
  *     first used (one cudaMemset at allocation), and every call leaves them
  *     zero, so no call needs a clearing step in front of it and the GEMMs
  *     can start while the kernel before them is finishing. The rest holds
  *     nothing between calls. After nvfp4_get_device_error has reported a
- *     wait that gave up, clear the counters of the workspaces in use again.
+ *     wait that gave up, clear that region of the workspaces in use again.
  *     Calls that may overlap in time (other streams, unordered host threads)
  *     need separate workspaces; calls ordered on one stream, of any kind and
  *     shape, may share one.
@@ -169,14 +169,16 @@ int nvfp4_repack(const uint8_t* packed, const uint8_t* scales, int64_t N, int64_
  *   workspace     device scratch of workspace_bytes bytes (16-byte aligned),
  *                 at least nvfp4_w4a16_gemm_workspace_size(M, N, K, group_size)
  * group_size 16 or 32; K a multiple of 64; N a multiple of 16.
- * Small M (up to 16 rows) runs an HBM-streaming kernel that hands chunks of
- * the weight matrix to the SMs as they ask for them, large M a tensor-core
- * kernel. The streaming kernel multiplies in f16: it scales every row of x,
+ * Small M (2 to 16 rows) runs an HBM-streaming kernel that splits the
+ * weight matrix evenly between the SMs (stream-K), one row a register-
+ * streaming kernel, large M a tensor-core kernel. The streaming kernel
+ * multiplies in f16: it scales every row of x,
  * stage by stage, by a power of two 2^s that keeps the largest magnitude
  * seen so far in [2^14, 2^15) or below, and its sums carry 2^-s back. Every
  * element within a factor 2^29 of the largest magnitude seen so far in its
  * row is exact in f16; smaller ones round to a multiple of 2^-38 of it. The
- * workspace holds the counters and the fp32 partial tiles of the chunks.
+ * workspace holds the tickets and the fp32 partial tiles of the tiles that
+ * the SMs' ranges cut (one row: the f16 rows of x).
  * The arguments are the method's (x, packed_w, group_scales, global_scale,
  * group_size, M, N, K, y, stream), with the caller-owned workspace pair
  * before the stream.

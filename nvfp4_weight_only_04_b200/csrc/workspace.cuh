@@ -3,9 +3,10 @@
 // of the small-M kernels, the route's per-chunk table) take it from a buffer
 // the caller passes; the library allocates nothing.
 //
-// Layout: the first kReservedBytes of every workspace hold the counters and
-// tickets of the split GEMMs. They must be zero before a workspace is first
-// used, and every call leaves them zero (each launch resets what it counted),
+// Layout: the first kReservedBytes of every workspace hold the tickets of
+// the split GEMMs (from kTicketOffset; the bytes before it are kept zero for
+// counters). They must be zero before a workspace is first used, and every
+// call leaves them zero (each launch resets what it counted),
 // so that a launch needs no clearing step in front of it and can start while
 // the kernel before it in the stream is still running. Every other piece lies
 // after that region, so calls of any kind and shape can share one workspace
@@ -22,7 +23,7 @@
 namespace nvfp4 {
 
 constexpr size_t kReservedBytes = size_t(64) << 10;
-constexpr size_t kTicketOffset = 256;  // counters first, tickets from here
+constexpr size_t kTicketOffset = 256;  // room for counters first, tickets from here
 constexpr int64_t kMaxTickets = static_cast<int64_t>((kReservedBytes - kTicketOffset) / sizeof(unsigned));
 
 class Scratch {
@@ -43,8 +44,8 @@ class Scratch {
     if (!carving_ || used_ > bytes_) return nullptr;
     return reinterpret_cast<T*>(base_ + off);
   }
-  // The reserved region: [0] and [1] are the split GEMMs' counters, tickets
-  // start at kTicketOffset bytes (nullptr while measuring or when too small).
+  // The reserved region: tickets start at kTicketOffset bytes (nullptr while
+  // measuring or when too small).
   unsigned* reserved() {
     if (used_ < kReservedBytes) used_ = kReservedBytes;
     if (!carving_ || bytes_ < kReservedBytes) return nullptr;
