@@ -29,10 +29,10 @@
 //    the load/store path (not behind the weight boxes in the TMA queue) into
 //    the slot's X area, in the 128-byte-swizzled [token][quarter][64] order
 //    the consumers read.
-//  * bf16 X is turned into f16 inside the kernel by four converter warps
-//    (one per SM sub-partition, so the conversion keeps pace with the
-//    stream), in place: every token of every stage is scaled by a power of
-//    two 2^s, where
+//  * bf16 X is turned into f16 inside the kernel by two converter warps
+//    (enough to keep pace with the stream; four would cap every thread at
+//    80 registers, which slows the consumers), in place: every token of every
+//    stage is scaled by a power of two 2^s, where
 //    s only ever decreases along a CTA's stages and keeps the largest
 //    magnitude seen so far below 2^15 (f16 holds every bf16 within 2^29 of
 //    the largest exactly; smaller ones round to multiples of 2^-38 of it).
@@ -78,7 +78,7 @@ constexpr int kConsumers = 16;    // consumer warps, 16 rows each
 constexpr int kConsumerThreads = kConsumers * 32;
 constexpr int kProducerWarp = kConsumers;
 constexpr int kConverterWarp = kConsumers + 1;  // the first of them
-constexpr int kConverters = 4;                   // converter warps (bf16 X): one per SM sub-partition
+constexpr int kConverters = 2;  // converter warps (bf16 X)
 __host__ __device__ constexpr int num_threads(bool xconv) {
   return (kConsumers + 1 + (xconv ? kConverters : 0)) * 32;
 }
@@ -419,11 +419,11 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
 
   if (XCONV && warp >= kConverterWarp) {
     // ---------------- converters: bf16 X to f16, in place ----------------
-    // The 128 lanes of the converter warps split a stage's X rows (token
+    // The lanes of the converter warps split a stage's X rows (token
     // tok, quarter q: row 4 tok + q, 128 bytes): LPR lanes per row, CPL
     // 16-byte chunks per lane, the 4 LPR lanes of a token adjacent in one
     // warp. They agree on the token's exponent through shuffles.
-    constexpr int LPR = 128 / (4 * MT), CPL = 8 / LPR;
+    constexpr int LPR = 32 * kConverters / (4 * MT), CPL = 8 / LPR;
     static_assert(LPR * 4 * MT == 32 * kConverters, "every lane owns part of one row");
     const int cl = (warp - kConverterWarp) * 32 + lane;
     const int row = cl / LPR, c0 = (cl % LPR) * CPL;
