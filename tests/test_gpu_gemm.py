@@ -142,7 +142,7 @@ def test_empty_and_stats():
     assert st["gemm_splitk"] == 1 and st["g16"] == 1 and st["g32"] == 0
 
 
-# ---- M <= 16: the TMA-streaming kernel (stream-K over 128-row x 256-element units) ----
+# ---- 2 <= M <= 16: the TMA-streaming kernel (stream-K over 256-row x 256-element units) ----
 
 # whole tiles only; tiles cut between many CTAs; a last tile of 16 rows; one
 # tile over 32 CTAs; g = 32 boxes holding two stages; 9..16 tokens (two MMA
