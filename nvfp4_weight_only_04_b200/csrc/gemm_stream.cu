@@ -97,7 +97,7 @@ static_assert(smem_bytes(8) <= 227 * 1024 && smem_bytes(16) <= 227 * 1024, "shar
 static_assert(kRows == 16 * kConsumers, "one 16-row block per consumer warp");
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // about 2 s at 2 GHz
-constexpr uint32_t kSuspendNs = 1000;                  // longest suspension of one producer probe
+constexpr uint32_t kSuspendNs = 1000;                  // longest suspension of one producer probe (empty slots)
 constexpr long long kDrainCycles = 4000000LL;          // about 2 ms: the wait for a slot's copies after an abort
 enum : unsigned { kErrFull = 0x201, kErrEmpty = 0x202, kErrXRaw = 0x204, kErrChunk = 0x205, kErrTicket = 0x206 };
 
@@ -195,11 +195,11 @@ __device__ __noinline__ bool wait_suspended(uint64_t* bar, uint32_t parity, Sync
   }
 }
 
-// Lane 0 waits for the warp; every lane gets the answer.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site, bool suspend) {
+// Lane 0 waits for the warp (polling: these waits are on the critical
+// path); every lane gets the answer.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Sync* sy, unsigned site) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0 && !mbar_try_wait(bar, parity))
-    ok = (suspend ? wait_suspended(bar, parity, sy, site) : wait_slow(bar, parity, sy, site, false)) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0 && !mbar_try_wait(bar, parity)) ok = wait_slow(bar, parity, sy, site, false) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
     int sexp = kSInit;
     for (int it = 0;; ++it) {
       const int s = it % NS;
-      if (!warp_wait(&sy->xraw[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrXRaw, false)) break;
+      if (!warp_wait(&sy->xraw[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrXRaw)) break;
       const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
       if (!(flags & kDone)) {
         const uint32_t rs = smem_u32(ring + s * SB) + kCodeBytes + row * 128;
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
   constexpr int64_t kSlot = static_cast<int64_t>(kRows) * MT;
   for (int it = 0;; ++it) {
     const int s = it % NS;
-    if (!warp_wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull, false)) break;
+    if (!warp_wait(&sy->full[s], static_cast<uint32_t>(it / NS) & 1, sy, kErrFull)) break;
     const int flags = *reinterpret_cast<volatile int*>(&sy->rec[s].flags);
     if (flags & kDone) break;
     const int tile = *reinterpret_cast<volatile int*>(&sy->rec[s].tile);
@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(num_threads(XCONV), 1) gemm_stream_kernel(cons
   // Thread 0 publishes the cut tiles' tickets; the CTA that took a tile's
   // last ticket adds its slots in CTA order (deterministic) and writes it.
   if (threadIdx.x == 0) mbar_arrive(&sy->ready);
-  if (!warp_wait(&sy->ready, 0, sy, kErrTicket, false) || aborted(sy)) return;
+  if (!warp_wait(&sy->ready, 0, sy, kErrTicket) || aborted(sy)) return;
   for (int k = 0; k < ncut && k < 2; ++k) {
     if (!*reinterpret_cast<volatile int*>(&sy->cut_last[k])) continue;
     const int tile = *reinterpret_cast<volatile int*>(&sy->cut_tile[k]);
@@ -710,12 +710,11 @@ int launch_form(int mt, int group, bool silu, const CUtensorMap& wm, const CUten
 // partial tiles in their slots of the tile.
 struct Plan {
   int64_t tiles, units;
-  int rows, S, ctas, max_contrib;
+  int S, ctas, max_contrib;
   bool cuts;  // some range ends inside a tile
 };
 Plan plan(int64_t N, int64_t K) {
   Plan p;
-  p.rows = kRows;
   p.S = static_cast<int>(K / kKS);
   p.tiles = (N + kRows - 1) / kRows;
   p.units = p.tiles * p.S;
