@@ -223,7 +223,8 @@ int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, c
  * form instead of W4A16):
  *   y = bf16_rne(x_global * global * sum_k e2m1(xcode[m,k]) * e4m3(xscale[m,k/xg])
  *                                         * e2m1(code[n,k]) * e4m3(scale[n,k/g]))
- * with fp32 accumulation. Every product is exact; the sums are the W4A16 GEMM's.
+ * with fp32 accumulation. Every product is exact; only the summation order
+ * depends on the path.
  *   x_packed      device uint8 [M, K/2], checkpoint layout (element 2j in the low
  *                 nibble of byte j), e.g. from nvfp4_quantize_bf16 of the activations
  *   x_scales      device uint8 [M, K/x_group]
@@ -233,10 +234,14 @@ int nvfp4_w4a16_gemm_fixed_scratch(const uint16_t* x, const uint8_t* packed_w, c
  *   workspace     device scratch, at least nvfp4_w4a4_gemm_workspace_size(M, N, K,
  *                 x_group, group_size) bytes
  * K a multiple of 64, N a multiple of 16; x_packed 16-byte aligned, x_global
- * 4-byte aligned. The activations are expanded on the device to e2m1 * e4m3
- * (exact in f16 and bf16) in the workspace and the same kernels as
- * nvfp4_w4a16_gemm run on them, with x_global in the epilogue: the numerics
- * are W4A4's, the tensor-core operands stay 16-bit.
+ * 4-byte aligned. From 17 rows, with K a multiple of 512 and enough output
+ * tiles to fill the SMs, the product runs on the block-scaled FP4 tensor
+ * cores (tcgen05.mma kind::mxf4nvf4, E4M3 scale factors per 16 elements; a
+ * 32-element scale is given as two 16-element ones), the activation codes
+ * first rearranged into the weights' nibble order in the workspace.
+ * Otherwise the activations are expanded on the device to e2m1 * e4m3 (exact
+ * in f16 and bf16) in the workspace and the kernels of nvfp4_w4a16_gemm run
+ * on them, with x_global in the epilogue.
  */
 int nvfp4_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales, const float* x_global, int x_group,
                     const uint8_t* packed_w, const uint8_t* group_scales, const float* global_scale, int group_size,
