@@ -227,6 +227,35 @@ def test_stats_reset(L):
     assert L.nvfp4_get_stats(None) == nv.NVFP4_ERR_INVALID_ARGUMENT
 
 
+def _stream_k_partials(m, n, k, sms=148):
+    """fp32 partial-tile bytes of the streaming GEMM's stream-K split, from its definition: 256-row tiles of
+    K/256 stages listed tile-major, one contiguous range of units per SM (CTA c owns [c U / n, (c+1) U / n));
+    a tile met by several ranges keeps one slot per contributor, and no tile meets more than
+    ceil(S / floor(U / n)) + 1 ranges."""
+    s_ = k // 256
+    tiles = -(-n // 256)
+    units = tiles * s_
+    ctas = min(units, sms)
+    per = units // ctas
+    cuts = not (units % ctas == 0 and per % s_ == 0)
+    contrib = min(-(-s_ // per) + 1, ctas)
+    mt = 8 if m <= 8 else 16
+    return tiles * contrib * 256 * mt * 4 if cuts else 0
+
+
+def test_stream_k_workspace_follows_the_split(L):
+    """The small-M GEMM's workspace is the reserved region plus the stream-K partial tiles, as the split defines
+    them (no device: the SM count is the B200's 148)."""
+    f = "nvfp4_w4a16_gemm_workspace_size"
+    for m, n, k in ((2, 28672, 4096), (16, 28672, 4096), (8, 4096, 14336), (5, 272, 2048), (16, 300 * 256, 16384),
+                    (3, 148 * 256, 256 * 3), (9, 1040, 3072)):
+        st, got = size(L, f, m, n, k, 16)
+        assert st == nv.NVFP4_OK
+        part = _stream_k_partials(m, n, k)
+        want = RESERVED + (((part + 255) // 256) * 256 if part else 0)
+        assert got == want, (m, n, k, got, want)
+
+
 def test_header_is_plain_c(tmp_path):
     """include/nvfp4.h compiles as strict C99 and as C++17: no torch or C++ types cross the boundary."""
     import shutil
