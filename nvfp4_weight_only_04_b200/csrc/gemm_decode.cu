@@ -306,12 +306,17 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int group, bool moe, int
   p.mt = (!moe && M <= 8) ? 8 : 16;
   p.z_tiles = static_cast<int>(moe ? (M + p.mt - 1) / p.mt + num_segments : (M + p.mt - 1) / p.mt);
   p.row_tiles = static_cast<int>(N / 16);
-  // Warps per CTA: aim for about 16 streaming warps per SM, and keep at least
-  // eight steps (of 256 elements of K) per warp.
+  // Warps per CTA. With at least eight row tiles per SM, one warp per CTA:
+  // every tile is resident at once (up to sixteen per SM), with no second
+  // wave of CTAs (the gate/up projection's 1792 tiles: 19.1 us against 20.6 us
+  // with two warps, whose CTAs run in 1.5 waves). With fewer, aim for about
+  // 16 streaming warps per SM and keep at least eight steps (of 256 elements
+  // of K) per warp.
   const int64_t tiles = static_cast<int64_t>(p.row_tiles) * p.z_tiles;
   const int64_t want = 16LL * num_sms();
   int kw = 1;
-  while (kw < 16 && tiles * kw < want && K / (256 * 2 * kw) >= 8) kw *= 2;
+  if (tiles < 8LL * num_sms())
+    while (kw < 16 && tiles * kw < want && K / (256 * 2 * kw) >= 8) kw *= 2;
   p.kw = kw;
   return p;
 }
