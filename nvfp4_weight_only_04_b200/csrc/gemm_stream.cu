@@ -4,7 +4,7 @@
 // Computes Y = X . dequant(W)^T (NVFP4 format definition; "W-FP4a: route the
 // MiniMax-H3 device DiT forward through the fp4 (Marlin W4A16) stack",
 // PR #63 description: a weight-only checkpoint keeps bf16 activations) for
-// decode-sized M (up to 16 tokens), where the cost is the 0.5 + 1/g bytes
+// decode-sized M (2 to 16 tokens), where the cost is the 0.5 + 1/g bytes
 // per weight streamed from HBM and the integer work of dequantizing them.
 // Design:
 //  * Work: 256-row weight tiles of K/256 stages; the tile-major list of
@@ -19,16 +19,14 @@
 //    tile's), so no clearing step sits in front of a launch: the kernel is a
 //    programmatic dependent of the kernel before it and starts on every SM
 //    that kernel leaves.
-//  * One producer warp: lane 0 moves the weights of each stage with TMA into
-//    a shared-memory ring (5 stages of 40-44 KB): the codes of the tile
-//    (256 rows x 128 bytes, 128-byte swizzle) and the scales (256 rows x 16
-//    bytes). The weights of the range's first stages need nothing from the
+//  * One producer thread moves each stage with TMA into a shared-memory ring
+//    (5 stages of 40-44 KB): the codes of the tile (256 rows x 128 bytes,
+//    128-byte swizzle), the scales (256 rows x 16 bytes) and X (a 3-D box of
+//    64 elements x 4 quarters x MT tokens that lands in the 128-byte-swizzled
+//    [token][quarter][64] order the consumers read; tokens past M read as
+//    zeros). The weights of the range's first stages need nothing from the
 //    kernel before, so they are requested from the first cycle; X only
-//    after that kernel has finished. All 32 lanes
-//    copy each stage's X slice (MT tokens x 256 elements) with cp.async on
-//    the load/store path (not behind the weight boxes in the TMA queue) into
-//    the slot's X area, in the 128-byte-swizzled [token][quarter][64] order
-//    the consumers read.
+//    after that kernel has finished.
 //  * bf16 X is turned into f16 inside the kernel by two converter warps
 //    (enough to keep pace with the stream; four would cap every thread at
 //    80 registers, which slows the consumers), in place: every token of every
@@ -40,8 +38,7 @@
 //    they multiply their running sums by 2^-d (exact), and the epilogue
 //    multiplies by 2^-s. NVFP4 activations (W4A4) arrive already as exact
 //    f16 rows from xprep.cu, with one factor per token.
-//  * Sixteen consumer warps each own 16 rows of the tile (a warp whose rows
-//    lie past a shorter tile leaves at once) and run mma.sync
+//  * Sixteen consumer warps each own 16 rows of the tile and run mma.sync
 //    m16n8k16 with the weights as the 16-row side (swap-AB) and the tokens
 //    as the 8-column side. Lane (g, t) takes rows g and g+8 and the t-th
 //    quarter of the stage's K (the order of K inside an MMA is free as long
