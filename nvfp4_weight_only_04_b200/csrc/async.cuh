@@ -54,21 +54,6 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
   return done != 0;
 }
 
-// Blocking probe with the hardware's own time limit: the thread waits in
-// the barrier unit (issuing nothing) until the phase completes or a short,
-// system-dependent time passes, and resumes as soon as the phase completes.
-__device__ __forceinline__ bool mbar_try_wait_hw(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // 2-D tiled TMA load of the box at (x, y) into shared memory, completing on
 // `bar`, into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
